@@ -1,0 +1,434 @@
+#!/usr/bin/env python
+"""Benchmark of the E8 quantize path on B200.
+
+One step = one pass of the whole path over the dense-MLP workload
+(up 4096x14336 and down 14336x4096 bf16 latent weights, N(0, 0.015^2)):
+  1. QAT forward: one e8q_project_encode launch over both matrices --
+     sign flip, blockwise RHT (B = 2048), row scale, E8 projection, core
+     index, ordered escape / overflow records with CSR, and the
+     original-basis bf16 dequantised weights (identity-STE forward);
+  2. STE backward: the upstream gradient is passed to the latents as is
+     (an alias, no kernel);
+  3. decode: e8q_dequant_gemv of the encoded up matrix at batch 1, 4, 16
+     and 64 (bf16 activations N(0, 1)).
+value = groups encoded per second over whole steps (Ggroups/s, all ranks).
+Inputs are larger than L2 (235 MB read per step), so no flush is needed.
+
+--impl reference runs the fp64 CPU oracle on a bounded sample of the same
+step on the host cores (rank 0 only).
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+
+METRIC = "E8 project+encode Ggroups/s and dequant-GEMV GB/s, % of B200 HBM peak"
+UNIT = "Ggroups/s"
+WORKLOAD = ("mlp_14336 QAT step: project+encode+STE-dequant of up 4096x14336 and down 14336x4096 bf16 "
+            "(one launch), identity-STE backward, then 2-bit dequant-GEMV of up at batch 1,4,16,64")
+D_MODEL, D_FF = 4096, 14336
+NOMINAL_HBM_GBS = 8000.0
+KERNEL_SOURCES = ["bit_e8_lattice_b200/csrc/" + f for f in
+                  ("e8q.cu", "encode.cuh", "lattice.cuh", "common.cuh", "gemv.cuh", "decode.cuh", "tables.cpp",
+                   "tables.h")]
+
+
+def source_sha() -> str:
+    h = hashlib.sha256()
+    for f in KERNEL_SOURCES:
+        p = os.path.join(ROOT, f)
+        if os.path.exists(p):
+            h.update(open(p, "rb").read())
+    return h.hexdigest()[:16]
+
+
+def measured_peaks() -> dict:
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def profile_traffic(kernel: str):
+    """Per-launch DRAM bytes from a committed ncu summary, if it was taken
+    on the current kernel sources; otherwise None."""
+    path = os.path.join(ROOT, "profiles", f"{kernel}_mlp_14336.md")
+    if not os.path.exists(path):
+        return None
+    vals = {}
+    for line in open(path):
+        if ":" in line and line.strip().startswith("-"):
+            k, v = line.strip().lstrip("- ").split(":", 1)
+            vals[k.strip()] = v.strip().strip("`")
+    if vals.get("source_sha") != source_sha():
+        return None
+    try:
+        return float(vals["traffic_bytes_per_launch"])
+    except (KeyError, ValueError):
+        return None
+
+
+class ClockSampler:
+    """Samples SM clock and clock-event reasons through NVML while running."""
+
+    def __init__(self, device_index: int, period_s: float = 0.002):
+        self.samples, self.reasons = [], set()
+        self.period = period_s
+        self._stop = threading.Event()
+        self.max_mhz = None
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            self.h = pynvml.nvmlDeviceGetHandleByIndex(device_index)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+        except Exception:  # NVML missing: no clock record
+            self.nv = None
+
+    def _run(self):
+        nv = self.nv
+        names = {
+            "gpu_idle": 0x1, "applications_clocks_setting": 0x2, "sw_power_cap": 0x4, "hw_slowdown": 0x8,
+            "sync_boost": 0x10, "sw_thermal_slowdown": 0x20, "hw_thermal_slowdown": 0x40,
+            "hw_power_brake_slowdown": 0x80, "display_clock_setting": 0x100,
+        }
+        while not self._stop.is_set():
+            try:
+                self.samples.append(nv.nvmlDeviceGetClockInfo(self.h, nv.NVML_CLOCK_SM))
+                r = nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in names.items():
+                    if r & bit and k != "gpu_idle":
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(self.period)
+
+    def __enter__(self):
+        if self.nv is not None:
+            self._t = threading.Thread(target=self._run, daemon=True)
+            self._t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.nv is not None:
+            self._t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons), "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------
+# CPU oracle sample (reference arm and cpu_baseline)
+# --------------------------------------------------------------------------
+def oracle_sample_step(data, batches, k):
+    """One bounded sample of the step on the host: rows of up and down
+    (in the workload's 1 : 3.5 proportion), projected, encoded and
+    dequantised to the original basis; the sampled up rows' GEMV outputs at
+    every batch.  Returns the number of groups processed."""
+    import oracle
+    from bit_e8_lattice_b200 import synth
+
+    (up, d_up), (down, d_dn), xs = data
+    n_up, n_dn = 2, 7
+    ru = [(k * n_up + i) % D_MODEL for i in range(n_up)]
+    rd = [(k * n_dn + i) % D_FF for i in range(n_dn)]
+    out_u = oracle.project_encode(synth.bf16_bits_to_f64(up[ru]), d_up, 2048, want_x=False, want_margin=False)
+    out_d = oracle.project_encode(synth.bf16_bits_to_f64(down[rd]), d_dn, 2048, want_x=False, want_margin=False)
+    oracle.dequant(out_u["P"], out_u["scale"], d_up, 2048, "original")
+    oracle.dequant(out_d["P"], out_d["scale"], d_dn, 2048, "original")
+    for b in batches:
+        oracle.gemv(out_u["P"], out_u["scale"], d_up, 2048, synth.bf16_bits_to_f64(xs[b]))
+    return n_up * (D_FF // 8) + n_dn * (D_MODEL // 8)
+
+
+def cpu_oracle_rate(data, batches, seconds: float = 10.0):
+    t0 = time.perf_counter()
+    groups, k = 0, 0
+    while True:
+        groups += oracle_sample_step(data, batches, k)
+        k += 1
+        el = time.perf_counter() - t0
+        if el >= seconds:
+            break
+    return groups / el / 1e9, el, k
+
+
+def host_data(batches):
+    from bit_e8_lattice_b200 import synth
+
+    (up, d_up), (down, d_dn) = synth.mlp_14336()
+    xs = {b: synth.gemv_x(b, D_FF) for b in batches}
+    return (up, d_up), (down, d_dn), xs
+
+
+# --------------------------------------------------------------------------
+def run_reference(args, batches):
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return 0
+    data = host_data(batches)
+    for k in range(args.warmup):
+        oracle_sample_step(data, batches, k)
+    times, groups = [], 0
+    for k in range(args.steps):
+        t0 = time.perf_counter()
+        groups += oracle_sample_step(data, batches, args.warmup + k)
+        times.append(time.perf_counter() - t0)
+    total = sum(times)
+    value = groups / total / 1e9
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "sample": "2 rows of up + 7 rows of down per step, all four GEMV batches "
+                                                   "on the sampled up rows"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
+                         "sample": "2 up rows + 7 down rows per step (9,760 groups)"},
+        "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+    return 0
+
+
+def main():
+    ap = argparse.ArgumentParser(description=__doc__)
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=50)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["e8q", "reference"], default="e8q")
+    ap.add_argument("--batches", default="1,4,16,64")
+    ap.add_argument("--e2e-steps", type=int, default=10)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    batches = [int(b) for b in args.batches.split(",") if b]
+    if args.impl == "reference":
+        return run_reference(args, batches)
+
+    import torch
+    import torch.distributed as dist
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        from datetime import timedelta
+
+        dist.init_process_group("nccl", timeout=timedelta(seconds=300))
+    torch.cuda.set_device(local)
+    dev = torch.device("cuda", local)
+
+    from bit_e8_lattice_b200 import e8q
+
+    e8q.init()
+    data = host_data(batches)
+    (up, d_up), (down, d_dn), xs = data
+
+    def t_bf16(bits, pin=False):
+        t = torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16)
+        return t.pin_memory() if pin else t.to(dev)
+
+    W = [t_bf16(up), t_bf16(down)]
+    S = [torch.from_numpy(d_up).to(dev), torch.from_numpy(d_dn).to(dev)]
+    X = {b: t_bf16(xs[b]) for b in batches}
+    grad = torch.from_numpy(np.zeros(1, np.int16)).to(dev)  # identity STE: the gradient is aliased, never touched
+    G = D_MODEL * (D_FF // 8) + D_FF * (D_MODEL // 8)
+    enc = e8q.Encoder([(D_MODEL, D_FF), (D_FF, D_MODEL)], S, torch.bfloat16, 0, 1.0, "original",
+                      esc_cap=G // 2, ovf_cap=G // 16)
+    res = enc(W)
+    gemvs = {b: e8q.Gemv(res.encoded[0], b) for b in batches}
+    stream = torch.cuda.current_stream()
+
+    def step():
+        enc(W)
+        for b in batches:
+            gemvs[b](X[b])
+
+    for _ in range(max(args.warmup, 3)):
+        step()
+    torch.cuda.synchronize()
+    ctr = res.read_counters()
+    if ctr["n_dropped"] or ctr["err"]:
+        raise RuntimeError(f"encode capacity or ordering problem: {ctr}")
+
+    # Timed region: K whole steps, captured as one CUDA graph (the library's
+    # launches carry no Python overhead between them), with a timing event
+    # node around every kernel call; falls back to eager launches if the
+    # capture is refused.
+    K = args.steps
+
+    def record_steps(ev, t_start, t_end):
+        t_start.record()
+        for k in range(K):
+            ev[k][0].record()
+            enc(W)
+            ev[k][1].record()
+            for j, b in enumerate(batches):
+                gemvs[b](X[b])
+                ev[k][2 + j].record()
+        t_end.record()
+
+    def make_events(external):
+        ev = [[torch.cuda.Event(enable_timing=True, external=external) for _ in range(2 + len(batches))]
+              for _ in range(K)]
+        return ev, torch.cuda.Event(enable_timing=True, external=external), \
+            torch.cuda.Event(enable_timing=True, external=external)
+
+    graph = None
+    mode = "cuda_graph"
+    try:
+        ev, t_start, t_end = make_events(True)
+        graph = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.graph(graph, stream=cap):
+            record_steps(ev, t_start, t_end)
+        stream.wait_stream(cap)
+        graph.replay()  # upload + warm
+        torch.cuda.synchronize()
+    except Exception as exc:  # capture refused: time eager launches instead
+        print(f"# graph capture unavailable ({exc}); timing eager launches", file=sys.stderr)
+        graph, mode = None, "eager"
+        torch.cuda.synchronize()
+        ev, t_start, t_end = make_events(False)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    with ClockSampler(local) as clocks:
+        if graph is not None:
+            graph.replay()
+        else:
+            record_steps(ev, t_start, t_end)
+        torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    ms = t_start.elapsed_time(t_end)
+    if world > 1:
+        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
+        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+        ms = float(tt.item())
+    value = world * G * K / (ms * 1e-3) / 1e9
+
+    enc_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
+    gem_ms = {b: [ev[k][1 + j].elapsed_time(ev[k][2 + j]) for k in range(K)] for j, b in enumerate(batches)}
+    ctr = res.read_counters()
+    n_esc, n_ovf = ctr["n_escape"], ctr["n_overflow"]
+    rows = D_MODEL + D_FF
+    enc_bytes = G * (16 + 2 + 16) + rows * (4 + 16) + 8 * n_esc + 20 * n_ovf
+    enc_avg = statistics.mean(enc_ms)
+    peaks = measured_peaks()
+    enc_gbs = enc_bytes / (enc_avg * 1e-3) / 1e9
+
+    # GEMV algorithmic bytes: indices, the up matrix's records, scales, x, y
+    up_groups = D_MODEL * (D_FF // 8)
+    rp = res.esc_row_ptr.cpu().numpy()
+    op = res.ovf_row_ptr.cpu().numpy()
+    up_esc, up_ovf = int(rp[D_MODEL] - rp[0]), int(op[D_MODEL] - op[0])
+    kernels = {"project_encode": {
+        "launch_us": 1e3 * enc_avg, "Ggroups_s": G / (enc_avg * 1e-3) / 1e9, "GB_s": enc_gbs,
+        "frac_measured_hbm": enc_gbs / peaks["hbm_gbs"], "frac_nominal_8TBs": enc_gbs / NOMINAL_HBM_GBS,
+        "bytes_per_launch": enc_bytes}}
+    for b in batches:
+        gb_bytes = 2 * up_groups + 8 * up_esc + 20 * up_ovf + 4 * D_MODEL + 16 * (D_MODEL + 1) + 2 * b * (D_FF + D_MODEL)
+        avg = statistics.mean(gem_ms[b])
+        gbs = gb_bytes / (avg * 1e-3) / 1e9
+        kernels[f"dequant_gemv_b{b}"] = {"launch_us": 1e3 * avg, "GB_s": gbs,
+                                         "frac_measured_hbm": gbs / peaks["hbm_gbs"],
+                                         "frac_nominal_8TBs": gbs / NOMINAL_HBM_GBS, "bytes_per_launch": gb_bytes}
+
+    # end to end through the public API: pinned host inputs in, results out
+    e2e = None
+    if args.e2e_steps > 0:
+        Wh = [t_bf16(up, True), t_bf16(down, True)]
+        Xh = {b: t_bf16(xs[b], True) for b in batches}
+        Yh = {b: torch.empty((b, D_MODEL), dtype=torch.bfloat16).pin_memory() for b in batches}
+        Ch = torch.empty(6, dtype=torch.int64).pin_memory()
+        Wd = [torch.empty_like(W[0]), torch.empty_like(W[1])]
+        Xd = {b: torch.empty_like(X[b]) for b in batches}
+        h2d = sum(w.numel() * 2 for w in Wh) + sum(x.numel() * 2 for x in Xh.values())
+        d2h = sum(y.numel() * 2 for y in Yh.values()) + 48
+
+        def e2e_step():
+            for i in range(2):
+                Wd[i].copy_(Wh[i], non_blocking=True)
+            for b in batches:
+                Xd[b].copy_(Xh[b], non_blocking=True)
+            r = enc(Wd)
+            for b in batches:
+                Yh[b].copy_(gemvs[b](Xd[b]), non_blocking=True)
+            Ch.copy_(r.counters, non_blocking=True)
+
+        for _ in range(2):
+            e2e_step()
+        torch.cuda.synchronize()
+        a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        a.record(stream)
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        z.record(stream)
+        torch.cuda.synchronize()
+        ems = a.elapsed_time(z)
+        if world > 1:
+            tt = torch.tensor([ems], device=dev, dtype=torch.float64)
+            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
+            ems = float(tt.item())
+        e2e = {"value": world * G * args.e2e_steps / (ems * 1e-3) / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        rate, el, nsamp = cpu_oracle_rate(data, batches, args.cpu_seconds)
+        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
+               "sample": f"{nsamp} samples of 2 up rows + 7 down rows (9,760 groups each) incl. dequant and GEMV "
+                         f"rows, {el:.1f} s"}
+
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        traffic = profile_traffic("k_encode")
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
+            "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "groups_per_step_per_gpu": G, "kappa": 1.0, "rht_block": 2048,
+                       "gemv_batches": batches, "l2": "inputs larger than L2: 235 MB of latent weights read per step",
+                       "escape_fraction": n_esc / G, "overflow_fraction": n_ovf / G,
+                       "payload_bits_pages_formula": 2 + 20 * (n_esc + n_ovf) / G,
+                       "parallelism": f"replicas x{world} (rows are independent; no collective)"},
+            "roofline": {"bound": "hbm", "kernel": "k_encode", "achieved": enc_gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": enc_gbs / peaks["hbm_gbs"], "traffic": traffic,
+                         "peak_source": peaks["source"], "algorithmic_bytes_per_launch": enc_bytes},
+            "kernels": kernels,
+            "cpu_baseline": cpu,
+            "e2e": e2e,
+            "gpu_launches": K * (1 + 2 * len(batches)),
+            "timing": mode,
+            "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
+if __name__ == "__main__":
+    sys.exit(main())

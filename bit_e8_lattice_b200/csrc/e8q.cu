@@ -1,0 +1,304 @@
+// libe8q: C ABI entry points (include/e8q.h) over the sm_100a kernels.
+// Argument checks, per-device constant tables, workspace sizing, launches.
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstring>
+#include <mutex>
+#include <vector>
+
+#include "../../include/e8q.h"
+#include "common.cuh"
+#include "decode.cuh"
+#include "encode.cuh"
+#include "gemv.cuh"
+#include "tables.h"
+
+namespace e8q {
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+bool g_ready[kMaxDevices];
+int g_sms[kMaxDevices];
+
+e8q_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? E8Q_OK : E8Q_ERR_CUDA; }
+
+e8q_status ensure_device(int* dev_out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess) return E8Q_ERR_CUDA;
+    if (dev < 0 || dev >= kMaxDevices) return E8Q_ERR_UNSUPPORTED;
+    std::lock_guard<std::mutex> lock(g_mu);
+    if (!g_ready[dev]) {
+        const HostTables* t = host_tables();
+        if (!t) return E8Q_ERR_UNSUPPORTED;
+        std::vector<uint2> core(65536), roots(240);
+        std::memcpy(core.data(), t->core.data(), 65536 * 8);
+        std::memcpy(roots.data(), t->roots.data(), 240 * 8);
+        e8q_status st = E8Q_OK;
+        if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_t1, t->t1.data(), t->t1.size() * sizeof(uint16_t)));
+        if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_t2, t->t2.data(), t->t2.size() * sizeof(uint16_t)));
+        if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_core8, core.data(), core.size() * sizeof(uint2)));
+        if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_root8, roots.data(), roots.size() * sizeof(uint2)));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_encode<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEncSmemBytes));
+        if (st == E8Q_OK)
+            st = cuda_ok(
+                cudaFuncSetAttribute(k_encode<kMaxMats>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEncSmemBytes));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileMaxElems * 4));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_rht_x, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxCols * 4));
+        if (st == E8Q_OK) st = cuda_ok(cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev));
+        if (st != E8Q_OK) return st;
+        g_ready[dev] = true;
+    }
+    *dev_out = dev;
+    return E8Q_OK;
+}
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// log2 of the effective RHT block, or -1 if invalid
+int resolve_logb(int64_t cols, int32_t block) {
+    if (block == 1) return 0;
+    int64_t b = block;
+    if (block == 0) {
+        b = cols & -cols;
+        if (b > 2048) b = 2048;
+    }
+    if (b < 8 || b > 2048 || (b & (b - 1)) != 0 || cols % b != 0) return -1;
+    int l = 0;
+    while ((int64_t{1} << l) < b) ++l;
+    return l;
+}
+
+bool valid_cols(int64_t cols) { return cols >= 8 && cols % 8 == 0; }
+
+e8q_status check_encoded(const e8q_encoded* m, int* logb) {
+    if (!m || m->rows < 0 || !valid_cols(m->cols)) return E8Q_ERR_INVALID_ARG;
+    if (m->cols > kMaxCols || m->rows > (int64_t{1} << 30)) return E8Q_ERR_UNSUPPORTED;
+    *logb = resolve_logb(m->cols, m->rht_block);
+    if (*logb < 0) return E8Q_ERR_INVALID_ARG;
+    if (m->rows > 0 && (!m->idx || !m->scale)) return E8Q_ERR_INVALID_ARG;
+    if ((m->esc_row_ptr && !m->esc) || (m->ovf_row_ptr && !m->ovf)) return E8Q_ERR_INVALID_ARG;
+    if (m->esc_count < 0 || m->ovf_count < 0) return E8Q_ERR_INVALID_ARG;
+    if (m->group_base < 0) return E8Q_ERR_INVALID_ARG;
+    return E8Q_OK;
+}
+
+}  // namespace
+}  // namespace e8q
+
+using namespace e8q;
+
+extern "C" {
+
+const char* e8q_status_string(e8q_status s) {
+    switch (s) {
+        case E8Q_OK: return "ok";
+        case E8Q_ERR_INVALID_ARG: return "invalid argument";
+        case E8Q_ERR_UNSUPPORTED: return "unsupported";
+        case E8Q_ERR_CUDA: return "cuda error";
+        case E8Q_ERR_WORKSPACE: return "workspace too small";
+    }
+    return "unknown status";
+}
+
+e8q_status e8q_init(void) {
+    int dev;
+    return ensure_device(&dev);
+}
+
+e8q_status e8q_core_table(int8_t* out_coord2) {
+    if (!out_coord2) return E8Q_ERR_INVALID_ARG;
+    const HostTables* t = host_tables();
+    if (!t) return E8Q_ERR_UNSUPPORTED;
+    std::memcpy(out_coord2, t->core.data(), t->core.size());
+    return E8Q_OK;
+}
+
+size_t e8q_encode_workspace_bytes(const e8q_matrix* mats, int32_t n_mats) {
+    size_t tiles = 0;
+    if (mats && n_mats > 0)
+        for (int i = 0; i < n_mats; ++i) {
+            if (mats[i].rows <= 0 || !valid_cols(mats[i].cols) || mats[i].cols > kMaxCols) continue;
+            const int rpt = rows_per_tile(static_cast<int>(mats[i].cols));
+            tiles += static_cast<size_t>((mats[i].rows + rpt - 1) / rpt);
+        }
+    const size_t bytes = 16 + 8 * tiles;
+    return (bytes + 255) / 256 * 256;
+}
+
+e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_encode_args* a, void* ws,
+                              size_t ws_bytes, e8q_stream stream) {
+    if (!mats || !a || n_mats < 1) return E8Q_ERR_INVALID_ARG;
+    if (n_mats > kMaxMats) return E8Q_ERR_UNSUPPORTED;
+    if (!a->counters || !(a->kappa > 0.f) || !std::isfinite(a->kappa)) return E8Q_ERR_INVALID_ARG;
+    if (a->dequant < E8Q_DEQUANT_NONE || a->dequant > E8Q_DEQUANT_ORIGINAL) return E8Q_ERR_INVALID_ARG;
+    if (a->esc_cap < 0 || a->ovf_cap < 0 || (a->esc_cap > 0 && !a->esc) || (a->ovf_cap > 0 && !a->ovf))
+        return E8Q_ERR_INVALID_ARG;
+    if (a->scale_in != 0 && a->scale_in != 1) return E8Q_ERR_INVALID_ARG;
+
+    static thread_local EncodeParams<kMaxMats> P;  // ~28 KB: keep it off the stack
+    std::memset(&P, 0, sizeof(P));
+    int64_t tiles = 0, rows_total = 0, groups_total = 0;
+    for (int i = 0; i < n_mats; ++i) {
+        const e8q_matrix& m = mats[i];
+        if (m.rows < 0 || !valid_cols(m.cols)) return E8Q_ERR_INVALID_ARG;
+        if (m.cols > kMaxCols) return E8Q_ERR_UNSUPPORTED;
+        const int logb = resolve_logb(m.cols, m.rht_block);
+        if (logb < 0) return E8Q_ERR_INVALID_ARG;
+        if (m.in_dtype != E8Q_F32 && m.in_dtype != E8Q_BF16) return E8Q_ERR_INVALID_ARG;
+        if (m.rows > 0) {
+            if (!m.w || !m.signs || !m.idx || !m.scale) return E8Q_ERR_INVALID_ARG;
+            if (!aligned(m.w, 16) || !aligned(m.signs, 8) || !aligned(m.idx, 2) || !aligned(m.scale, 4))
+                return E8Q_ERR_INVALID_ARG;
+            if (a->dequant != E8Q_DEQUANT_NONE && (!m.dequant || !aligned(m.dequant, 16))) return E8Q_ERR_INVALID_ARG;
+        }
+        const int rpt = rows_per_tile(static_cast<int>(m.cols));
+        MatDesc& d = P.m[i];
+        d.w = m.w;
+        d.signs = m.signs;
+        d.idx = m.idx;
+        d.scale = m.scale;
+        d.dq = m.dequant;
+        d.rows = static_cast<int32_t>(m.rows);
+        d.cols = static_cast<int32_t>(m.cols);
+        d.meta = logb | ((m.in_dtype == E8Q_BF16) ? 16 : 0) | (rpt << 8);
+        d.tile_base = static_cast<int32_t>(tiles);
+        d.row_base = static_cast<int32_t>(rows_total);
+        d.group_base = static_cast<uint32_t>(groups_total);
+        tiles += (m.rows + rpt - 1) / rpt;
+        rows_total += m.rows;
+        groups_total += m.rows * (m.cols / 8);
+        if (groups_total >= (int64_t{1} << 31) || rows_total >= (int64_t{1} << 31)) return E8Q_ERR_UNSUPPORTED;
+    }
+    const size_t need = e8q_encode_workspace_bytes(mats, n_mats);
+    if (!ws || ws_bytes < need || !aligned(ws, 8)) return E8Q_ERR_WORKSPACE;
+
+    int dev;
+    e8q_status st = ensure_device(&dev);
+    if (st != E8Q_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = cuda_ok(cudaMemsetAsync(a->counters, 0, sizeof(e8q_counters), s));
+    if (st == E8Q_OK) st = cuda_ok(cudaMemsetAsync(ws, 0, need, s));
+    if (st != E8Q_OK) return st;
+    if (tiles == 0) {  // nothing to encode: empty CSR
+        if (a->esc_row_ptr) st = cuda_ok(cudaMemsetAsync(a->esc_row_ptr + rows_total, 0, sizeof(int64_t), s));
+        if (st == E8Q_OK && a->ovf_row_ptr)
+            st = cuda_ok(cudaMemsetAsync(a->ovf_row_ptr + rows_total, 0, sizeof(int64_t), s));
+        return st;
+    }
+    P.esc = a->esc;
+    P.ovf = a->ovf;
+    P.esc_rp = a->esc_row_ptr;
+    P.ovf_rp = a->ovf_row_ptr;
+    P.ctr = a->counters;
+    P.ws = static_cast<unsigned long long*>(ws);
+    P.esc_cap = a->esc_cap;
+    P.ovf_cap = a->ovf_cap;
+    P.kappa = a->kappa;
+    P.dq_mode = a->dequant;
+    P.scale_in = a->scale_in;
+    P.n_mats = n_mats;
+    P.n_tiles = static_cast<int32_t>(tiles);
+    P.total_rows = static_cast<int32_t>(rows_total);
+    const int grid = static_cast<int>(tiles < g_sms[dev] ? tiles : g_sms[dev]);
+    if (n_mats == 1) {
+        EncodeParams<1> P1;
+        std::memcpy(&P1, &P, offsetof(EncodeParams<1>, m));
+        P1.m[0] = P.m[0];
+        k_encode<1><<<grid, kEncThreads, kEncSmemBytes, s>>>(P1);
+    } else {
+        k_encode<kMaxMats><<<grid, kEncThreads, kEncSmemBytes, s>>>(P);
+    }
+    return cuda_ok(cudaGetLastError());
+}
+
+e8q_status e8q_decode(const e8q_encoded* m, int32_t basis, void* out_bf16, e8q_stream stream) {
+    int logb;
+    e8q_status st = check_encoded(m, &logb);
+    if (st != E8Q_OK) return st;
+    if (basis != E8Q_DEQUANT_ROTATED && basis != E8Q_DEQUANT_ORIGINAL) return E8Q_ERR_INVALID_ARG;
+    if (m->rows == 0) return E8Q_OK;
+    if (!out_bf16 || !aligned(out_bf16, 16)) return E8Q_ERR_INVALID_ARG;
+    if (basis == E8Q_DEQUANT_ORIGINAL && (!m->signs || !aligned(m->signs, 8))) return E8Q_ERR_INVALID_ARG;
+    int dev;
+    st = ensure_device(&dev);
+    if (st != E8Q_OK) return st;
+    DecodeParams p;
+    p.idx = m->idx;
+    p.scale = m->scale;
+    p.signs = m->signs;
+    p.esc = m->esc;
+    p.esc_rp = m->esc_row_ptr;
+    p.ovf = m->ovf;
+    p.ovf_rp = m->ovf_row_ptr;
+    p.esc_n = m->esc_row_ptr ? m->esc_count : 0;
+    p.ovf_n = m->ovf_row_ptr ? m->ovf_count : 0;
+    p.out = static_cast<uint16_t*>(out_bf16);
+    p.group_base = m->group_base;
+    p.rows = static_cast<int32_t>(m->rows);
+    p.cols = static_cast<int32_t>(m->cols);
+    p.logb = logb;
+    p.basis = basis;
+    p.rpt = rows_per_tile(p.cols);
+    p.n_tiles = (p.rows + p.rpt - 1) / p.rpt;
+    const int grid = p.n_tiles < 2 * g_sms[dev] ? p.n_tiles : 2 * g_sms[dev];
+    k_decode<<<grid, kDecThreads, kTileMaxElems * 4, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+    return cuda_ok(cudaGetLastError());
+}
+
+size_t e8q_gemv_workspace_bytes(const e8q_encoded* m, int32_t batch) {
+    if (!m || m->cols <= 0 || batch <= 0) return 256;
+    const size_t bytes = static_cast<size_t>(batch) * static_cast<size_t>(m->cols) * 4;
+    return (bytes + 255) / 256 * 256;
+}
+
+e8q_status e8q_dequant_gemv(const e8q_encoded* m, const void* x_bf16, int32_t batch, void* y_bf16, void* ws,
+                            size_t ws_bytes, e8q_stream stream) {
+    int logb;
+    e8q_status st = check_encoded(m, &logb);
+    if (st != E8Q_OK) return st;
+    if (batch < 1 || batch > 256) return E8Q_ERR_INVALID_ARG;
+    if (!x_bf16 || !y_bf16 || !m->signs || !aligned(x_bf16, 16) || !aligned(y_bf16, 2)) return E8Q_ERR_INVALID_ARG;
+    const size_t need = e8q_gemv_workspace_bytes(m, batch);
+    if (!ws || ws_bytes < need || !aligned(ws, 16)) return E8Q_ERR_WORKSPACE;
+    if (m->rows == 0) return E8Q_OK;
+    int dev;
+    st = ensure_device(&dev);
+    if (st != E8Q_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    RhtParams rp;
+    rp.x = static_cast<const uint16_t*>(x_bf16);
+    rp.signs = m->signs;
+    rp.xr = static_cast<float*>(ws);
+    rp.cols = static_cast<int32_t>(m->cols);
+    rp.logb = logb;
+    k_rht_x<<<batch, kRhtThreads, static_cast<size_t>(m->cols) * 4, s>>>(rp);
+    st = cuda_ok(cudaGetLastError());
+    if (st != E8Q_OK) return st;
+    GemvParams gp;
+    gp.idx = m->idx;
+    gp.scale = m->scale;
+    gp.esc = m->esc;
+    gp.esc_rp = m->esc_row_ptr;
+    gp.ovf = m->ovf;
+    gp.ovf_rp = m->ovf_row_ptr;
+    gp.esc_n = m->esc_row_ptr ? m->esc_count : 0;
+    gp.ovf_n = m->ovf_row_ptr ? m->ovf_count : 0;
+    gp.xr = static_cast<const float*>(ws);
+    gp.y = static_cast<uint16_t*>(y_bf16);
+    gp.group_base = m->group_base;
+    gp.rows = static_cast<int32_t>(m->rows);
+    gp.cols = static_cast<int32_t>(m->cols);
+    gp.batch = batch;
+    const int warps_per_cta = kGemvThreads / 32;
+    int grid = static_cast<int>((m->rows + warps_per_cta - 1) / warps_per_cta);
+    if (grid > 8 * g_sms[dev]) grid = 8 * g_sms[dev];
+    k_gemv<<<grid, kGemvThreads, 0, s>>>(gp);
+    return cuda_ok(cudaGetLastError());
+}
+
+}  // extern "C"

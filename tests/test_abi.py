@@ -1,0 +1,136 @@
+"""CPU-side checks of the C ABI: the library loads, exports every function
+that include/e8q.h declares, rejects bad arguments before touching a
+device, and its host-built core table agrees with the oracle's
+(Table 3, core decoding agreement).  No compute call is made here."""
+import ctypes
+import os
+import re
+
+import numpy as np
+import pytest
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "e8q.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from bit_e8_lattice_b200 import build, e8q
+
+    build.build()
+    return e8q.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    names = re.findall(r"\b(e8q_[a-z0-9_]+)\s*\(", src)
+    return sorted(set(names))
+
+
+def test_every_declared_function_is_exported(lib):
+    names = declared_functions()
+    assert {"e8q_project_encode", "e8q_decode", "e8q_dequant_gemv"} <= set(names)
+    for n in names:
+        assert hasattr(lib, n), n
+
+
+def test_struct_sizes_match_header():
+    from bit_e8_lattice_b200 import e8q
+
+    assert ctypes.sizeof(e8q.Matrix) == 64
+    assert ctypes.sizeof(e8q.EncodedC) == 104
+    assert e8q.ESC_DTYPE.itemsize == 8
+    assert e8q.OVF_DTYPE.itemsize == 20
+
+
+def test_status_strings(lib):
+    assert lib.e8q_status_string(0) == b"ok"
+    assert lib.e8q_status_string(1) == b"invalid argument"
+    assert lib.e8q_status_string(4) == b"workspace too small"
+
+
+def test_core_table_matches_oracle(lib):
+    import oracle
+    from bit_e8_lattice_b200 import e8q
+
+    np.testing.assert_array_equal(e8q.core_table(), oracle.core_points())
+
+
+def _mat(rows=4, cols=64, block=0, dtype=1):
+    from bit_e8_lattice_b200 import e8q
+
+    m = e8q.Matrix()
+    m.w = m.signs = m.idx = m.scale = 0x100000  # never dereferenced: the call fails before any device work
+    m.dequant = None
+    m.rows, m.cols, m.rht_block, m.in_dtype = rows, cols, block, dtype
+    return m
+
+
+def _args(**kw):
+    from bit_e8_lattice_b200 import e8q
+
+    a = e8q.EncodeArgs()
+    a.kappa = kw.get("kappa", 1.0)
+    a.dequant = kw.get("dequant", 0)
+    a.scale_in = 0
+    a.counters = 0x100000
+    return a
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(cols=12), 1),            # not a multiple of 8
+    (dict(cols=16392), 2),         # wider than this build handles
+    (dict(block=3), 1),            # not a power of two
+    (dict(block=4096), 1),         # larger than 2048
+    (dict(cols=96, block=64), 1),  # does not divide cols
+    (dict(dtype=7), 1),
+    (dict(rows=-1), 1),
+])
+def test_encode_rejects_bad_matrices(lib, kw, expect):
+    from bit_e8_lattice_b200 import e8q
+
+    mats = (e8q.Matrix * 1)(_mat(**kw))
+    rc = lib.e8q_project_encode(mats, 1, ctypes.byref(_args()), ctypes.c_void_p(0x100000), 1 << 20, None)
+    assert rc == expect
+
+
+def test_encode_rejects_bad_args(lib):
+    from bit_e8_lattice_b200 import e8q
+
+    mats = (e8q.Matrix * 1)(_mat())
+    assert lib.e8q_project_encode(mats, 0, ctypes.byref(_args()), ctypes.c_void_p(0x100000), 1 << 20, None) == 1
+    assert lib.e8q_project_encode(mats, 1, ctypes.byref(_args(kappa=0.0)), ctypes.c_void_p(0x100000), 1 << 20, None) == 1
+    assert lib.e8q_project_encode(mats, 1, ctypes.byref(_args(dequant=5)), ctypes.c_void_p(0x100000), 1 << 20, None) == 1
+    # dequant requested without an output buffer
+    assert lib.e8q_project_encode(mats, 1, ctypes.byref(_args(dequant=2)), ctypes.c_void_p(0x100000), 1 << 20, None) == 1
+    # workspace too small
+    need = lib.e8q_encode_workspace_bytes(mats, 1)
+    assert need >= 16
+    assert lib.e8q_project_encode(mats, 1, ctypes.byref(_args()), ctypes.c_void_p(0x100000), need - 1, None) == 4
+    assert lib.e8q_project_encode(mats, 449, ctypes.byref(_args()), ctypes.c_void_p(0x100000), 1 << 20, None) == 2
+
+
+def test_workspace_bytes_counts_tiles(lib):
+    from bit_e8_lattice_b200 import e8q
+
+    # 37 rows of 256 columns: 16 rows per tile -> 3 tiles
+    mats = (e8q.Matrix * 2)(_mat(rows=37, cols=256), _mat(rows=3, cols=14336))
+    assert lib.e8q_encode_workspace_bytes(mats, 2) == 256  # 16 + 8*6 rounded up
+    mats = (e8q.Matrix * 1)(_mat(rows=4096, cols=14336))
+    assert lib.e8q_encode_workspace_bytes(mats, 1) == (16 + 8 * 4096 + 255) // 256 * 256
+
+
+def test_decode_and_gemv_reject_bad_args(lib):
+    from bit_e8_lattice_b200 import e8q
+
+    m = e8q.EncodedC(0x100000, 0x100000, 0x100000, None, None, None, None, 0, 0, 4, 12, 0, 0, 0)
+    assert lib.e8q_decode(ctypes.byref(m), 1, ctypes.c_void_p(0x100000), None) == 1  # cols % 8
+    m.cols = 64
+    assert lib.e8q_decode(ctypes.byref(m), 9, ctypes.c_void_p(0x100000), None) == 1  # basis
+    assert lib.e8q_dequant_gemv(ctypes.byref(m), ctypes.c_void_p(0x100000), 0, ctypes.c_void_p(0x100000),
+                                ctypes.c_void_p(0x100000), 1 << 20, None) == 1  # batch 0
+    need = lib.e8q_gemv_workspace_bytes(ctypes.byref(m), 4)
+    assert need == 1024
+    assert lib.e8q_dequant_gemv(ctypes.byref(m), ctypes.c_void_p(0x100000), 4, ctypes.c_void_p(0x100000),
+                                ctypes.c_void_p(0x100000), need - 1, None) == 4

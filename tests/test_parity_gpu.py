@@ -1,0 +1,269 @@
+"""Parity of the CUDA path (through the C ABI) against the fp64 oracle.
+
+Inputs come from ``bit_e8_lattice_b200.synth``; expected values from
+``oracle`` only.  Tolerances are stated in ``tests/parity.py``.
+"""
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from bit_e8_lattice_b200 import synth
+from parity import MARGIN, check_encode, check_gemv, check_original_dequant, check_rotated_dequant, gpu_points
+import lattice_np
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def e8q():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_e8_lattice_b200 import e8q as m
+
+    m.init()
+    return m
+
+
+def dev_bf16(bits):
+    return torch.from_numpy(np.ascontiguousarray(bits).view(np.int16)).view(torch.bfloat16).cuda()
+
+
+def dev(a):
+    return torch.from_numpy(np.ascontiguousarray(a)).cuda()
+
+
+def host_idx(t):
+    return t.cpu().numpy().view(np.uint16)
+
+
+def run_encode(e8q, mats, signs, blocks=0, kappa=1.0, dequant="none", scales=None, dtype=torch.bfloat16,
+               esc_cap=None, ovf_cap=None):
+    ws = [dev_bf16(m) if dtype == torch.bfloat16 else dev(m.astype(np.float32)) for m in mats]
+    ss = [dev(s) for s in signs]
+    sc = [dev(s.astype(np.float32)) for s in scales] if scales is not None else None
+    enc = e8q.Encoder([w.shape for w in ws], ss, dtype, blocks, kappa, dequant, scales is not None, esc_cap, ovf_cap)
+    res = enc(ws, sc)
+    torch.cuda.synchronize()
+    return enc, res
+
+
+def values(m, dtype):
+    return synth.bf16_bits_to_f64(m) if dtype == torch.bfloat16 else m.astype(np.float64)
+
+
+def compare_all(e8q, res, mats, signs, blocks, kappa=1.0, dtype=torch.bfloat16, label="", rows=None):
+    ctr = res.read_counters()
+    assert ctr["err"] == 0 and ctr["n_dropped"] == 0, ctr
+    esc, ovf = res.escape_records(), res.overflow_records()
+    stats = []
+    for i, m in enumerate(mats):
+        C = m.shape[1]
+        B = blocks[i] if isinstance(blocks, (list, tuple)) else blocks
+        B = oracle.default_block(C) if B == 0 else B
+        rsel = np.arange(m.shape[0]) if rows is None else rows[i]
+        out = oracle.project_encode(values(m, dtype)[rsel], signs[i], B, kappa)
+        st = check_encode(out, host_idx(res.idx[i]), res.scale[i].cpu().numpy(), esc, ovf, res.group_base[i], rsel,
+                          C // 8, label=f"{label}[{i}]")
+        stats.append(st)
+    return stats
+
+
+# ----------------------------------------------------------------------
+def test_core_decoding_agreement_decode_and_gemv(e8q):
+    """Table 3: all 65,536 core codewords decode to the same coordinates
+    through the decode kernel and through the GEMV kernel."""
+    core = oracle.core_points().astype(np.int32)
+    idx = torch.arange(65536, dtype=torch.int32).to(torch.int16).reshape(65536, 1).cuda()
+    scale = torch.full((65536,), 2.0, dtype=torch.float32, device="cuda")
+    signs = torch.ones(8, dtype=torch.int8, device="cuda")
+    m = e8q.Encoded(idx, scale, signs, None, None, None, None, 65536, 8, 0, 1)
+    out = e8q.e8q_decode(m, "rotated")
+    got = synth.bf16_bits_to_f64(out.cpu().view(torch.int16).numpy().view(np.uint16))
+    np.testing.assert_array_equal(got, core.astype(np.float64))  # 2 * P/2 = P, exact in bf16
+    x = dev_bf16(synth.f64_to_bf16_bits(np.eye(8)))
+    y = e8q.Gemv(m, 8)(x)
+    got = synth.bf16_bits_to_f64(y.cpu().view(torch.int16).numpy().view(np.uint16)).T
+    np.testing.assert_array_equal(got, core.astype(np.float64))
+
+
+def test_small_f32_encode_decode(e8q):
+    w, d = synth.small_f32()
+    enc, res = run_encode(e8q, [w], [d], 256, dtype=torch.float32, dequant="rotated")
+    st = compare_all(e8q, res, [w], [d], 256, dtype=torch.float32, label="small_f32")[0]
+    assert st["near_ties"] <= 4 and 0.1 < st["rho"] < 0.4
+    P = st["points"]
+    scale = res.scale[0].cpu().numpy()
+    dq = res.dequant[0].cpu().view(torch.int16).numpy()
+    check_rotated_dequant(dq, P, scale, d, 256, "encode dequant rotated")
+    enc_m = res.encoded[0]
+    out = e8q.e8q_decode(enc_m, "rotated").cpu().view(torch.int16).numpy()
+    check_rotated_dequant(out, P, scale, d, 256, "decode rotated")
+    out = e8q.e8q_decode(enc_m, "original").cpu().view(torch.int16).numpy()
+    check_original_dequant(out, P, scale, d, 256, "decode original")
+
+
+def test_free_vectors_exact_projection(e8q):
+    """4,096 vectors 3*N(0, I), no transform, scale 1: the projection sees
+    exactly the oracle's x."""
+    x = synth.free_vectors()
+    ones = np.ones(8, np.int8)
+    enc, res = run_encode(e8q, [x], [ones], 1, dtype=torch.float32, scales=[np.ones(len(x))])
+    out = oracle.project_encode_vectors(x.astype(np.float64))
+    out["scale"] = np.ones(len(x))
+    out["x"] = x.astype(np.float64)
+    st = check_encode(out, host_idx(res.idx[0]), res.scale[0].cpu().numpy(), res.escape_records(),
+                      res.overflow_records(), 0, None, 1, "free_vectors")
+    assert st["overflow"] > 0
+
+
+@pytest.mark.parametrize("lo,hi", [(0, 48), (56, 56), (64, 64)])
+def test_escape_rule_on_whole_shells(e8q, lo, hi):
+    """Every E8 point of |p|^2 <= 12, = 14 and = 16 given exactly: core
+    index, escape root and overflow decision agree with the oracle's
+    brute-force search over the 240 roots."""
+    P, _ = lattice_np.e8_points(hi, lo)
+    x = (P / 2.0).astype(np.float32)
+    enc, res = run_encode(e8q, [x], [np.ones(8, np.int8)], 1, dtype=torch.float32, scales=[np.ones(len(x))],
+                          esc_cap=len(x), ovf_cap=len(x))
+    out = oracle.project_encode_vectors(x.astype(np.float64))
+    np.testing.assert_array_equal(out["P"], P)
+    Pg, kind, root, _, _ = gpu_points(host_idx(res.idx[0]).reshape(-1), res.escape_records(), res.overflow_records(),
+                                      len(x))
+    np.testing.assert_array_equal(Pg, P)
+    np.testing.assert_array_equal(host_idx(res.idx[0]).reshape(-1).astype(np.int64), out["idx"])
+    np.testing.assert_array_equal(kind, out["kind"])
+    np.testing.assert_array_equal(root[kind == 1], out["root"][kind == 1])
+
+
+def test_attn_2048_full(e8q):
+    w, d = synth.attn_2048()
+    enc, res = run_encode(e8q, [w], [d], 0, dequant="original")
+    st = compare_all(e8q, res, [w], [d], [2048], label="attn_2048")[0]
+    assert st["near_ties"] < 200
+    P = st["points"]
+    scale = res.scale[0].cpu().numpy()
+    check_original_dequant(res.dequant[0].cpu().view(torch.int16).numpy(), P, scale, d, 2048, "attn original")
+    out = e8q.e8q_decode(res.encoded[0], "rotated").cpu().view(torch.int16).numpy()
+    check_rotated_dequant(out, P, scale, d, 2048, "attn decode rotated")
+
+
+def test_moe_batched_two_experts_full(e8q):
+    mats = synth.moe_bank(experts=2)
+    W = [m for m, _ in mats]
+    S = [s for _, s in mats]
+    enc, res = run_encode(e8q, W, S, 0)
+    stats = compare_all(e8q, res, W, S, 0, label="moe2")
+    for st in stats:
+        assert st["groups"] > 0
+
+
+@pytest.mark.parametrize("rows,cols,block", [(37, 256, 0), (5, 8, 0), (9, 24, 0), (3, 40, 0), (6, 96, 0),
+                                             (70, 64, 0), (4, 16384, 0), (3, 768, 256), (2, 4096, 512), (129, 8, 1)])
+def test_shapes_and_ragged_tiles(e8q, rows, cols, block):
+    rng = np.random.default_rng(rows * 1000 + cols)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((rows, cols)) * 0.03)
+    d = synth.signs(rows, cols)
+    enc, res = run_encode(e8q, [w], [d], block, dequant="original")
+    B = oracle.default_block(cols) if block == 0 else block
+    st = compare_all(e8q, res, [w], [d], [B], label=f"{rows}x{cols}")[0]
+    check_original_dequant(res.dequant[0].cpu().view(torch.int16).numpy(), st["points"], res.scale[0].cpu().numpy(),
+                           d, B, "original")
+    rp = res.esc_row_ptr.cpu().numpy()
+    assert rp[0] == 0 and (np.diff(rp) >= 0).all() and rp[-1] == res.read_counters()["n_escape"]
+
+
+def test_f32_input_block_2048(e8q):
+    rng = np.random.default_rng(77)
+    w = (rng.standard_normal((40, 4096)) * 0.02).astype(np.float32)
+    d = synth.signs(77, 4096)
+    enc, res = run_encode(e8q, [w], [d], 0, dtype=torch.float32)
+    compare_all(e8q, res, [w], [d], [2048], dtype=torch.float32, label="f32_4096")
+
+
+@pytest.mark.parametrize("kappa", [0.6, 2.5])
+def test_kappa(e8q, kappa):
+    w, d = synth.small_f32()
+    enc, res = run_encode(e8q, [w], [d], 0, kappa=kappa, dtype=torch.float32)
+    compare_all(e8q, res, [w], [d], [256], kappa=kappa, dtype=torch.float32, label=f"kappa{kappa}")
+
+
+def test_nonfinite_and_zero_rows(e8q):
+    rng = np.random.default_rng(5)
+    w = (rng.standard_normal((6, 64)) * 0.02).astype(np.float32)
+    w[1, 3] = np.nan
+    w[2, 10] = np.inf
+    w[2, 11] = -np.inf
+    w[3] = 0.0
+    d = synth.signs(5, 64)
+    enc, res = run_encode(e8q, [w], [d], 0, dtype=torch.float32)
+    ctr = res.read_counters()
+    assert ctr["n_nonfinite"] == 3
+    out = oracle.project_encode(w.astype(np.float64), d, 64)
+    assert out["nonfinite"] == 3
+    check_encode(out, host_idx(res.idx[0]), res.scale[0].cpu().numpy(), res.escape_records(), res.overflow_records(),
+                 0, None, 8, "nonfinite")
+    assert res.scale[0].cpu().numpy()[3] == 0.0 and (host_idx(res.idx[0])[3] == 0).all()
+
+
+def test_empty_matrix(e8q):
+    d = synth.signs(1, 64)
+    enc, res = run_encode(e8q, [np.zeros((0, 64), np.uint16)], [d], 0)
+    ctr = res.read_counters()
+    assert ctr["n_escape"] == 0 and ctr["n_overflow"] == 0
+    assert res.esc_row_ptr.cpu().numpy().tolist() == [0]
+
+
+def test_capacity_shortfall_is_reported(e8q):
+    w, d = synth.small_f32()
+    _, full = run_encode(e8q, [w], [d], 0, dtype=torch.float32)
+    ref_e = full.escape_records().copy()
+    ref_rp = full.esc_row_ptr.cpu().numpy().copy()
+    tot = full.read_counters()
+    _, res = run_encode(e8q, [w], [d], 0, dtype=torch.float32, esc_cap=5, ovf_cap=0)
+    ctr = res.read_counters()
+    assert ctr["n_escape"] == tot["n_escape"] and ctr["n_overflow"] == tot["n_overflow"]
+    assert ctr["n_dropped"] == (tot["n_escape"] - 5) + tot["n_overflow"]
+    np.testing.assert_array_equal(res.escape_records()[:5], ref_e[:5])
+    np.testing.assert_array_equal(res.esc_row_ptr.cpu().numpy(), ref_rp)
+
+
+def test_scale_in(e8q):
+    w, d = synth.small_f32()
+    s = np.sqrt((w.astype(np.float64) ** 2).mean(1)) * 0.75
+    enc, res = run_encode(e8q, [w], [d], 0, dtype=torch.float32, scales=[s.astype(np.float32)])
+    # the oracle with a fixed scale: kappa chosen so that rms / kappa == s
+    s32 = s.astype(np.float32).astype(np.float64)
+    out = oracle.project_encode(w.astype(np.float64), d, 256, kappa=1.0)
+    rms = out["scale"]
+    out = oracle.project_encode(w.astype(np.float64), d, 256, kappa=1.0 / 0.75)
+    np.testing.assert_allclose(res.scale[0].cpu().numpy(), s32, rtol=0)
+    np.testing.assert_allclose(out["scale"], s32, rtol=1e-6)
+    check_encode(out, host_idx(res.idx[0]), out["scale"], res.escape_records(), res.overflow_records(), 0, None, 32,
+                 "scale_in")
+
+
+def test_deterministic_outputs(e8q):
+    w, d = synth.attn_2048()
+    _, a = run_encode(e8q, [w], [d], 0)
+    ia, ea, oa = host_idx(a.idx[0]).copy(), a.escape_records().copy(), a.overflow_records().copy()
+    sa = a.scale[0].cpu().numpy().copy()
+    _, b = run_encode(e8q, [w], [d], 0)
+    np.testing.assert_array_equal(ia, host_idx(b.idx[0]))
+    np.testing.assert_array_equal(sa, b.scale[0].cpu().numpy())
+    assert ea.tobytes() == b.escape_records().tobytes() and oa.tobytes() == b.overflow_records().tobytes()
+
+
+@pytest.mark.parametrize("batch", [1, 4, 16, 64])
+def test_gemv_small(e8q, batch):
+    rng = np.random.default_rng(batch)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((512, 2048)) * 0.015)
+    d = synth.signs(batch, 2048)
+    enc, res = run_encode(e8q, [w], [d], 0)
+    st = compare_all(e8q, res, [w], [d], [2048], label="gemv_w")[0]
+    xb = synth.gemv_x(batch, 2048)
+    y = e8q.Gemv(res.encoded[0], batch)(dev_bf16(xb))
+    torch.cuda.synchronize()
+    y_ref = oracle.gemv(st["points"], res.scale[0].cpu().numpy().astype(np.float64), d, 2048,
+                        synth.bf16_bits_to_f64(xb))
+    check_gemv(y.cpu().view(torch.int16).numpy(), y_ref, f"gemv b={batch}")
