@@ -15,10 +15,10 @@ constexpr int kMaxTileRows = 64;
 constexpr int kMaxCols = 16384;
 
 // Constant tables, one copy per device, filled once from the host.
-__device__ uint16_t g_t1[2 * 2401 * 7];
-__device__ uint16_t g_t2[2 * 2401];
-__device__ uint2 g_core8[65536];  // 8 int8 doubled coordinates per core index
-__device__ uint2 g_root8[240];
+__device__ __align__(16) uint16_t g_t1[2 * 2401 * 7];
+__device__ __align__(16) uint16_t g_t2[2 * 2401];
+__device__ __align__(16) uint2 g_core8[65536];  // 8 int8 doubled coordinates per core index
+__device__ __align__(16) uint2 g_root8[240];
 
 // Rows per tile: enough rows that a tile holds about 4K elements.
 __host__ __device__ inline int rows_per_tile(int cols) {

@@ -85,20 +85,19 @@ __global__ void __launch_bounds__(kDecThreads) k_decode(const __grid_constant__ 
                                     pack_bf16x2(bf16_of_product(s, 0.5f * b.z), bf16_of_product(s, 0.5f * b.w)));
             }
         } else {
-            for (int q = tid; q < (n >> 3); q += kDecThreads) {
-                const float s = p.scale[r0 + q / gpr];
+            for (int q = tid; q < (n >> 3); q += kDecThreads) {  // p = P / 2, exact
                 float4* v = reinterpret_cast<float4*>(tile) + 2 * q;
                 float4 a = v[0], b = v[1];
-                a.x = s * (0.5f * a.x); a.y = s * (0.5f * a.y); a.z = s * (0.5f * a.z); a.w = s * (0.5f * a.w);
-                b.x = s * (0.5f * b.x); b.y = s * (0.5f * b.y); b.z = s * (0.5f * b.z); b.w = s * (0.5f * b.w);
+                a.x *= 0.5f; a.y *= 0.5f; a.z *= 0.5f; a.w *= 0.5f;
+                b.x *= 0.5f; b.y *= 0.5f; b.z *= 0.5f; b.w *= 0.5f;
                 v[0] = a;
                 v[1] = b;
             }
             __syncthreads();
-            if (p.logb > 0) fwht_smem(tile, n, p.logb);
-            const float inv = 1.0f / sqrtf(B);
+            if (p.logb > 0) fwht_smem(tile, n, p.logb);  // H(p): exact in fp32
             for (int q = tid; q < (n >> 3); q += kDecThreads) {
                 const int c0 = (q << 3) % C;
+                const float inv = p.scale[r0 + q / gpr] / sqrtf(B);
                 const uint2 dv = *reinterpret_cast<const uint2*>(p.signs + c0);
                 const float4 a = reinterpret_cast<const float4*>(tile)[2 * q];
                 const float4 b = reinterpret_cast<const float4*>(tile)[2 * q + 1];

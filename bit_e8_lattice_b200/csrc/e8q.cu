@@ -11,6 +11,7 @@
 #include "common.cuh"
 #include "decode.cuh"
 #include "encode.cuh"
+#include "encode_fast.cuh"
 #include "gemv.cuh"
 #include "tables.h"
 
@@ -46,6 +47,12 @@ e8q_status ensure_device(int* dev_out) {
             st = cuda_ok(
                 cudaFuncSetAttribute(k_encode<kMaxMats>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEncSmemBytes));
         if (st == E8Q_OK)
+            st = cuda_ok(
+                cudaFuncSetAttribute(k_encode_fast<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kFastSmemBytes));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_encode_fast<kMaxMats>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              kFastSmemBytes));
+        if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileMaxElems * 4));
         if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_rht_x, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxCols * 4));
@@ -74,6 +81,40 @@ int resolve_logb(int64_t cols, int32_t block) {
 }
 
 bool valid_cols(int64_t cols) { return cols >= 8 && cols % 8 == 0; }
+
+size_t align256(size_t x) { return (x + 255) / 256 * 256; }
+
+// The fast kernel takes bf16 rows whose width is a multiple of 256, with an
+// RHT block of at least 256, and 16-byte aligned index / output buffers.
+bool fast_path_ok(const e8q_matrix& m, int logb, int dequant) {
+    if (m.in_dtype != E8Q_BF16 || m.cols % 256 != 0 || logb < 8) return false;
+    if (m.rows > 0 && (!aligned(m.idx, 16) || (dequant != E8Q_DEQUANT_NONE && !aligned(m.dequant, 16)))) return false;
+    return true;
+}
+
+struct TileCounts {
+    int64_t generic = 0;
+    int64_t fast = 0;
+};
+
+TileCounts count_tiles(const e8q_matrix* mats, int n) {
+    TileCounts tc;
+    for (int i = 0; i < n; ++i) {
+        if (mats[i].rows <= 0 || !valid_cols(mats[i].cols) || mats[i].cols > kMaxCols) continue;
+        const int c = static_cast<int>(mats[i].cols);
+        tc.generic += (mats[i].rows + rows_per_tile(c) - 1) / rows_per_tile(c);
+        tc.fast += (mats[i].rows + fast_rows_per_tile(c) - 1) / fast_rows_per_tile(c);
+    }
+    return tc;
+}
+
+// workspace: [ticket, unused, status[tiles]] then the fast kernel's
+// per-CTA overflow-coordinate scratch (3 tiles x 2048 groups x 16 bytes)
+size_t status_bytes(const TileCounts& tc) { return align256(16 + 8 * static_cast<size_t>(tc.generic)); }
+size_t scratch_bytes(const TileCounts& tc) {
+    const int64_t ctas = tc.fast < kFastMaxCtas ? tc.fast : kFastMaxCtas;
+    return static_cast<size_t>(ctas) * 3 * kFastTileGroups * 16;
+}
 
 e8q_status check_encoded(const e8q_encoded* m, int* logb) {
     if (!m || m->rows < 0 || !valid_cols(m->cols)) return E8Q_ERR_INVALID_ARG;
@@ -119,15 +160,9 @@ e8q_status e8q_core_table(int8_t* out_coord2) {
 }
 
 size_t e8q_encode_workspace_bytes(const e8q_matrix* mats, int32_t n_mats) {
-    size_t tiles = 0;
-    if (mats && n_mats > 0)
-        for (int i = 0; i < n_mats; ++i) {
-            if (mats[i].rows <= 0 || !valid_cols(mats[i].cols) || mats[i].cols > kMaxCols) continue;
-            const int rpt = rows_per_tile(static_cast<int>(mats[i].cols));
-            tiles += static_cast<size_t>((mats[i].rows + rpt - 1) / rpt);
-        }
-    const size_t bytes = 16 + 8 * tiles;
-    return (bytes + 255) / 256 * 256;
+    TileCounts tc;
+    if (mats && n_mats > 0) tc = count_tiles(mats, n_mats);
+    return status_bytes(tc) + scratch_bytes(tc);
 }
 
 e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_encode_args* a, void* ws,
@@ -142,6 +177,13 @@ e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_
 
     static thread_local EncodeParams<kMaxMats> P;  // ~28 KB: keep it off the stack
     std::memset(&P, 0, sizeof(P));
+    bool fast = true;
+    for (int i = 0; i < n_mats; ++i) {
+        const int logb = resolve_logb(mats[i].cols, mats[i].rht_block);
+        if (!valid_cols(mats[i].cols) || mats[i].cols > kMaxCols || logb < 0 ||
+            !fast_path_ok(mats[i], logb, a->dequant))
+            fast = false;
+    }
     int64_t tiles = 0, rows_total = 0, groups_total = 0;
     for (int i = 0; i < n_mats; ++i) {
         const e8q_matrix& m = mats[i];
@@ -156,7 +198,7 @@ e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_
                 return E8Q_ERR_INVALID_ARG;
             if (a->dequant != E8Q_DEQUANT_NONE && (!m.dequant || !aligned(m.dequant, 16))) return E8Q_ERR_INVALID_ARG;
         }
-        const int rpt = rows_per_tile(static_cast<int>(m.cols));
+        const int rpt = fast ? fast_rows_per_tile(static_cast<int>(m.cols)) : rows_per_tile(static_cast<int>(m.cols));
         MatDesc& d = P.m[i];
         d.w = m.w;
         d.signs = m.signs;
@@ -174,15 +216,16 @@ e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_
         groups_total += m.rows * (m.cols / 8);
         if (groups_total >= (int64_t{1} << 31) || rows_total >= (int64_t{1} << 31)) return E8Q_ERR_UNSUPPORTED;
     }
-    const size_t need = e8q_encode_workspace_bytes(mats, n_mats);
-    if (!ws || ws_bytes < need || !aligned(ws, 8)) return E8Q_ERR_WORKSPACE;
+    const TileCounts tc = count_tiles(mats, n_mats);
+    const size_t need = status_bytes(tc) + scratch_bytes(tc);
+    if (!ws || ws_bytes < need || !aligned(ws, 256)) return E8Q_ERR_WORKSPACE;
 
     int dev;
     e8q_status st = ensure_device(&dev);
     if (st != E8Q_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
     st = cuda_ok(cudaMemsetAsync(a->counters, 0, sizeof(e8q_counters), s));
-    if (st == E8Q_OK) st = cuda_ok(cudaMemsetAsync(ws, 0, need, s));
+    if (st == E8Q_OK) st = cuda_ok(cudaMemsetAsync(ws, 0, 16 + 8 * static_cast<size_t>(tiles), s));
     if (st != E8Q_OK) return st;
     if (tiles == 0) {  // nothing to encode: empty CSR
         if (a->esc_row_ptr) st = cuda_ok(cudaMemsetAsync(a->esc_row_ptr + rows_total, 0, sizeof(int64_t), s));
@@ -204,6 +247,21 @@ e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_
     P.n_mats = n_mats;
     P.n_tiles = static_cast<int32_t>(tiles);
     P.total_rows = static_cast<int32_t>(rows_total);
+    if (fast) {
+        int64_t g = tiles < g_sms[dev] ? tiles : g_sms[dev];
+        if (g > kFastMaxCtas) g = kFastMaxCtas;
+        const int grid = static_cast<int>(g);
+        int16_t* scratch = reinterpret_cast<int16_t*>(static_cast<char*>(ws) + status_bytes(tc));
+        if (n_mats == 1) {
+            EncodeParams<1> P1;
+            std::memcpy(&P1, &P, offsetof(EncodeParams<1>, m));
+            P1.m[0] = P.m[0];
+            k_encode_fast<1><<<grid, kFastThreads, kFastSmemBytes, s>>>(P1, scratch);
+        } else {
+            k_encode_fast<kMaxMats><<<grid, kFastThreads, kFastSmemBytes, s>>>(P, scratch);
+        }
+        return cuda_ok(cudaGetLastError());
+    }
     const int grid = static_cast<int>(tiles < g_sms[dev] ? tiles : g_sms[dev]);
     if (n_mats == 1) {
         EncodeParams<1> P1;

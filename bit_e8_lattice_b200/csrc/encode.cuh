@@ -276,10 +276,10 @@ __global__ void __launch_bounds__(kEncThreads, 1) k_encode(const __grid_constant
                     o.w = pack_bf16x2(bf16_of_product(s, 0.5f * P[6]), bf16_of_product(s, 0.5f * P[7]));
                     reinterpret_cast<uint4*>(static_cast<uint16_t*>(M.dq) + static_cast<size_t>(r0) * C)[g] = o;
                 } else if (p.dq_mode == E8Q_DEQUANT_ORIGINAL) {
-                    const float s = s_rows[r];
+                    // p itself; H(p) stays exact in fp32 and is scaled once afterwards
                     float4* dst = reinterpret_cast<float4*>(tile) + 2 * g;
-                    dst[0] = make_float4(s * (0.5f * P[0]), s * (0.5f * P[1]), s * (0.5f * P[2]), s * (0.5f * P[3]));
-                    dst[1] = make_float4(s * (0.5f * P[4]), s * (0.5f * P[5]), s * (0.5f * P[6]), s * (0.5f * P[7]));
+                    dst[0] = make_float4(0.5f * P[0], 0.5f * P[1], 0.5f * P[2], 0.5f * P[3]);
+                    dst[1] = make_float4(0.5f * P[4], 0.5f * P[5], 0.5f * P[6], 0.5f * P[7]);
                 }
             }
             const unsigned be = __ballot_sync(0xFFFFFFFFu, kind == 1);
@@ -335,10 +335,10 @@ __global__ void __launch_bounds__(kEncThreads, 1) k_encode(const __grid_constant
         if (p.dq_mode == E8Q_DEQUANT_ORIGINAL) {
             __syncthreads();
             if (logb > 0) fwht_smem(tile, n, logb);
-            const float inv = 1.0f / sqrtf(B);
             uint4* dst = reinterpret_cast<uint4*>(static_cast<uint16_t*>(M.dq) + static_cast<size_t>(r0) * C);
             for (int q = tid; q < (n >> 3); q += kEncThreads) {
                 const int c0 = (q << 3) % C;
+                const float inv = s_rows[(q << 3) / C] / sqrtf(B);
                 const uint2 dv = *reinterpret_cast<const uint2*>(M.signs + c0);
                 const float4 a = reinterpret_cast<const float4*>(tile)[2 * q];
                 const float4 b = reinterpret_cast<const float4*>(tile)[2 * q + 1];

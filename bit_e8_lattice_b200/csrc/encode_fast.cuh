@@ -1,0 +1,748 @@
+// K1 fast path: RHT + row scale + E8 projection + core encoding + ordered
+// records (+ dequantised output) for bf16 weights whose width is a multiple
+// of 256 and whose RHT block is 256..2048 ("E8-QAT", Figure 2 (a)-(c)).
+//
+// CTA = 8 compute warps + 1 service warp, persistent over row tiles of up
+// to 16K elements taken from an atomic ticket.
+//   service warp: claims the next tile and prefetches it with a 1-D bulk
+//     copy (TMA engine) into the other shared-memory buffer; publishes the
+//     finished tile's record counts; stores its 16-bit indices with a bulk
+//     copy; resolves, one tile later still, the tile's place among all
+//     earlier tiles' records (decoupled look-back, bounded waits).
+//   compute warps: one 2048-element window each.  Hadamard in registers:
+//     bits {0,1,3,4} of the element index by one bf16 m16n8k16 tensor-core
+//     MMA against H_16 straight from the (sign-flipped) bf16 input, bit 2
+//     and bits 8..10 as fp32 butterflies, then an in-warp transpose through
+//     shared memory and bits 5..7.  Row scales from per-window sums of
+//     squares; projection, core rank and escape search in registers; groups
+//     outside the core go to a per-warp queue so the root search runs with
+//     all lanes busy.  Records are emitted in group order two tiles later.
+// Record order, CSR and results are the same as the generic kernel's.
+#pragma once
+#include "common.cuh"
+#include "encode.cuh"
+#include "lattice.cuh"
+#include "ptx.cuh"
+
+namespace e8q {
+
+constexpr int kFastWarps = 8;
+constexpr int kFastThreads = (kFastWarps + 1) * 32;
+constexpr int kFastTileElems = 16384;
+constexpr int kFastTileGroups = kFastTileElems / 8;
+constexpr int kFastMaxCtas = 160;
+constexpr int kQueueCap = 64;
+constexpr int kWaitLimit = 1 << 24;
+
+__host__ __device__ inline int fast_rows_per_tile(int cols) {
+    int r = kFastTileElems / cols;
+    return r < 1 ? 1 : (r > kMaxTileRows ? kMaxTileRows : r);
+}
+
+// shared-memory layout (bytes)
+constexpr int kFsIn = 0;                                      // bf16 [2][16384]
+constexpr int kFsT1 = kFsIn + 2 * kFastTileElems * 2;         // 65536
+constexpr int kFsT2 = kFsT1 + kEncT1Bytes;
+constexpr int kFsMap = kFsT2 + kEncT2Bytes;                   // u32 [3][2048]
+constexpr int kFsIdx = kFsMap + 3 * kFastTileGroups * 4;      // u16 [2][2048]
+constexpr int kFsGss = kFsIdx + 2 * kFastTileGroups * 2;      // f32 [2048]
+constexpr int kFsQueue = kFsGss + kFastTileGroups * 4;        // u32 [8][64][5]
+constexpr int kFsChunk = kFsQueue + kFastWarps * kQueueCap * 20;  // u32 [3][2][65]
+constexpr int kFastSmemBytes = kFsChunk + 3 * 2 * 65 * 4 + 8;
+
+struct FastTile {
+    int t;        // ticket (>= n_tiles: none)
+    int mat;
+    int r0;
+    int nr;
+    unsigned ne;  // escape records of the tile
+    unsigned no;  // overflow records of the tile
+};
+
+// ---------------------------------------------------------------- helpers
+__device__ __forceinline__ void bfly(float& a, float& b) {
+    const float x = a;
+    a = x + b;
+    b = x - b;
+}
+
+__device__ __forceinline__ void bfly2(float& a0, float& a1, float& b0, float& b1) {
+    const float2 a = make_float2(a0, a1), b = make_float2(b0, b1);
+    const float2 s = __fadd2_rn(a, b);
+    const float2 d = __ffma2_rn(b, make_float2(-1.f, -1.f), a);
+    a0 = s.x; a1 = s.y; b0 = d.x; b1 = d.y;
+}
+
+// butterflies between the 8-value rows v[k] and v[k ^ m] for register bit m
+template <int M>
+__device__ __forceinline__ void stage_rows(float (&v)[8][8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k)
+        if ((k & M) == 0)
+#pragma unroll
+            for (int e = 0; e < 8; e += 2) bfly2(v[k][e], v[k][e + 1], v[k + M][e], v[k + M][e + 1]);
+}
+
+// butterflies between element e and e + 4 of every row (element bit 2)
+__device__ __forceinline__ void stage_e2(float (&v)[8][8]) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        bfly2(v[k][0], v[k][1], v[k][4], v[k][5]);
+        bfly2(v[k][2], v[k][3], v[k][6], v[k][7]);
+    }
+}
+
+// Swap lane bits 2..4 with the register row index (8x8 blocks of 8 values)
+// through a 4 KB shared-memory region, two rounds of four values; the slot
+// function keeps every 128-bit store and load phase free of bank conflicts.
+__device__ __forceinline__ void warp_transpose(float (&v)[8][8], float4* scratch, int lane) {
+    const int a = lane >> 2, q = lane & 3;
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int s = 8 * (4 * k + (a >> 1)) + 2 * q + ((a ^ k) & 1);
+            scratch[s] = make_float4(v[k][4 * half], v[k][4 * half + 1], v[k][4 * half + 2], v[k][4 * half + 3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int h = 0; h < 8; ++h) {
+            const int s = 8 * (4 * a + (h >> 1)) + 2 * q + ((h ^ a) & 1);
+            const float4 t = scratch[s];
+            v[h][4 * half] = t.x;
+            v[h][4 * half + 1] = t.y;
+            v[h][4 * half + 2] = t.z;
+            v[h][4 * half + 3] = t.w;
+        }
+        __syncwarp();
+    }
+}
+
+// sign flip of 8 bf16 values held as 4 packed pairs, from 8 int8 signs
+__device__ __forceinline__ void apply_signs(unsigned (&r)[4], uint2 dv) {
+    r[0] ^= prmt(dv.x, 0u, 0x1404u) & 0x80008000u;
+    r[1] ^= prmt(dv.x, 0u, 0x3424u) & 0x80008000u;
+    r[2] ^= prmt(dv.y, 0u, 0x1404u) & 0x80008000u;
+    r[3] ^= prmt(dv.y, 0u, 0x3424u) & 0x80008000u;
+}
+
+__device__ __forceinline__ unsigned bf16_pm1(int neg) { return neg ? 0xBF80u : 0x3F80u; }
+
+struct HFrag {  // B fragments of H_16 for the two n-halves
+    unsigned b10, b11, b20, b21;
+};
+
+__device__ __forceinline__ HFrag make_hfrag(int lane) {
+    const int g = lane >> 2, q = lane & 3;
+    auto h = [](int k, int n) { return __popc(k & n) & 1; };
+    HFrag f;
+    f.b10 = bf16_pm1(h(2 * q, g)) | (bf16_pm1(h(2 * q + 1, g)) << 16);
+    f.b11 = bf16_pm1(h(2 * q + 8, g)) | (bf16_pm1(h(2 * q + 9, g)) << 16);
+    f.b20 = bf16_pm1(h(2 * q, g + 8)) | (bf16_pm1(h(2 * q + 1, g + 8)) << 16);
+    f.b21 = bf16_pm1(h(2 * q + 8, g + 8)) | (bf16_pm1(h(2 * q + 9, g + 8)) << 16);
+    return f;
+}
+
+// H_16 over element bits {0,1} and lane bits {0,1} of one row of 8 values
+// given as packed bf16 pairs (R0 = e0,e1 ... R3 = e6,e7).
+__device__ __forceinline__ void mma_h16(float (&o)[8], unsigned r0, unsigned r1, unsigned r2, unsigned r3,
+                                        const HFrag& f) {
+    float d1[4], d2[4];
+    mma_bf16_m16n8k16(d1, r0, r2, r1, r3, f.b10, f.b11);
+    mma_bf16_m16n8k16(d2, r0, r2, r1, r3, f.b20, f.b21);
+    o[0] = d1[0]; o[1] = d1[1]; o[4] = d1[2]; o[5] = d1[3];
+    o[2] = d2[0]; o[3] = d2[1]; o[6] = d2[2]; o[7] = d2[3];
+}
+
+// Forward transform of one window (8 chunks of 256 elements).  On return
+// v is in the transposed layout: lane (a, q), row h hold the group
+// g = 32 a + 4 h + q of the window.  Returns the lane's sum of squares.
+__device__ __forceinline__ float window_forward(float (&v)[8][8], const unsigned (&raw)[8][4], int logb, int nchunks,
+                                                float4* scratch, int lane, const HFrag& hf) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        if (k < nchunks) {
+            mma_h16(v[k], raw[k][0], raw[k][1], raw[k][2], raw[k][3], hf);
+        } else {
+#pragma unroll
+            for (int e = 0; e < 8; ++e) v[k][e] = 0.f;
+        }
+    }
+    stage_e2(v);
+    if (logb >= 9) stage_rows<1>(v);
+    if (logb >= 10) stage_rows<2>(v);
+    if (logb >= 11) stage_rows<4>(v);
+    warp_transpose(v, scratch, lane);
+    stage_rows<1>(v);
+    stage_rows<2>(v);
+    stage_rows<4>(v);
+    float ss = 0.f;
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) ss = fmaf(v[h][e], v[h][e], ss);
+    return ss;
+}
+
+__device__ __forceinline__ void load_window_raw(unsigned (&raw)[8][4], const uint16_t* src_smem_or_global,
+                                                bool from_global, const int8_t* signs, int cols, int col0, int nchunks,
+                                                int lane, unsigned long long& nonfinite) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        if (k < nchunks) {
+            const uint16_t* p = src_smem_or_global + 256 * k + 8 * lane;
+            uint4 q;
+            if (from_global) q = __ldg(reinterpret_cast<const uint4*>(p));
+            else q = *reinterpret_cast<const uint4*>(p);
+            raw[k][0] = q.x; raw[k][1] = q.y; raw[k][2] = q.z; raw[k][3] = q.w;
+            if (from_global) {  // slow path: non-finite values read as 0
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const unsigned x = raw[k][j];
+                    unsigned keep = 0xFFFFFFFFu;
+                    if ((x & 0x7F80u) == 0x7F80u) { keep &= 0xFFFF0000u; ++nonfinite; }
+                    if ((x & 0x7F800000u) == 0x7F800000u) { keep &= 0x0000FFFFu; ++nonfinite; }
+                    raw[k][j] = x & keep;
+                }
+            }
+            const int c = (col0 + 256 * k + 8 * lane) % cols;
+            apply_signs(raw[k], __ldg(reinterpret_cast<const uint2*>(signs + c)));
+        } else {
+            raw[k][0] = raw[k][1] = raw[k][2] = raw[k][3] = 0u;
+        }
+    }
+}
+
+// Escape search for one queued group (all lanes of the warp run this).
+__device__ __forceinline__ void resolve_queued(const uint32_t* e, const uint16_t* st1, const uint16_t* st2,
+                                               uint32_t* map, uint16_t* sidx, int16_t* ovf_scratch,
+                                               unsigned long long& clamped) {
+    const int g = static_cast<int>(e[0] & 0xFFFFu);
+    int P[8];
+    P[0] = static_cast<int16_t>(e[0] >> 16);
+    P[1] = static_cast<int16_t>(e[1] & 0xFFFFu);
+    P[2] = static_cast<int16_t>(e[1] >> 16);
+    P[3] = static_cast<int16_t>(e[2] & 0xFFFFu);
+    P[4] = static_cast<int16_t>(e[2] >> 16);
+    P[5] = static_cast<int16_t>(e[3] & 0xFFFFu);
+    P[6] = static_cast<int16_t>(e[3] >> 16);
+    P[7] = static_cast<int16_t>(e[4] & 0xFFFFu);
+    int R[8], Q[8];
+    best_escape_root(P, R);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) Q[i] = P[i] - R[i];
+    const int rq = core_rank(Q, st1, st2);
+    if (rq >= 0) {
+        const int rr = core_rank(R, st1, st2) - 1;
+        map[g] = static_cast<uint32_t>(rq) | (static_cast<uint32_t>(rr) << 16) | (1u << 24);
+        sidx[g] = static_cast<uint16_t>(rq);
+    } else {
+        map[g] = 2u << 24;
+        sidx[g] = 0;
+        uint4 o;
+        o.x = e[0] >> 16 | (e[1] << 16);
+        o.y = (e[1] >> 16) | (e[2] << 16);
+        o.z = (e[2] >> 16) | (e[3] << 16);
+        o.w = (e[3] >> 16) | (e[4] << 16);
+        *reinterpret_cast<uint4*>(ovf_scratch + 8 * g) = o;
+        if (e[4] & 0x10000u) ++clamped;
+    }
+}
+
+template <int MAXM>
+__device__ __forceinline__ FastTile make_tile(const EncodeParams<MAXM>& p, int t) {
+    FastTile ft;
+    ft.t = t;
+    ft.ne = ft.no = 0;
+    if (t < p.n_tiles) {
+        ft.mat = find_matrix(p, t);
+        const MatDesc& M = p.m[ft.mat];
+        const int rpt = meta_rpt(M.meta);
+        ft.r0 = (t - M.tile_base) * rpt;
+        ft.nr = min(rpt, M.rows - ft.r0);
+    } else {
+        ft.mat = 0;
+        ft.r0 = 0;
+        ft.nr = 0;
+    }
+    return ft;
+}
+
+template <int MAXM>
+__global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_constant__ EncodeParams<MAXM> p,
+                                                                  int16_t* __restrict__ ovf_scratch_all) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    uint16_t* inbuf = reinterpret_cast<uint16_t*>(smem + kFsIn);
+    uint16_t* st1 = reinterpret_cast<uint16_t*>(smem + kFsT1);
+    uint16_t* st2 = reinterpret_cast<uint16_t*>(smem + kFsT2);
+    uint32_t* smap = reinterpret_cast<uint32_t*>(smem + kFsMap);
+    uint16_t* sidx = reinterpret_cast<uint16_t*>(smem + kFsIdx);
+    float* sgss = reinterpret_cast<float*>(smem + kFsGss);
+    uint32_t* squeue = reinterpret_cast<uint32_t*>(smem + kFsQueue);
+    uint32_t* schunk = reinterpret_cast<uint32_t*>(smem + kFsChunk);
+
+    __shared__ __align__(8) uint64_t s_full[2];
+    __shared__ FastTile s_info[4];
+    __shared__ float s_rss[kMaxTileRows], s_rows[kMaxTileRows], s_rowc[kMaxTileRows], s_rowm[kMaxTileRows];
+    __shared__ float s_wss[kFastWarps];
+    __shared__ unsigned s_ex[3][2];
+
+    const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+    const bool service = warp == kFastWarps;
+    int16_t* ovf_scratch = ovf_scratch_all + static_cast<size_t>(blockIdx.x) * 3 * kFastTileGroups * 8;
+    unsigned long long* status = p.ws + 2;
+
+    {  // constant tables
+        const uint4* a = reinterpret_cast<const uint4*>(g_t1);
+        uint4* b = reinterpret_cast<uint4*>(st1);
+        for (int i = tid; i < (2 * 2401 * 7 * 2) / 16; i += kFastThreads) b[i] = a[i];
+        for (int i = ((2 * 2401 * 7 * 2) / 16) * 8 + tid; i < 2 * 2401 * 7; i += kFastThreads) st1[i] = g_t1[i];
+        for (int i = tid; i < 2 * 2401; i += kFastThreads) st2[i] = g_t2[i];
+    }
+    if (tid == 0) {
+        mbar_init(&s_full[0], 1);
+        mbar_init(&s_full[1], 1);
+        fence_mbar_init();
+        for (int s = 0; s < 4; ++s) s_info[s] = make_tile(p, 0x7FFFFFFF);
+        const int t0 = static_cast<int>(atomicAdd(&p.ws[0], 1ull));
+        s_info[0] = make_tile(p, t0);
+        if (t0 < p.n_tiles) {
+            const FastTile& ft = s_info[0];
+            const MatDesc& M = p.m[ft.mat];
+            const unsigned bytes = static_cast<unsigned>(ft.nr) * M.cols * 2u;
+            mbar_arrive_expect_tx(&s_full[0], bytes);
+            bulk_load(inbuf, static_cast<const uint16_t*>(M.w) + static_cast<size_t>(ft.r0) * M.cols, bytes,
+                      &s_full[0]);
+        }
+    }
+    __syncthreads();
+
+    const HFrag hf = make_hfrag(lane);
+    unsigned long long nonfinite = 0, clamped = 0;
+    int qhead = 0, qcount = 0;  // per-warp escape queue (warp-uniform)
+    uint32_t* myq = squeue + warp * kQueueCap * 5;
+
+    for (int i = 0;; ++i) {
+        const FastTile cur = s_info[i & 3];
+        const FastTile prev1 = s_info[(i + 3) & 3];
+        const FastTile prev2 = s_info[(i + 2) & 3];
+        const bool cur_ok = cur.t < p.n_tiles, p1_ok = i >= 1 && prev1.t < p.n_tiles,
+                   p2_ok = i >= 2 && prev2.t < p.n_tiles;
+        if (!cur_ok && !p1_ok && !p2_ok) break;
+        const int b = i & 1, msl = i % 3, msl2 = (i + 1) % 3;
+
+        if (!service) {
+            // ================================================ compute warps
+            if (cur_ok) {
+                const MatDesc& M = p.m[cur.mat];
+                const int C = M.cols, gpr = C >> 3, logb = meta_logb(M.meta);
+                const int n = cur.nr * C, G = cur.nr * gpr;
+                const int nwin = (n + 2047) >> 11;
+                const bool win_rows = (C & 2047) == 0;  // every window inside one row
+                {  // wait for the tile's bytes (bounded)
+                    int spins = 0;
+                    while (!mbar_try_wait(&s_full[b], (i >> 1) & 1)) {
+                        if (++spins > kWaitLimit) {
+                            if (lane == 0) atomicOr(&p.ctr->err, 2ull);
+                            break;
+                        }
+                    }
+                }
+                float v[8][8];
+                const int w = warp;
+                const int wbase = 2048 * w;
+                const int nchunks = max(0, min(8, (n - wbase) >> 8));
+                uint16_t* win = inbuf + b * kFastTileElems + wbase;
+                float4* scratch = reinterpret_cast<float4*>(win);
+                if (w < nwin) {
+                    unsigned raw[8][4];
+                    load_window_raw(raw, win, false, M.signs, C, wbase, nchunks, lane, nonfinite);
+                    __syncwarp();
+                    float ss = window_forward(v, raw, logb, nchunks, scratch, lane, hf);
+                    if (__any_sync(0xFFFFFFFFu, !isfinite(ss))) {  // non-finite input: redo from global, sanitised
+                        const uint16_t* g = static_cast<const uint16_t*>(M.w) + static_cast<size_t>(cur.r0) * C + wbase;
+                        load_window_raw(raw, g, true, M.signs, C, wbase, nchunks, lane, nonfinite);
+                        __syncwarp();
+                        ss = window_forward(v, raw, logb, nchunks, scratch, lane, hf);
+                    }
+                    if (win_rows) {
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
+                        if (lane == 0) s_wss[w] = ss;
+                    } else {
+                        const int a = lane >> 2, q = lane & 3;
+#pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            float gs = 0.f;
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) gs = fmaf(v[h][e], v[h][e], gs);
+                            if (a < nchunks) sgss[256 * w + 32 * a + 4 * h + q] = gs;
+                        }
+                    }
+                }
+                named_bar_sync(1, kFastWarps * 32);
+                // row scales
+                const float Bf = static_cast<float>(1 << logb);
+                if (win_rows) {
+                    if (tid < cur.nr) {
+                        const int wpr = C >> 11;
+                        float ssr = 0.f;
+                        for (int k = 0; k < wpr; ++k) ssr += s_wss[tid * wpr + k];
+                        s_rss[tid] = ssr;
+                    }
+                } else {
+                    for (int r = warp; r < cur.nr; r += kFastWarps) {
+                        float a = 0.f;
+                        for (int g = lane; g < gpr; g += 32) a += sgss[r * gpr + g];
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, off);
+                        if (lane == 0) s_rss[r] = a;
+                    }
+                }
+                named_bar_sync(1, kFastWarps * 32);
+                if (tid < cur.nr) {
+                    float s;
+                    if (p.scale_in) {
+                        s = M.scale[cur.r0 + tid];
+                        if (!(s > 0.f) || !isfinite(s)) s = 0.f;
+                    } else {
+                        s = sqrtf(s_rss[tid] / (Bf * static_cast<float>(C))) / p.kappa;
+                        M.scale[cur.r0 + tid] = s;
+                    }
+                    s_rows[tid] = s;
+                    s_rowc[tid] = (s > 0.f) ? 2.0f / (s * sqrtf(Bf)) : 0.f;
+                    s_rowm[tid] = s / sqrtf(Bf);
+                }
+                named_bar_sync(1, kFastWarps * 32);
+
+                // projection + encoding of the warp's 8 x 32 groups
+                uint32_t* map = smap + msl * kFastTileGroups;
+                uint16_t* idxs = sidx + b * kFastTileGroups;
+                int16_t* oscr = ovf_scratch + static_cast<size_t>(msl) * kFastTileGroups * 8;
+                if (w < nwin) {
+                    const int a = lane >> 2, q = lane & 3;
+                    const bool lane_ok = a < nchunks;
+                    const int row_w = win_rows ? (wbase / C) : 0;
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) {
+                        const int gw = 32 * a + 4 * h + q;
+                        const int gt = 256 * w + gw;
+                        const int row = win_rows ? row_w : (8 * gt) / C;
+                        const float c = s_rowc[lane_ok ? row : 0];
+                        float X[8];
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) X[e] = fminf(fmaxf(fmaf(v[h][e], c, 0.f), -1048576.f), 1048576.f);
+                        int P[8];
+                        e8_nearest_doubled(X, P);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v[h][e] = static_cast<float>(P[e]);  // keep P for dequant
+                        const int rk = lane_ok ? core_rank(P, st1, st2) : 0;
+                        const bool pend = lane_ok && rk < 0;
+                        if (lane_ok && !pend) {
+                            map[gt] = static_cast<uint32_t>(rk);
+                            idxs[gt] = static_cast<uint16_t>(rk);
+                        }
+                        const unsigned bal = __ballot_sync(0xFFFFFFFFu, pend);
+                        if (pend) {
+                            const int slot = (qhead + qcount + __popc(bal & lanemask_lt())) & (kQueueCap - 1);
+                            uint32_t* e = myq + 5 * slot;
+                            int Pc[8];
+                            bool clamp = false;
+#pragma unroll
+                            for (int k = 0; k < 8; ++k) {
+                                Pc[k] = max(-32768, min(32767, P[k]));
+                                clamp |= Pc[k] != P[k];
+                            }
+                            e[0] = static_cast<uint32_t>(gt) | (static_cast<uint32_t>(Pc[0] & 0xFFFF) << 16);
+                            e[1] = static_cast<uint32_t>(Pc[1] & 0xFFFF) | (static_cast<uint32_t>(Pc[2] & 0xFFFF) << 16);
+                            e[2] = static_cast<uint32_t>(Pc[3] & 0xFFFF) | (static_cast<uint32_t>(Pc[4] & 0xFFFF) << 16);
+                            e[3] = static_cast<uint32_t>(Pc[5] & 0xFFFF) | (static_cast<uint32_t>(Pc[6] & 0xFFFF) << 16);
+                            e[4] = static_cast<uint32_t>(Pc[7] & 0xFFFF) | (clamp ? 0x10000u : 0u);
+                        }
+                        qcount += __popc(bal);
+                        if (qcount >= 32) {
+                            __syncwarp();
+                            resolve_queued(myq + 5 * ((qhead + lane) & (kQueueCap - 1)), st1, st2, map, idxs, oscr,
+                                           clamped);
+                            qhead = (qhead + 32) & (kQueueCap - 1);
+                            qcount -= 32;
+                            __syncwarp();
+                        }
+                    }
+                    if (qcount > 0) {
+                        __syncwarp();
+                        if (lane < qcount)
+                            resolve_queued(myq + 5 * ((qhead + lane) & (kQueueCap - 1)), st1, st2, map, idxs, oscr,
+                                           clamped);
+                        qhead = (qhead + qcount) & (kQueueCap - 1);
+                        qcount = 0;
+                        __syncwarp();
+                    }
+
+                    // dequantised weights
+                    if (p.dq_mode == E8Q_DEQUANT_ROTATED) {
+                        uint16_t* dq = static_cast<uint16_t*>(M.dq) + static_cast<size_t>(cur.r0) * C;
+#pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            if (!lane_ok) continue;
+                            const int gt = 256 * w + 32 * a + 4 * h + q;
+                            const float s = s_rows[win_rows ? row_w : (8 * gt) / C];
+                            uint4 o;
+                            o.x = pack_bf16x2(bf16_of_product(s, 0.5f * v[h][0]), bf16_of_product(s, 0.5f * v[h][1]));
+                            o.y = pack_bf16x2(bf16_of_product(s, 0.5f * v[h][2]), bf16_of_product(s, 0.5f * v[h][3]));
+                            o.z = pack_bf16x2(bf16_of_product(s, 0.5f * v[h][4]), bf16_of_product(s, 0.5f * v[h][5]));
+                            o.w = pack_bf16x2(bf16_of_product(s, 0.5f * v[h][6]), bf16_of_product(s, 0.5f * v[h][7]));
+                            *reinterpret_cast<uint4*>(dq + 8 * gt) = o;
+                        }
+                    } else if (p.dq_mode == E8Q_DEQUANT_ORIGINAL) {
+                        // H(p) exactly: tensor-core stage on bf16 p = P/2 (split in two
+                        // bf16 terms when some |P| >= 256), fp32 butterflies for the rest.
+                        bool big = false;
+#pragma unroll
+                        for (int h = 0; h < 8; ++h)
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) big |= fabsf(v[h][e]) > 255.f;
+                        big = __any_sync(0xFFFFFFFFu, big);
+#pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            float o[8];
+                            unsigned r[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const __nv_bfloat162 t = __floats2bfloat162_rn(0.5f * v[h][2 * j], 0.5f * v[h][2 * j + 1]);
+                                r[j] = *reinterpret_cast<const unsigned*>(&t);
+                            }
+                            mma_h16(o, r[0], r[1], r[2], r[3], hf);
+                            if (big) {  // p = t0 + t1 + t2, each term exact in bf16 (24 bits)
+                                float rem[8];
+#pragma unroll
+                                for (int j = 0; j < 4; ++j) {
+                                    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&r[j]);
+                                    rem[2 * j] = 0.5f * v[h][2 * j] - __bfloat162float(hi.x);
+                                    rem[2 * j + 1] = 0.5f * v[h][2 * j + 1] - __bfloat162float(hi.y);
+                                }
+#pragma unroll
+                                for (int term = 0; term < 2; ++term) {
+#pragma unroll
+                                    for (int j = 0; j < 4; ++j) {
+                                        const __nv_bfloat162 t = __floats2bfloat162_rn(rem[2 * j], rem[2 * j + 1]);
+                                        r[j] = *reinterpret_cast<const unsigned*>(&t);
+                                        rem[2 * j] -= __bfloat162float(t.x);
+                                        rem[2 * j + 1] -= __bfloat162float(t.y);
+                                    }
+                                    float o2[8];
+                                    mma_h16(o2, r[0], r[1], r[2], r[3], hf);
+#pragma unroll
+                                    for (int e = 0; e < 8; ++e) o[e] += o2[e];
+                                }
+                            }
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) v[h][e] = o[e];
+                        }
+                        stage_e2(v);
+                        stage_rows<1>(v);
+                        stage_rows<2>(v);
+                        stage_rows<4>(v);
+                        warp_transpose(v, scratch, lane);
+                        if (logb >= 9) stage_rows<1>(v);
+                        if (logb >= 10) stage_rows<2>(v);
+                        if (logb >= 11) stage_rows<4>(v);
+                        uint16_t* dq = static_cast<uint16_t*>(M.dq) + static_cast<size_t>(cur.r0) * C;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) {
+                            if (k >= nchunks) continue;
+                            const int te = wbase + 256 * k + 8 * lane;  // tile element of the 8-run
+                            const float m = s_rowm[win_rows ? row_w : te / C];
+                            unsigned o[4];
+#pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const __nv_bfloat162 t = __floats2bfloat162_rn(v[k][2 * j] * m, v[k][2 * j + 1] * m);
+                                o[j] = *reinterpret_cast<const unsigned*>(&t);
+                            }
+                            apply_signs(o, __ldg(reinterpret_cast<const uint2*>(M.signs + te % C)));
+                            *reinterpret_cast<uint4*>(dq + te) = make_uint4(o[0], o[1], o[2], o[3]);
+                        }
+                    }
+                }
+                named_bar_sync(1, kFastWarps * 32);
+                // per-chunk record counts and their prefix (group order)
+                uint32_t* cnt = schunk + msl * 130;
+                const int nch = (G + 31) >> 5;
+                for (int c = warp; c < nch; c += kFastWarps) {
+                    const int g = 32 * c + lane;
+                    const uint32_t k = g < G ? (map[g] >> 24) : 0u;
+                    const unsigned be = __ballot_sync(0xFFFFFFFFu, k == 1), bo = __ballot_sync(0xFFFFFFFFu, k == 2);
+                    if (lane == 0) {
+                        cnt[c] = __popc(be);
+                        cnt[65 + c] = __popc(bo);
+                    }
+                }
+                named_bar_sync(1, kFastWarps * 32);
+                if (warp == 0) {
+                    unsigned ce0 = lane < nch ? cnt[lane] : 0u, ce1 = lane + 32 < nch ? cnt[lane + 32] : 0u;
+                    unsigned co0 = lane < nch ? cnt[65 + lane] : 0u, co1 = lane + 32 < nch ? cnt[65 + lane + 32] : 0u;
+                    unsigned se0 = ce0, se1 = ce1, so0 = co0, so1 = co1;  // inclusive scans
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const unsigned a0 = __shfl_up_sync(0xFFFFFFFFu, se0, off), a1 = __shfl_up_sync(0xFFFFFFFFu, se1, off);
+                        const unsigned b0 = __shfl_up_sync(0xFFFFFFFFu, so0, off), b1 = __shfl_up_sync(0xFFFFFFFFu, so1, off);
+                        if (lane >= off) { se0 += a0; se1 += a1; so0 += b0; so1 += b1; }
+                    }
+                    const unsigned te0 = __shfl_sync(0xFFFFFFFFu, se0, 31), to0 = __shfl_sync(0xFFFFFFFFu, so0, 31);
+                    const unsigned te1 = __shfl_sync(0xFFFFFFFFu, se1, 31), to1 = __shfl_sync(0xFFFFFFFFu, so1, 31);
+                    cnt[lane] = se0 - ce0;
+                    cnt[lane + 32] = te0 + se1 - ce1;
+                    cnt[65 + lane] = so0 - co0;
+                    cnt[65 + lane + 32] = to0 + so1 - co1;
+                    if (lane == 0) {
+                        cnt[64] = te0 + te1;
+                        cnt[65 + 64] = to0 + to1;
+                        s_info[i & 3].ne = te0 + te1;
+                        s_info[i & 3].no = to0 + to1;
+                    }
+                }
+            }
+            // emit the records of the tile finished two iterations ago, once
+            // the service warp has placed it
+            named_bar_sync(2, kFastThreads);
+            if (p2_ok) {
+                const MatDesc& M = p.m[prev2.mat];
+                const int gpr = M.cols >> 3, G = prev2.nr * gpr, nch = (G + 31) >> 5;
+                const uint32_t* map = smap + msl2 * kFastTileGroups;
+                const uint32_t* cnt = schunk + msl2 * 130;
+                const int16_t* oscr = ovf_scratch + static_cast<size_t>(msl2) * kFastTileGroups * 8;
+                const long long ex_e = s_ex[msl2][0], ex_o = s_ex[msl2][1];
+                const uint32_t gid0 = M.group_base + static_cast<uint32_t>(prev2.r0) * gpr;
+                for (int c = warp; c < nch; c += kFastWarps) {
+                    const int g = 32 * c + lane;
+                    const uint32_t m = g < G ? map[g] : 0u;
+                    const uint32_t k = m >> 24;
+                    const unsigned be = __ballot_sync(0xFFFFFFFFu, k == 1), bo = __ballot_sync(0xFFFFFFFFu, k == 2);
+                    if (k == 1) {
+                        const long long pos = ex_e + cnt[c] + __popc(be & lanemask_lt());
+                        if (pos < p.esc_cap) {
+                            e8q_escape r;
+                            r.group = gid0 + g;
+                            r.core = static_cast<uint16_t>(m & 0xFFFFu);
+                            r.root = static_cast<uint8_t>((m >> 16) & 0xFFu);
+                            r.reserved = 0;
+                            p.esc[pos] = r;
+                        }
+                    } else if (k == 2) {
+                        const long long pos = ex_o + cnt[65 + c] + __popc(bo & lanemask_lt());
+                        if (pos < p.ovf_cap) {
+                            const uint4 cw = *reinterpret_cast<const uint4*>(oscr + 8 * g);
+                            uint32_t* dst = reinterpret_cast<uint32_t*>(p.ovf + pos);
+                            dst[0] = gid0 + g;
+                            dst[1] = cw.x; dst[2] = cw.y; dst[3] = cw.z; dst[4] = cw.w;
+                        }
+                    }
+                }
+                if (tid < prev2.nr) {
+                    const int c = (tid * gpr) >> 5;  // rows start on chunk boundaries (gpr % 32 == 0)
+                    if (p.esc_rp) p.esc_rp[M.row_base + prev2.r0 + tid] = ex_e + cnt[c];
+                    if (p.ovf_rp) p.ovf_rp[M.row_base + prev2.r0 + tid] = ex_o + cnt[65 + c];
+                }
+                if (prev2.t == p.n_tiles - 1 && tid == 0) {
+                    const long long te = ex_e + cnt[64], to = ex_o + cnt[65 + 64];
+                    if (p.esc_rp) p.esc_rp[p.total_rows] = te;
+                    if (p.ovf_rp) p.ovf_rp[p.total_rows] = to;
+                    p.ctr->n_escape = te;
+                    p.ctr->n_overflow = to;
+                    p.ctr->n_dropped = (te > p.esc_cap ? te - p.esc_cap : 0) + (to > p.ovf_cap ? to - p.ovf_cap : 0);
+                }
+            }
+            fence_proxy_async_smem();
+        } else {
+            // ================================================= service warp
+            if (lane == 0) {
+                int tn = 0x7FFFFFFF;
+                if (cur_ok) tn = static_cast<int>(atomicAdd(&p.ws[0], 1ull));
+                const FastTile nt = make_tile(p, tn);
+                s_info[(i + 1) & 3] = nt;
+                if (tn < p.n_tiles) {
+                    const MatDesc& M = p.m[nt.mat];
+                    const unsigned bytes = static_cast<unsigned>(nt.nr) * M.cols * 2u;
+                    uint64_t* bar = &s_full[(i + 1) & 1];
+                    mbar_arrive_expect_tx(bar, bytes);
+                    bulk_load(inbuf + ((i + 1) & 1) * kFastTileElems,
+                              static_cast<const uint16_t*>(M.w) + static_cast<size_t>(nt.r0) * M.cols, bytes, bar);
+                }
+                if (p1_ok) {
+                    const MatDesc& M = p.m[prev1.mat];
+                    const int gpr = M.cols >> 3;
+                    const unsigned long long own =
+                        (static_cast<unsigned long long>(prev1.ne) << 31) | prev1.no;
+                    st_volatile_u64(&status[prev1.t], (prev1.t == 0 ? (2ull << 62) : (1ull << 62)) | own);
+                    bulk_store(M.idx + static_cast<size_t>(prev1.r0) * gpr, sidx + ((i + 1) & 1) * kFastTileGroups,
+                               static_cast<unsigned>(prev1.nr) * gpr * 2u);
+                    bulk_commit();
+                }
+            }
+            __syncwarp();
+            if (p2_ok) {
+                unsigned ex_e = 0, ex_o = 0;
+                if (prev2.t > 0) {
+                    unsigned acc_e = 0, acc_o = 0;
+                    int j = prev2.t - 1, spins = 0;
+                    while (true) {
+                        const int k = j - lane;
+                        const unsigned long long s = (k >= 0) ? ld_volatile_u64(&status[k]) : (2ull << 62);
+                        const unsigned flag = static_cast<unsigned>(s >> 62);
+                        const unsigned notready = __ballot_sync(0xFFFFFFFFu, flag == 0);
+                        const unsigned ispre = __ballot_sync(0xFFFFFFFFu, flag == 2);
+                        const unsigned window = ispre ? (((ispre & (0u - ispre)) << 1) - 1u) : 0xFFFFFFFFu;
+                        if (notready & window) {
+                            if (++spins > kSpinLimit) {
+                                if (lane == 0) atomicOr(&p.ctr->err, 1ull);
+                                break;
+                            }
+                            __nanosleep(64);
+                            continue;
+                        }
+                        const bool in = (window >> lane) & 1u;
+                        unsigned ve = in ? static_cast<unsigned>((s >> 31) & 0x7FFFFFFFu) : 0u;
+                        unsigned vo = in ? static_cast<unsigned>(s & 0x7FFFFFFFu) : 0u;
+#pragma unroll
+                        for (int off = 16; off > 0; off >>= 1) {
+                            ve += __shfl_xor_sync(0xFFFFFFFFu, ve, off);
+                            vo += __shfl_xor_sync(0xFFFFFFFFu, vo, off);
+                        }
+                        acc_e += ve;
+                        acc_o += vo;
+                        if (ispre) break;
+                        j -= 32;
+                    }
+                    ex_e = acc_e;
+                    ex_o = acc_o;
+                    if (lane == 0)
+                        st_volatile_u64(&status[prev2.t],
+                                        (2ull << 62) |
+                                            (static_cast<unsigned long long>((ex_e + prev2.ne) & 0x7FFFFFFFu) << 31) |
+                                            ((ex_o + prev2.no) & 0x7FFFFFFFu));
+                }
+                if (lane == 0) {
+                    s_ex[msl2][0] = ex_e;
+                    s_ex[msl2][1] = ex_o;
+                }
+            }
+            named_bar_sync(2, kFastThreads);
+            if (lane == 0) bulk_wait_read_all();
+            __syncwarp();
+        }
+        __syncthreads();
+    }
+    if (service && lane == 0) bulk_wait_all();
+
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+        nonfinite += __shfl_xor_sync(0xFFFFFFFFu, nonfinite, off);
+        clamped += __shfl_xor_sync(0xFFFFFFFFu, clamped, off);
+    }
+    if (lane == 0) {
+        if (nonfinite) atomicAdd(&p.ctr->n_nonfinite, nonfinite);
+        if (clamped) atomicAdd(&p.ctr->n_clamped, clamped);
+    }
+}
+
+}  // namespace e8q

@@ -8,8 +8,8 @@ Tolerances (derived in the design notes):
 * scales: relative 1e-5 (fp32 transform and sum against fp64);
 * rotated-domain dequant: bit-exact given the GPU's indices, records, scale;
 * original-basis dequant: <= 1 bf16 ulp of the fp64 value, plus 2^-20 s_r;
-* GEMV: max|y - y_ref| / rms(y_ref) <= 1e-2 per batch row and
-  ||y - y_ref|| / ||y_ref|| <= 1e-2.
+* GEMV: ||y - y_ref|| / ||y_ref|| <= 1e-2, and each output within its bf16
+  rounding (2^-8 |y_ref|) plus 1e-3 rms(y_ref) of its batch row.
 """
 import numpy as np
 
@@ -99,11 +99,14 @@ def check_original_dequant(bits_gpu, P_gpu, scale_gpu, signs, block, label=""):
 
 
 def check_gemv(y_gpu, y_ref, label=""):
+    """Normwise relative error <= 1e-2 (the stated GEMV bound), and every
+    element within its bf16 output rounding (2^-8 relative) plus 1e-3 of
+    the row's rms for the fp32 accumulation."""
     y = synth.bf16_bits_to_f64(np.asarray(y_gpu).view(np.uint16)).reshape(y_ref.shape)
     for b in range(y_ref.shape[0]):
         rms = np.sqrt((y_ref[b] ** 2).mean())
-        worst = np.abs(y[b] - y_ref[b]).max() / rms
-        assert worst <= 1e-2, f"{label}: batch row {b} max error {worst:.3g} of rms"
+        excess = np.abs(y[b] - y_ref[b]) - (2.0 ** -8 * np.abs(y_ref[b]) + 1e-3 * rms)
+        assert excess.max() <= 0, f"{label}: batch row {b}: {int((excess > 0).sum())} outputs beyond bf16 rounding"
     rel = np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref)
     assert rel <= 1e-2, f"{label}: relative error {rel:.3g}"
     return rel

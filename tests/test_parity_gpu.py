@@ -38,13 +38,19 @@ def host_idx(t):
 
 
 def run_encode(e8q, mats, signs, blocks=0, kappa=1.0, dequant="none", scales=None, dtype=torch.bfloat16,
-               esc_cap=None, ovf_cap=None):
+               esc_cap=None, ovf_cap=None, allow_drop=False):
     ws = [dev_bf16(m) if dtype == torch.bfloat16 else dev(m.astype(np.float32)) for m in mats]
     ss = [dev(s) for s in signs]
     sc = [dev(s.astype(np.float32)) for s in scales] if scales is not None else None
+    groups = sum(m.shape[0] * (m.shape[1] // 8) for m in mats)
+    esc_cap = max(64, groups) if esc_cap is None else esc_cap
+    ovf_cap = max(64, groups) if ovf_cap is None else ovf_cap
     enc = e8q.Encoder([w.shape for w in ws], ss, dtype, blocks, kappa, dequant, scales is not None, esc_cap, ovf_cap)
     res = enc(ws, sc)
     torch.cuda.synchronize()
+    ctr = res.read_counters()
+    assert ctr["err"] == 0, ctr
+    assert allow_drop or ctr["n_dropped"] == 0, ctr
     return enc, res
 
 
@@ -206,6 +212,75 @@ def test_nonfinite_and_zero_rows(e8q):
     assert res.scale[0].cpu().numpy()[3] == 0.0 and (host_idx(res.idx[0])[3] == 0).all()
 
 
+def test_bf16_tiles_dequant_both_bases(e8q):
+    """256-wide bf16 rows (64 rows per tile) with both dequant outputs."""
+    rng = np.random.default_rng(21)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((200, 256)) * 0.02)
+    d = synth.signs(21, 256)
+    for mode in ("rotated", "original"):
+        enc, res = run_encode(e8q, [w], [d], 0, dequant=mode)
+        st = compare_all(e8q, res, [w], [d], [256], label=f"bf16 256 {mode}")[0]
+        dq = res.dequant[0].cpu().view(torch.int16).numpy()
+        scale = res.scale[0].cpu().numpy()
+        if mode == "rotated":
+            check_rotated_dequant(dq, st["points"], scale, d, 256, "rotated")
+        else:
+            check_original_dequant(dq, st["points"], scale, d, 256, "original")
+        out = e8q.e8q_decode(res.encoded[0], mode).cpu().view(torch.int16).numpy()
+        np.testing.assert_array_equal(out, dq)  # decode reproduces the encode-time output bit for bit
+
+
+def test_bf16_nonfinite_inputs(e8q):
+    rng = np.random.default_rng(22)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((8, 2048)) * 0.02)
+    w[1, 5] = 0x7FC0   # NaN
+    w[3, 100] = 0x7F80  # +Inf
+    w[3, 2000] = 0xFF80  # -Inf
+    w[6] = 0           # zero row
+    d = synth.signs(22, 2048)
+    enc, res = run_encode(e8q, [w], [d], 0, dequant="original")
+    assert res.read_counters()["n_nonfinite"] == 3
+    vals = synth.bf16_bits_to_f64(w)
+    out = oracle.project_encode(vals, d, 2048)
+    assert out["nonfinite"] == 3
+    st = check_encode(out, host_idx(res.idx[0]), res.scale[0].cpu().numpy(), res.escape_records(),
+                      res.overflow_records(), 0, None, 256, "bf16 nonfinite")
+    check_original_dequant(res.dequant[0].cpu().view(torch.int16).numpy(), st["points"], res.scale[0].cpu().numpy(),
+                           d, 2048, "nonfinite original")
+
+
+def test_large_points_small_scale(e8q):
+    """kappa = 200: |x| in the hundreds, lattice points far outside the core
+    (overflow records with large coordinates) and the original-basis dequant
+    of large |P|."""
+    rng = np.random.default_rng(23)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((4, 2048)) * 0.02)
+    d = synth.signs(23, 2048)
+    enc, res = run_encode(e8q, [w], [d], 0, kappa=200.0, dequant="original")
+    st = compare_all(e8q, res, [w], [d], [2048], kappa=200.0, label="kappa200")[0]
+    assert np.abs(st["points"]).max() > 255
+    check_original_dequant(res.dequant[0].cpu().view(torch.int16).numpy(), st["points"], res.scale[0].cpu().numpy(),
+                           d, 2048, "kappa200 original")
+
+
+def test_bf16_capacity_and_scale_in(e8q):
+    w, d = synth.attn_2048()
+    _, full = run_encode(e8q, [w], [d], 0)
+    tot = full.read_counters()
+    ref_e, ref_o = full.escape_records().copy(), full.overflow_records().copy()
+    ref_rp = full.esc_row_ptr.cpu().numpy().copy()
+    _, res = run_encode(e8q, [w], [d], 0, esc_cap=1000, ovf_cap=10, allow_drop=True)
+    ctr = res.read_counters()
+    assert ctr["n_dropped"] == (tot["n_escape"] - 1000) + (tot["n_overflow"] - 10)
+    np.testing.assert_array_equal(res.escape_records()[:1000], ref_e[:1000])
+    np.testing.assert_array_equal(res.overflow_records()[:10], ref_o[:10])
+    np.testing.assert_array_equal(res.esc_row_ptr.cpu().numpy(), ref_rp)
+    s = full.scale[0].cpu().numpy()
+    _, given = run_encode(e8q, [w], [d], 0, scales=[s])
+    np.testing.assert_array_equal(host_idx(given.idx[0]), host_idx(full.idx[0]))
+    assert given.escape_records().tobytes() == ref_e.tobytes()
+
+
 def test_empty_matrix(e8q):
     d = synth.signs(1, 64)
     enc, res = run_encode(e8q, [np.zeros((0, 64), np.uint16)], [d], 0)
@@ -220,7 +295,7 @@ def test_capacity_shortfall_is_reported(e8q):
     ref_e = full.escape_records().copy()
     ref_rp = full.esc_row_ptr.cpu().numpy().copy()
     tot = full.read_counters()
-    _, res = run_encode(e8q, [w], [d], 0, dtype=torch.float32, esc_cap=5, ovf_cap=0)
+    _, res = run_encode(e8q, [w], [d], 0, dtype=torch.float32, esc_cap=5, ovf_cap=0, allow_drop=True)
     ctr = res.read_counters()
     assert ctr["n_escape"] == tot["n_escape"] and ctr["n_overflow"] == tot["n_overflow"]
     assert ctr["n_dropped"] == (tot["n_escape"] - 5) + tot["n_overflow"]
@@ -234,8 +309,6 @@ def test_scale_in(e8q):
     enc, res = run_encode(e8q, [w], [d], 0, dtype=torch.float32, scales=[s.astype(np.float32)])
     # the oracle with a fixed scale: kappa chosen so that rms / kappa == s
     s32 = s.astype(np.float32).astype(np.float64)
-    out = oracle.project_encode(w.astype(np.float64), d, 256, kappa=1.0)
-    rms = out["scale"]
     out = oracle.project_encode(w.astype(np.float64), d, 256, kappa=1.0 / 0.75)
     np.testing.assert_allclose(res.scale[0].cpu().numpy(), s32, rtol=0)
     np.testing.assert_allclose(out["scale"], s32, rtol=1e-6)
@@ -267,3 +340,68 @@ def test_gemv_small(e8q, batch):
     y_ref = oracle.gemv(st["points"], res.scale[0].cpu().numpy().astype(np.float64), d, 2048,
                         synth.bf16_bits_to_f64(xb))
     check_gemv(y.cpu().view(torch.int16).numpy(), y_ref, f"gemv b={batch}")
+
+
+# ----------------------------------------------------------------------
+# full-size workloads, in the launch configuration bench.py times
+# ----------------------------------------------------------------------
+@pytest.fixture(scope="module")
+def mlp_full(e8q):
+    (up, d_up), (down, d_dn) = synth.mlp_14336()
+    G = 4096 * (14336 // 8) + 14336 * (4096 // 8)
+    W = [dev_bf16(up), dev_bf16(down)]
+    S = [dev(d_up), dev(d_dn)]
+    enc = e8q.Encoder([(4096, 14336), (14336, 4096)], S, torch.bfloat16, 0, 1.0, "original", esc_cap=G // 2,
+                      ovf_cap=G // 16)
+    res = enc(W)
+    torch.cuda.synchronize()
+    return dict(up=up, down=down, d_up=d_up, d_dn=d_dn, res=res, enc=enc, W=W)
+
+
+def test_mlp_full_size_sampled_rows(e8q, mlp_full):
+    res = mlp_full["res"]
+    ctr = res.read_counters()
+    assert ctr["err"] == 0 and ctr["n_dropped"] == 0
+    rng = np.random.default_rng(123)
+    rows = [np.sort(rng.choice(4096, 6, replace=False)), np.sort(rng.choice(14336, 6, replace=False))]
+    mats = [mlp_full["up"], mlp_full["down"]]
+    signs = [mlp_full["d_up"], mlp_full["d_dn"]]
+    stats = compare_all(e8q, res, mats, signs, [2048, 2048], rows=rows, label="mlp")
+    for i, st in enumerate(stats):
+        dq = res.dequant[i].cpu().view(torch.int16).numpy()[rows[i]]
+        check_original_dequant(dq, st["points"], res.scale[i].cpu().numpy()[rows[i]], signs[i], 2048,
+                               f"mlp[{i}] original")
+    rp = res.esc_row_ptr.cpu().numpy()
+    assert rp[0] == 0 and (np.diff(rp) >= 0).all() and rp[-1] == ctr["n_escape"]
+
+
+@pytest.mark.parametrize("batch", [1, 4, 16, 64])
+def test_gemv_full_size(e8q, mlp_full, batch):
+    res = mlp_full["res"]
+    m = res.encoded[0]
+    idx = host_idx(res.idx[0]).reshape(-1)
+    P, _, _, _, _ = gpu_points(idx, res.escape_records(), res.overflow_records(), idx.size, 0)
+    xb = synth.gemv_x(batch, 14336)
+    y = e8q.Gemv(m, batch)(dev_bf16(xb))
+    torch.cuda.synchronize()
+    y_ref = oracle.gemv(P, res.scale[0].cpu().numpy().astype(np.float64), mlp_full["d_up"], 2048,
+                        synth.bf16_bits_to_f64(xb))
+    check_gemv(y.cpu().view(torch.int16).numpy(), y_ref, f"gemv full b={batch}")
+
+
+def test_moe_bank_full_size_sampled(e8q):
+    """All 384 expert matrices (604M weights) in one launch; two rows of
+    every eighth matrix checked against the oracle."""
+    mats = synth.moe_bank()
+    W = [m for m, _ in mats]
+    S = [s for _, s in mats]
+    G = sum(m.shape[0] * (m.shape[1] // 8) for m in W)
+    enc, res = run_encode(e8q, W, S, 0, esc_cap=G // 2, ovf_cap=G // 16)
+    esc, ovf = res.escape_records(), res.overflow_records()
+    rng = np.random.default_rng(7)
+    for i in range(0, len(W), 8):
+        C = W[i].shape[1]
+        rsel = np.sort(rng.choice(W[i].shape[0], 2, replace=False))
+        out = oracle.project_encode(synth.bf16_bits_to_f64(W[i][rsel]), S[i], oracle.default_block(C))
+        check_encode(out, host_idx(res.idx[i]), res.scale[i].cpu().numpy(), esc, ovf, res.group_base[i], rsel, C // 8,
+                     label=f"moe[{i}]")
