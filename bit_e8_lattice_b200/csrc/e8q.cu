@@ -142,6 +142,7 @@ const char* e8q_status_string(e8q_status s) {
         case E8Q_ERR_UNSUPPORTED: return "unsupported";
         case E8Q_ERR_CUDA: return "cuda error";
         case E8Q_ERR_WORKSPACE: return "workspace too small";
+        case E8Q_ERR_SCRATCH_LIMIT: return "problem too large for the built-in scratch of e8q_project_encode_noalloc";
     }
     return "unknown status";
 }
@@ -360,3 +361,115 @@ e8q_status e8q_dequant_gemv(const e8q_encoded* m, const void* x_bf16, int32_t ba
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------
+// Encode with a built-in scratch (no allocation by the library or caller)
+// ---------------------------------------------------------------------
+namespace e8q {
+namespace {
+// Ticket and tile-status words of the encode kernel, for callers that cannot
+// allocate.  Host code must not pass this name to a kernel: on the host it is
+// only a stand-in; the device address comes from cudaGetSymbolAddress.
+constexpr size_t kNoAllocScratchBytes = size_t{2} << 20;
+static __device__ __align__(256) unsigned long long g_noalloc_scratch[kNoAllocScratchBytes / 8];
+std::mutex g_noalloc_mu;
+void* g_noalloc_addr[kMaxDevices];
+}  // namespace
+}  // namespace e8q
+
+extern "C" e8q_status e8q_project_encode_noalloc(const e8q_matrix* mats, int32_t n_mats, const e8q_encode_args* a,
+                                                 e8q_stream stream) {
+    if (!mats || !a || n_mats < 1) return E8Q_ERR_INVALID_ARG;
+    if (n_mats > kMaxMats) return E8Q_ERR_UNSUPPORTED;
+    if (!a->counters || !(a->kappa > 0.f) || !std::isfinite(a->kappa)) return E8Q_ERR_INVALID_ARG;
+    if (a->dequant < E8Q_DEQUANT_NONE || a->dequant > E8Q_DEQUANT_ORIGINAL) return E8Q_ERR_INVALID_ARG;
+    if (a->esc_cap < 0 || a->ovf_cap < 0 || (a->esc_cap > 0 && !a->esc) || (a->ovf_cap > 0 && !a->ovf))
+        return E8Q_ERR_INVALID_ARG;
+    if (a->scale_in != 0 && a->scale_in != 1) return E8Q_ERR_INVALID_ARG;
+
+    static thread_local EncodeParams<kMaxMats> P;
+    std::memset(&P, 0, sizeof(P));
+    int64_t tiles = 0, rows_total = 0, groups_total = 0;
+    for (int i = 0; i < n_mats; ++i) {
+        const e8q_matrix& m = mats[i];
+        if (m.rows < 0 || !valid_cols(m.cols)) return E8Q_ERR_INVALID_ARG;
+        if (m.cols > kMaxCols) return E8Q_ERR_UNSUPPORTED;
+        const int logb = resolve_logb(m.cols, m.rht_block);
+        if (logb < 0) return E8Q_ERR_INVALID_ARG;
+        if (m.in_dtype != E8Q_F32 && m.in_dtype != E8Q_BF16) return E8Q_ERR_INVALID_ARG;
+        if (m.rows > 0) {
+            if (!m.w || !m.signs || !m.idx || !m.scale) return E8Q_ERR_INVALID_ARG;
+            if (!aligned(m.w, 16) || !aligned(m.signs, 8) || !aligned(m.idx, 2) || !aligned(m.scale, 4))
+                return E8Q_ERR_INVALID_ARG;
+            if (a->dequant != E8Q_DEQUANT_NONE && (!m.dequant || !aligned(m.dequant, 16))) return E8Q_ERR_INVALID_ARG;
+        }
+        const int rpt = rows_per_tile(static_cast<int>(m.cols));
+        MatDesc& d = P.m[i];
+        d.w = m.w;
+        d.signs = m.signs;
+        d.idx = m.idx;
+        d.scale = m.scale;
+        d.dq = m.dequant;
+        d.rows = static_cast<int32_t>(m.rows);
+        d.cols = static_cast<int32_t>(m.cols);
+        d.meta = logb | ((m.in_dtype == E8Q_BF16) ? 16 : 0) | (rpt << 8);
+        d.tile_base = static_cast<int32_t>(tiles);
+        d.row_base = static_cast<int32_t>(rows_total);
+        d.group_base = static_cast<uint32_t>(groups_total);
+        tiles += (m.rows + rpt - 1) / rpt;
+        rows_total += m.rows;
+        groups_total += m.rows * (m.cols / 8);
+        if (groups_total >= (int64_t{1} << 31) || rows_total >= (int64_t{1} << 31)) return E8Q_ERR_UNSUPPORTED;
+    }
+    const size_t need = 16 + 8 * static_cast<size_t>(tiles);
+    if (need > kNoAllocScratchBytes) return E8Q_ERR_SCRATCH_LIMIT;
+
+    int dev;
+    e8q_status st = ensure_device(&dev);
+    if (st != E8Q_OK) return st;
+    void* scratch = nullptr;
+    {
+        std::lock_guard<std::mutex> lock(g_noalloc_mu);
+        if (!g_noalloc_addr[dev]) {
+            void* p = nullptr;
+            if (cudaGetSymbolAddress(&p, g_noalloc_scratch) != cudaSuccess || !p) return E8Q_ERR_CUDA;
+            g_noalloc_addr[dev] = p;
+        }
+        scratch = g_noalloc_addr[dev];
+    }
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    st = cuda_ok(cudaMemsetAsync(a->counters, 0, sizeof(e8q_counters), s));
+    if (st == E8Q_OK) st = cuda_ok(cudaMemsetAsync(scratch, 0, need, s));
+    if (st != E8Q_OK) return st;
+    if (tiles == 0) {
+        if (a->esc_row_ptr) st = cuda_ok(cudaMemsetAsync(a->esc_row_ptr + rows_total, 0, sizeof(int64_t), s));
+        if (st == E8Q_OK && a->ovf_row_ptr)
+            st = cuda_ok(cudaMemsetAsync(a->ovf_row_ptr + rows_total, 0, sizeof(int64_t), s));
+        return st;
+    }
+    P.esc = a->esc;
+    P.ovf = a->ovf;
+    P.esc_rp = a->esc_row_ptr;
+    P.ovf_rp = a->ovf_row_ptr;
+    P.ctr = a->counters;
+    P.ws = static_cast<unsigned long long*>(scratch);
+    P.esc_cap = a->esc_cap;
+    P.ovf_cap = a->ovf_cap;
+    P.kappa = a->kappa;
+    P.dq_mode = a->dequant;
+    P.scale_in = a->scale_in;
+    P.n_mats = n_mats;
+    P.n_tiles = static_cast<int32_t>(tiles);
+    P.total_rows = static_cast<int32_t>(rows_total);
+    const int grid = static_cast<int>(tiles < g_sms[dev] ? tiles : g_sms[dev]);
+    if (n_mats == 1) {
+        EncodeParams<1> P1;
+        std::memcpy(&P1, &P, offsetof(EncodeParams<1>, m));
+        P1.m[0] = P.m[0];
+        k_encode<1><<<grid, kEncThreads, kEncSmemBytes, s>>>(P1);
+    } else {
+        k_encode<kMaxMats><<<grid, kEncThreads, kEncSmemBytes, s>>>(P);
+    }
+    return cuda_ok(cudaGetLastError());
+}
+

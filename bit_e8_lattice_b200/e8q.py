@@ -73,6 +73,8 @@ def lib():
         L.e8q_encode_workspace_bytes.restype = sz
         L.e8q_project_encode.argtypes = [ctypes.POINTER(Matrix), i32, ctypes.POINTER(EncodeArgs), vp, sz, vp]
         L.e8q_project_encode.restype = ctypes.c_int
+        L.e8q_project_encode_noalloc.argtypes = [ctypes.POINTER(Matrix), i32, ctypes.POINTER(EncodeArgs), vp]
+        L.e8q_project_encode_noalloc.restype = ctypes.c_int
         L.e8q_decode.argtypes = [ctypes.POINTER(EncodedC), i32, vp, vp]
         L.e8q_decode.restype = ctypes.c_int
         L.e8q_gemv_workspace_bytes.argtypes = [ctypes.POINTER(EncodedC), i32]
@@ -244,6 +246,22 @@ class Encoder:
                                       ctypes.c_void_p(self.workspace.data_ptr()), self.workspace.numel(),
                                       _stream_handle(stream))
         _check(rc, "e8q_project_encode")
+        return self.result()
+
+    def run_noalloc(self, weights: Sequence[torch.Tensor], stream=None) -> EncodeResult:
+        """Same encode through e8q_project_encode_noalloc: the library's
+        built-in scratch instead of this encoder's workspace (for callers
+        that cannot allocate; calls on one device must not overlap)."""
+        if len(weights) != len(self.shapes):
+            raise E8qError("number of weights does not match the encoder")
+        for i, w in enumerate(weights):
+            _require_cuda(w, "weight")
+            if tuple(w.shape) != self.shapes[i] or w.dtype != self.in_dtype:
+                raise E8qError(f"weight {i}: expected {self.shapes[i]} {self.in_dtype}, got {tuple(w.shape)} {w.dtype}")
+            self._mats[i].w = w.data_ptr()
+        rc = lib().e8q_project_encode_noalloc(self._mats, len(self.shapes), ctypes.byref(self._args),
+                                              _stream_handle(stream))
+        _check(rc, "e8q_project_encode_noalloc")
         return self.result()
 
     def result(self) -> EncodeResult:

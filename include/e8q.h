@@ -70,7 +70,8 @@ typedef enum {
     E8Q_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or enum */
     E8Q_ERR_UNSUPPORTED = 2, /* valid but outside this build's limits */
     E8Q_ERR_CUDA = 3,        /* a CUDA call or launch failed */
-    E8Q_ERR_WORKSPACE = 4    /* workspace missing or too small */
+    E8Q_ERR_WORKSPACE = 4,   /* workspace missing or too small */
+    E8Q_ERR_SCRATCH_LIMIT = 5 /* larger than e8q_project_encode_noalloc's built-in scratch */
 } e8q_status;
 
 typedef enum { E8Q_F32 = 0, E8Q_BF16 = 1 } e8q_dtype;
@@ -217,6 +218,32 @@ size_t e8q_gemv_workspace_bytes(const e8q_encoded* m /* host */, int32_t batch);
  */
 e8q_status e8q_dequant_gemv(const e8q_encoded* m /* host */, const void* x_bf16, int32_t batch, void* y_bf16,
                             void* ws, size_t ws_bytes, e8q_stream stream);
+
+/*
+ * Project + encode without allocating anything: the same computation and
+ * outputs as e8q_project_encode, for callers that cannot allocate device
+ * memory at all -- code running where cudaMalloc is unavailable or
+ * forbidden (inside a fixed memory pool, a plug-in of a host framework that
+ * owns all allocations, a real-time path that must not allocate).  The paper
+ * has no counterpart; this is a convenience of this library.
+ *
+ * The ordering scratch lives in a 2 MiB array compiled into the library
+ * (a file-scope __device__ array: every GPU that loads the library holds
+ * it until the process exits), so there is no ws argument.  A call needs
+ * 16 + 8 * tiles bytes of it, tiles = sum over matrices of
+ * ceil(rows / max(1, min(64, 4096 / cols))); a call that needs more returns
+ * E8Q_ERR_SCRATCH_LIMIT (about 1 G weights of any shape fit).  The kernel
+ * is the general one (any supported shape and dtype); it clears the part of
+ * the scratch it uses on `stream` before running.
+ *
+ * The first call on each device looks up the device address of the scratch
+ * array (and uploads the constant tables); make it before any stream
+ * capture.  All calls share the one array: calls that overlap on the GPU
+ * (other streams, other host threads) race and must be serialised by the
+ * caller.  Other arguments, outputs and errors as for e8q_project_encode.
+ */
+e8q_status e8q_project_encode_noalloc(const e8q_matrix* mats, int32_t n_mats, const e8q_encode_args* args,
+                                      e8q_stream stream);
 
 #ifdef __cplusplus
 }
