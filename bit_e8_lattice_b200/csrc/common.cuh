@@ -19,6 +19,7 @@ __device__ __align__(16) uint16_t g_t1[2 * 2401 * 7];
 __device__ __align__(16) uint16_t g_t2[2 * 2401];
 __device__ __align__(16) uint2 g_core8[65536];  // 8 int8 doubled coordinates per core index
 __device__ __align__(16) uint2 g_root8[240];
+__device__ __align__(16) uint8_t g_rootkey[512];  // root index by construction key
 
 // Rows per tile: enough rows that a tile holds about 4K elements.
 __host__ __device__ inline int rows_per_tile(int cols) {

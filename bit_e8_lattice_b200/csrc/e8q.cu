@@ -41,6 +41,7 @@ e8q_status ensure_device(int* dev_out) {
         if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_t2, t->t2.data(), t->t2.size() * sizeof(uint16_t)));
         if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_core8, core.data(), core.size() * sizeof(uint2)));
         if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_root8, roots.data(), roots.size() * sizeof(uint2)));
+        if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_rootkey, t->root_of_key.data(), 512));
         if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_encode<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEncSmemBytes));
         if (st == E8Q_OK)
@@ -248,6 +249,11 @@ e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_
     P.n_mats = n_mats;
     P.n_tiles = static_cast<int32_t>(tiles);
     P.total_rows = static_cast<int32_t>(rows_total);
+    {  // |2x| <= 2 kappa sqrt(cols): clamp coordinates only when that could pass 2^14
+        int64_t maxc = 0;
+        for (int i = 0; i < n_mats; ++i) maxc = mats[i].cols > maxc ? mats[i].cols : maxc;
+        P.clamp = (a->scale_in != 0 || 2.0 * a->kappa * std::sqrt(static_cast<double>(maxc)) > 16384.0) ? 1 : 0;
+    }
     if (fast) {
         int64_t g = tiles < g_sms[dev] ? tiles : g_sms[dev];
         if (g > kFastMaxCtas) g = kFastMaxCtas;

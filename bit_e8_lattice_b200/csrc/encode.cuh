@@ -33,6 +33,7 @@ struct EncodeParams {
     int32_t n_mats;
     int32_t n_tiles;
     int32_t total_rows;
+    int32_t clamp;  // fast kernel: inputs may reach |2x| >= 2^14 (given scales or large kappa)
     MatDesc m[MAXM];
 };
 

@@ -31,7 +31,6 @@ constexpr int kFastThreads = (kFastWarps + 1) * 32;
 constexpr int kFastTileElems = 16384;
 constexpr int kFastTileGroups = kFastTileElems / 8;
 constexpr int kFastMaxCtas = 160;
-constexpr int kQueueCap = 64;
 constexpr int kWaitLimit = 1 << 24;
 
 __host__ __device__ inline int fast_rows_per_tile(int cols) {
@@ -46,9 +45,9 @@ constexpr int kFsT2 = kFsT1 + kEncT1Bytes;
 constexpr int kFsMap = kFsT2 + kEncT2Bytes;                   // u32 [3][2048]
 constexpr int kFsIdx = kFsMap + 3 * kFastTileGroups * 4;      // u16 [2][2048]
 constexpr int kFsGss = kFsIdx + 2 * kFastTileGroups * 2;      // f32 [2048]
-constexpr int kFsQueue = kFsGss + kFastTileGroups * 4;        // u32 [8][64][5]
-constexpr int kFsChunk = kFsQueue + kFastWarps * kQueueCap * 20;  // u32 [3][2][65]
-constexpr int kFastSmemBytes = kFsChunk + 3 * 2 * 65 * 4 + 8;
+constexpr int kFsChunk = kFsGss + kFastTileGroups * 4;        // u32 [3][2][65]
+constexpr int kFsRootKey = kFsChunk + 3 * 2 * 65 * 4 + 8;      // u8 [512]
+constexpr int kFastSmemBytes = kFsRootKey + 512;
 
 struct FastTile {
     int t;        // ticket (>= n_tiles: none)
@@ -60,6 +59,12 @@ struct FastTile {
 };
 
 // ---------------------------------------------------------------- helpers
+// Position of a tile group's entry in the per-tile map: the projection
+// writes groups 32a + 4h + q (lane a, q; row h) together and the emission
+// reads 32 consecutive groups together; xor-ing bits 2..4 with bits 5..7
+// keeps both free of shared-memory bank conflicts.
+__device__ __forceinline__ int map_slot(int g) { return g ^ (((g >> 5) & 7) << 2); }
+
 __device__ __forceinline__ void bfly(float& a, float& b) {
     const float x = a;
     a = x + b;
@@ -176,19 +181,23 @@ __device__ __forceinline__ float window_forward(float (&v)[8][8], const unsigned
     stage_rows<1>(v);
     stage_rows<2>(v);
     stage_rows<4>(v);
-    float ss = 0.f;
+    float2 ss = make_float2(0.f, 0.f);
 #pragma unroll
     for (int h = 0; h < 8; ++h)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) ss = fmaf(v[h][e], v[h][e], ss);
-    return ss;
+        for (int e = 0; e < 8; e += 2) {
+            const float2 t = make_float2(v[h][e], v[h][e + 1]);
+            ss = __ffma2_rn(t, t, ss);
+        }
+    return ss.x + ss.y;
 }
 
 __device__ __forceinline__ void load_window_raw(unsigned (&raw)[8][4], const uint16_t* src_smem_or_global,
                                                 bool from_global, const int8_t* signs, int cols, int col0, int nchunks,
                                                 int lane, unsigned long long& nonfinite) {
+    int c = (col0 + 8 * lane) % cols;  // column of this lane's first element; chunks step 256
 #pragma unroll
-    for (int k = 0; k < 8; ++k) {
+    for (int k = 0; k < 8; ++k, c = (c + 256 >= cols) ? c + 256 - cols : c + 256) {
         if (k < nchunks) {
             const uint16_t* p = src_smem_or_global + 256 * k + 8 * lane;
             uint4 q;
@@ -205,7 +214,6 @@ __device__ __forceinline__ void load_window_raw(unsigned (&raw)[8][4], const uin
                     raw[k][j] = x & keep;
                 }
             }
-            const int c = (col0 + 256 * k + 8 * lane) % cols;
             apply_signs(raw[k], __ldg(reinterpret_cast<const uint2*>(signs + c)));
         } else {
             raw[k][0] = raw[k][1] = raw[k][2] = raw[k][3] = 0u;
@@ -213,10 +221,10 @@ __device__ __forceinline__ void load_window_raw(unsigned (&raw)[8][4], const uin
     }
 }
 
-// Escape search for one queued group (all lanes of the warp run this).
-__device__ __forceinline__ void resolve_queued(const uint32_t* e, const uint16_t* st1, const uint16_t* st2,
-                                               uint32_t* map, uint16_t* sidx, int16_t* ovf_scratch,
-                                               unsigned long long& clamped) {
+// Escape search for one queued group (entry: group | P0, P1 | P2, ... P7 | flag).
+__device__ __forceinline__ void resolve_entry(const uint32_t* e, const uint16_t* st1, const uint16_t* st2,
+                                              const uint8_t* rootkey, uint32_t* map, int16_t* ovf_scratch,
+                                              unsigned long long& clamped) {
     const int g = static_cast<int>(e[0] & 0xFFFFu);
     int P[8];
     P[0] = static_cast<int16_t>(e[0] >> 16);
@@ -227,20 +235,18 @@ __device__ __forceinline__ void resolve_queued(const uint32_t* e, const uint16_t
     P[5] = static_cast<int16_t>(e[3] & 0xFFFFu);
     P[6] = static_cast<int16_t>(e[3] >> 16);
     P[7] = static_cast<int16_t>(e[4] & 0xFFFFu);
-    int R[8], Q[8];
-    best_escape_root(P, R);
+    int Q[8], key, n2 = 0;
 #pragma unroll
-    for (int i = 0; i < 8; ++i) Q[i] = P[i] - R[i];
-    const int rq = core_rank(Q, st1, st2);
+    for (int i = 0; i < 8; ++i) n2 += P[i] * P[i];
+    const int v = escape_search(P, Q, key);
+    const int rq = core_rank_n2(Q, n2 - 2 * v + 8, st1, st2);  // |P - R|^2 = |P|^2 - 2 <P, R> + |R|^2
     if (rq >= 0) {
-        const int rr = core_rank(R, st1, st2) - 1;
-        map[g] = static_cast<uint32_t>(rq) | (static_cast<uint32_t>(rr) << 16) | (1u << 24);
-        sidx[g] = static_cast<uint16_t>(rq);
+        const uint32_t rr = rootkey[key];
+        map[map_slot(g)] = static_cast<uint32_t>(rq) | (rr << 16) | (1u << 24);
     } else {
-        map[g] = 2u << 24;
-        sidx[g] = 0;
+        map[map_slot(g)] = 2u << 24;
         uint4 o;
-        o.x = e[0] >> 16 | (e[1] << 16);
+        o.x = (e[0] >> 16) | (e[1] << 16);
         o.y = (e[1] >> 16) | (e[2] << 16);
         o.z = (e[2] >> 16) | (e[3] << 16);
         o.w = (e[3] >> 16) | (e[4] << 16);
@@ -278,8 +284,8 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
     uint32_t* smap = reinterpret_cast<uint32_t*>(smem + kFsMap);
     uint16_t* sidx = reinterpret_cast<uint16_t*>(smem + kFsIdx);
     float* sgss = reinterpret_cast<float*>(smem + kFsGss);
-    uint32_t* squeue = reinterpret_cast<uint32_t*>(smem + kFsQueue);
     uint32_t* schunk = reinterpret_cast<uint32_t*>(smem + kFsChunk);
+    uint8_t* srootkey = smem + kFsRootKey;
 
     __shared__ __align__(8) uint64_t s_full[2];
     __shared__ FastTile s_info[4];
@@ -298,6 +304,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
         for (int i = tid; i < (2 * 2401 * 7 * 2) / 16; i += kFastThreads) b[i] = a[i];
         for (int i = ((2 * 2401 * 7 * 2) / 16) * 8 + tid; i < 2 * 2401 * 7; i += kFastThreads) st1[i] = g_t1[i];
         for (int i = tid; i < 2 * 2401; i += kFastThreads) st2[i] = g_t2[i];
+        for (int i = tid; i < 512; i += kFastThreads) srootkey[i] = g_rootkey[i];
     }
     if (tid == 0) {
         mbar_init(&s_full[0], 1);
@@ -319,8 +326,6 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
 
     const HFrag hf = make_hfrag(lane);
     unsigned long long nonfinite = 0, clamped = 0;
-    int qhead = 0, qcount = 0;  // per-warp escape queue (warp-uniform)
-    uint32_t* myq = squeue + warp * kQueueCap * 5;
 
     for (int i = 0;; ++i) {
         const FastTile cur = s_info[i & 3];
@@ -423,60 +428,80 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     const int a = lane >> 2, q = lane & 3;
                     const bool lane_ok = a < nchunks;
                     const int row_w = win_rows ? (wbase / C) : 0;
+                    // row of the lane's groups: its 8 groups span 232 elements, so the row
+                    // advances at most once (at hcut) when the width is not a multiple of 2048
+                    const int e0 = 8 * (256 * w + 32 * a + q);
+                    const int r0l = e0 / C, hcut = (C - e0 % C + 31) >> 5;
+                    // escape queue in the window's shared-memory region (free until the
+                    // original-basis dequant): 5 words per entry, at most 159 live entries
+                    uint32_t* qbuf = reinterpret_cast<uint32_t*>(win);
+                    int qn = 0;
 #pragma unroll
                     for (int h = 0; h < 8; ++h) {
-                        const int gw = 32 * a + 4 * h + q;
-                        const int gt = 256 * w + gw;
-                        const int row = win_rows ? row_w : (8 * gt) / C;
+                        const int gt = 256 * w + 32 * a + 4 * h + q;
+                        const int row = win_rows ? row_w : r0l + (h >= hcut ? 1 : 0);
                         const float c = s_rowc[lane_ok ? row : 0];
                         float X[8];
 #pragma unroll
-                        for (int e = 0; e < 8; ++e) X[e] = fminf(fmaxf(fmaf(v[h][e], c, 0.f), -1048576.f), 1048576.f);
-                        int P[8];
-                        e8_nearest_doubled(X, P);
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) v[h][e] = static_cast<float>(P[e]);  // keep P for dequant
-                        const int rk = lane_ok ? core_rank(P, st1, st2) : 0;
-                        const bool pend = lane_ok && rk < 0;
-                        if (lane_ok && !pend) {
-                            map[gt] = static_cast<uint32_t>(rk);
-                            idxs[gt] = static_cast<uint16_t>(rk);
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 t = __fmul2_rn(make_float2(v[h][2 * j], v[h][2 * j + 1]), make_float2(c, c));
+                            X[2 * j] = t.x;
+                            X[2 * j + 1] = t.y;
                         }
+                        if (p.clamp) {
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) X[e] = fminf(fmaxf(X[e], -1048576.f), 1048576.f);
+                        }
+                        float Pf[8];
+                        const bool odd = e8_nearest_lean(X, Pf);
+#pragma unroll
+                        for (int e = 0; e < 8; ++e) v[h][e] = Pf[e];  // keep p for the dequant
+                        const int rk = lane_ok ? core_rank_f(Pf, odd, st1, st2) : 0;
+                        const bool pend = lane_ok && rk < 0;
+                        if (lane_ok && !pend) map[map_slot(gt)] = static_cast<uint32_t>(rk);
                         const unsigned bal = __ballot_sync(0xFFFFFFFFu, pend);
                         if (pend) {
-                            const int slot = (qhead + qcount + __popc(bal & lanemask_lt())) & (kQueueCap - 1);
-                            uint32_t* e = myq + 5 * slot;
-                            int Pc[8];
+                            uint32_t* e = qbuf + 5 * (qn + __popc(bal & lanemask_lt()));
+                            int Pi[8];
                             bool clamp = false;
 #pragma unroll
                             for (int k = 0; k < 8; ++k) {
-                                Pc[k] = max(-32768, min(32767, P[k]));
-                                clamp |= Pc[k] != P[k];
+                                Pi[k] = __float_as_int(Pf[k] + 12582912.f) - 0x4B400000;
+                                if (p.clamp) {
+                                    const int c16 = max(-32768, min(32767, Pi[k]));
+                                    clamp |= c16 != Pi[k];
+                                    Pi[k] = c16;
+                                }
                             }
-                            e[0] = static_cast<uint32_t>(gt) | (static_cast<uint32_t>(Pc[0] & 0xFFFF) << 16);
-                            e[1] = static_cast<uint32_t>(Pc[1] & 0xFFFF) | (static_cast<uint32_t>(Pc[2] & 0xFFFF) << 16);
-                            e[2] = static_cast<uint32_t>(Pc[3] & 0xFFFF) | (static_cast<uint32_t>(Pc[4] & 0xFFFF) << 16);
-                            e[3] = static_cast<uint32_t>(Pc[5] & 0xFFFF) | (static_cast<uint32_t>(Pc[6] & 0xFFFF) << 16);
-                            e[4] = static_cast<uint32_t>(Pc[7] & 0xFFFF) | (clamp ? 0x10000u : 0u);
+                            e[0] = static_cast<uint32_t>(gt) | (static_cast<uint32_t>(Pi[0]) << 16);
+                            e[1] = (static_cast<uint32_t>(Pi[1]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[2]) << 16);
+                            e[2] = (static_cast<uint32_t>(Pi[3]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[4]) << 16);
+                            e[3] = (static_cast<uint32_t>(Pi[5]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[6]) << 16);
+                            e[4] = (static_cast<uint32_t>(Pi[7]) & 0xFFFFu) | (clamp ? 0x10000u : 0u);
                         }
-                        qcount += __popc(bal);
-                        if (qcount >= 32) {
+                        qn += __popc(bal);
+                        if (h == 3 || h == 7) {
                             __syncwarp();
-                            resolve_queued(myq + 5 * ((qhead + lane) & (kQueueCap - 1)), st1, st2, map, idxs, oscr,
-                                           clamped);
-                            qhead = (qhead + 32) & (kQueueCap - 1);
-                            qcount -= 32;
+                            int qh = 0;
+                            const int until = (h == 7) ? qn : (qn & ~31);
+                            for (; qh < until; qh += 32)
+                                if (qh + lane < qn)
+                                    resolve_entry(qbuf + 5 * (qh + lane), st1, st2, srootkey, map, oscr, clamped);
                             __syncwarp();
+                            if (h == 3 && qh > 0) {  // move the partial batch to the front
+                                const int left = qn - qh;
+                                uint32_t t[5];
+                                if (lane < left)
+#pragma unroll
+                                    for (int k = 0; k < 5; ++k) t[k] = qbuf[5 * (qh + lane) + k];
+                                __syncwarp();
+                                if (lane < left)
+#pragma unroll
+                                    for (int k = 0; k < 5; ++k) qbuf[5 * lane + k] = t[k];
+                                __syncwarp();
+                                qn = left;
+                            }
                         }
-                    }
-                    if (qcount > 0) {
-                        __syncwarp();
-                        if (lane < qcount)
-                            resolve_queued(myq + 5 * ((qhead + lane) & (kQueueCap - 1)), st1, st2, map, idxs, oscr,
-                                           clamped);
-                        qhead = (qhead + qcount) & (kQueueCap - 1);
-                        qcount = 0;
-                        __syncwarp();
                     }
 
                     // dequantised weights
@@ -486,7 +511,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         for (int h = 0; h < 8; ++h) {
                             if (!lane_ok) continue;
                             const int gt = 256 * w + 32 * a + 4 * h + q;
-                            const float s = s_rows[win_rows ? row_w : (8 * gt) / C];
+                            const float s = s_rows[win_rows ? row_w : r0l + (h >= hcut ? 1 : 0)];
                             uint4 o;
                             o.x = pack_bf16x2(bf16_of_product(s, 0.5f * v[h][0]), bf16_of_product(s, 0.5f * v[h][1]));
                             o.y = pack_bf16x2(bf16_of_product(s, 0.5f * v[h][2]), bf16_of_product(s, 0.5f * v[h][3]));
@@ -548,18 +573,22 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         if (logb >= 10) stage_rows<2>(v);
                         if (logb >= 11) stage_rows<4>(v);
                         uint16_t* dq = static_cast<uint16_t*>(M.dq) + static_cast<size_t>(cur.r0) * C;
+                        int tc = (wbase + 8 * lane) % C, tr = (wbase + 8 * lane) / C;  // column, row of chunk 0
 #pragma unroll
                         for (int k = 0; k < 8; ++k) {
+                            const int col = tc, rowk = tr;
+                            tc += 256;
+                            if (tc >= C) { tc -= C; ++tr; }
                             if (k >= nchunks) continue;
                             const int te = wbase + 256 * k + 8 * lane;  // tile element of the 8-run
-                            const float m = s_rowm[win_rows ? row_w : te / C];
+                            const float m = s_rowm[win_rows ? row_w : rowk];
                             unsigned o[4];
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
                                 const __nv_bfloat162 t = __floats2bfloat162_rn(v[k][2 * j] * m, v[k][2 * j + 1] * m);
                                 o[j] = *reinterpret_cast<const unsigned*>(&t);
                             }
-                            apply_signs(o, __ldg(reinterpret_cast<const uint2*>(M.signs + te % C)));
+                            apply_signs(o, __ldg(reinterpret_cast<const uint2*>(M.signs + col)));
                             *reinterpret_cast<uint4*>(dq + te) = make_uint4(o[0], o[1], o[2], o[3]);
                         }
                     }
@@ -570,7 +599,9 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                 const int nch = (G + 31) >> 5;
                 for (int c = warp; c < nch; c += kFastWarps) {
                     const int g = 32 * c + lane;
-                    const uint32_t k = g < G ? (map[g] >> 24) : 0u;
+                    const uint32_t m = g < G ? map[map_slot(g)] : 0u;
+                    const uint32_t k = m >> 24;
+                    if (g < G) idxs[g] = static_cast<uint16_t>(k == 2 ? 0u : (m & 0xFFFFu));
                     const unsigned be = __ballot_sync(0xFFFFFFFFu, k == 1), bo = __ballot_sync(0xFFFFFFFFu, k == 2);
                     if (lane == 0) {
                         cnt[c] = __popc(be);
@@ -615,7 +646,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                 const uint32_t gid0 = M.group_base + static_cast<uint32_t>(prev2.r0) * gpr;
                 for (int c = warp; c < nch; c += kFastWarps) {
                     const int g = 32 * c + lane;
-                    const uint32_t m = g < G ? map[g] : 0u;
+                    const uint32_t m = g < G ? map[map_slot(g)] : 0u;
                     const uint32_t k = m >> 24;
                     const unsigned be = __ballot_sync(0xFFFFFFFFu, k == 1), bo = __ballot_sync(0xFFFFFFFFu, k == 2);
                     if (k == 1) {

@@ -203,3 +203,254 @@ __device__ __forceinline__ int8_t coord_of(uint2 packed, int i) {
 }
 
 }  // namespace e8q
+
+namespace e8q {
+
+// Same nearest point as e8_nearest_doubled, with fewer instructions: packed
+// fp32 pairs for the rounding, parities from the xor of raw bits, and the
+// parity fix applied to the first coordinate whose error equals the extreme
+// one (no index tracking).  Returns the lattice point as exact floats P
+// (doubled coordinates) and whether it is of the odd (D8 + 1/2) type.
+__device__ __forceinline__ bool e8_nearest_lean(const float (&X)[8], float (&P)[8]) {
+    const float kM = 25165824.0f;  // 1.5 * 2^24
+    float E[8], e[8];
+    unsigned gx = 0u, ex = 0u;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+        const float2 x = make_float2(X[2 * j], X[2 * j + 1]);
+        const float2 g = __fadd2_rn(x, make_float2(kM, kM));
+        const float2 Ev = __fadd2_rn(g, make_float2(-kM, -kM));
+        const float2 d = __ffma2_rn(Ev, make_float2(-1.f, -1.f), x);
+        gx ^= __float_as_uint(g.x) ^ __float_as_uint(g.y);
+        ex ^= __float_as_uint(d.x) ^ __float_as_uint(d.y);
+        E[2 * j] = Ev.x; E[2 * j + 1] = Ev.y;
+        e[2 * j] = d.x; e[2 * j + 1] = d.y;
+    }
+    const bool oddA = (gx & 1u) != 0;              // sum of E/2 is odd
+    const bool oddB = ((gx ^ (ex >> 31)) & 1u) != 0;  // parity of sum(E/2) differs from that of the minus count
+    float2 q = __fmul2_rn(make_float2(e[0], e[1]), make_float2(e[0], e[1]));
+    q = __ffma2_rn(make_float2(e[2], e[3]), make_float2(e[2], e[3]), q);
+    q = __ffma2_rn(make_float2(e[4], e[5]), make_float2(e[4], e[5]), q);
+    q = __ffma2_rn(make_float2(e[6], e[7]), make_float2(e[6], e[7]), q);
+    const float da = q.x + q.y;
+    const float st = ((fabsf(e[0]) + fabsf(e[1])) + (fabsf(e[2]) + fabsf(e[3]))) +
+                     ((fabsf(e[4]) + fabsf(e[5])) + (fabsf(e[6]) + fabsf(e[7])));
+    const float tmax = fmaxf(fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3]))),
+                             fmaxf(fmaxf(fabsf(e[4]), fabsf(e[5])), fmaxf(fabsf(e[6]), fabsf(e[7]))));
+    const float tmin = fminf(fminf(fminf(fabsf(e[0]), fabsf(e[1])), fminf(fabsf(e[2]), fabsf(e[3]))),
+                             fminf(fminf(fabsf(e[4]), fabsf(e[5])), fminf(fabsf(e[6]), fabsf(e[7]))));
+    const float DA = da + (oddA ? (4.f - 4.f * tmax) : 0.f);
+    const float DB = (8.f - 2.f * st + da) + (oddB ? 4.f * tmin : 0.f);
+    const bool useB = DB < DA;
+    const float ub = useB ? 1.f : 0.f;
+    const float m = useB ? tmin : tmax;
+    const float dir = useB ? -2.f : 2.f;  // towards x: the error's sign (D8), its opposite (D8 + 1/2)
+    bool pending = useB ? oddB : oddA;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const float sg = __uint_as_float((__float_as_uint(e[i]) & 0x80000000u) | 0x3F800000u);
+        float p = fmaf(sg, ub, E[i]);
+        const bool hit = pending && fabsf(e[i]) == m;
+        pending = pending && !hit;
+        p = hit ? fmaf(sg, dir, p) : p;
+        P[i] = p;
+    }
+    return useB;
+}
+
+// Core index of a point given as exact floats (doubled coordinates) and its
+// type, or -1 outside the core; the two table keys are formed with exact
+// small-integer float arithmetic.
+__device__ __forceinline__ int core_rank_f(const float (&P)[8], bool odd, const uint16_t* __restrict__ t1,
+                                           const uint16_t* __restrict__ t2) {
+    float2 n = __fmul2_rn(make_float2(P[0], P[4]), make_float2(P[0], P[4]));
+    n = __ffma2_rn(make_float2(P[1], P[5]), make_float2(P[1], P[5]), n);
+    n = __ffma2_rn(make_float2(P[2], P[6]), make_float2(P[2], P[6]), n);
+    n = __ffma2_rn(make_float2(P[3], P[7]), make_float2(P[3], P[7]), n);
+    const float n2 = n.x + n.y;
+    if (!(n2 <= 48.f)) return -1;
+    float2 k = __fmul2_rn(make_float2(P[0], P[4]), make_float2(343.f, 343.f));
+    k = __ffma2_rn(make_float2(P[1], P[5]), make_float2(49.f, 49.f), k);
+    k = __ffma2_rn(make_float2(P[2], P[6]), make_float2(7.f, 7.f), k);
+    k = __fadd2_rn(make_float2(P[3], P[7]), k);
+    // base-7 digits (P + 6) >> 1, plus 2401 for the odd type
+    const float base = odd ? 3401.f : 1200.f;  // even digit (P + 6) / 2: 0.5 k + 1200; odd (P + 5) / 2: 0.5 k + 1000
+    const float hk = fmaf(k.x, 0.5f, base), lk = fmaf(k.y, 0.5f, base);
+    const float i1 = fmaf(hk, 7.f, n2 * 0.125f);
+    const int a = t1[__float_as_int(i1 + 8388608.f) - 0x4B000000];
+    const int b = t2[__float_as_int(lk + 8388608.f) - 0x4B000000];
+    const int r = a + b;
+    return (a != 0xFFFF && r < 65536) ? r : -1;
+}
+
+// best_escape_root with bit masks instead of index loops (same choice).
+__device__ __forceinline__ void best_escape_root_lean(const int (&P)[8], int (&R)[8]) {
+    int w[8];
+    unsigned pos = 0u, zer = 0u, negm = 0u;
+    int a1 = 0, vH = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        w[i] = abs(P[i]);
+        a1 = max(a1, w[i]);
+        vH += w[i];
+        pos |= (P[i] >= 0 ? 1u : 0u) << i;
+        zer |= (P[i] == 0 ? 1u : 0u) << i;
+    }
+    negm = ~pos & 0xFFu;
+    unsigned m1 = 0u;
+    int a2 = -1, wmin = w[0];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        m1 |= (w[i] == a1 ? 1u : 0u) << i;
+        a2 = max(a2, w[i] == a1 ? -1 : w[i]);
+        wmin = min(wmin, w[i]);
+    }
+    const bool single = __popc(m1) == 1;
+    if (!single) a2 = a1;
+    unsigned pick;  // the two positions of the integer-type root
+    if (single) {
+        unsigned m2 = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m2 |= (w[i] == a2 ? 1u : 0u) << i;
+        const unsigned mp = m2 & pos;
+        const unsigned j = mp ? (mp & (0u - mp)) : (1u << (31 - __clz(m2)));
+        pick = m1 | j;
+    } else {
+        const unsigned jp = m1 & pos, jn = m1 & negm;
+        const int np = __popc(jp);
+        if (np >= 2) {
+            const unsigned f = jp & (0u - jp);
+            const unsigned r = jp & ~f;
+            pick = f | (r & (0u - r));
+        } else if (np == 1) {
+            pick = jp | (1u << (31 - __clz(jn)));
+        } else {
+            const unsigned l = 1u << (31 - __clz(jn));
+            const unsigned r = jn & ~l;
+            pick = l | (1u << (31 - __clz(r)));
+        }
+    }
+    const int vI = 2 * (a1 + a2);
+    // half-type root: the signs of P, one flip if the minus count is odd
+    unsigned hneg = negm;
+    if (__popc(negm) & 1) {
+        if (zer) {
+            hneg |= 1u << (31 - __clz(zer));
+        } else {
+            unsigned T = 0u;
+#pragma unroll
+            for (int i = 0; i < 8; ++i) T |= (w[i] == wmin ? 1u : 0u) << i;
+            const unsigned tn = T & negm;
+            const unsigned k = tn ? (tn & (0u - tn)) : (1u << (31 - __clz(T)));
+            hneg ^= k;
+            vH -= 2 * wmin;
+        }
+    }
+    const int ri0 = (pick & 1u) ? ((pos & 1u) ? 2 : -2) : 0;
+    const int rh0 = (hneg & 1u) ? -1 : 1;
+    const bool useI = (vI > vH) || (vI == vH && ri0 > rh0);
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int ri = ((pick >> i) & 1u) ? (((pos >> i) & 1u) ? 2 : -2) : 0;
+        const int rh = ((hneg >> i) & 1u) ? -1 : 1;
+        R[i] = useI ? ri : rh;
+    }
+}
+
+}  // namespace e8q
+
+namespace e8q {
+
+// The escape choice of best_escape_root, returned as the core candidate
+// Q = P - R, the root's construction key (tables.h) and <P, R>.
+__device__ __forceinline__ int escape_search(const int (&P)[8], int (&Q)[8], int& key) {
+    int w[8];
+    unsigned pos = 0u, zer = 0u;
+    int a1 = 0, vH = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        w[i] = abs(P[i]);
+        a1 = max(a1, w[i]);
+        vH += w[i];
+        pos |= (P[i] >= 0 ? 1u : 0u) << i;
+        zer |= (P[i] == 0 ? 1u : 0u) << i;
+    }
+    const unsigned negm = ~pos & 0xFFu;
+    unsigned m1 = 0u, T = 0u;
+    int a2 = -1, wmin = w[0];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        m1 |= (w[i] == a1 ? 1u : 0u) << i;
+        a2 = max(a2, w[i] == a1 ? -1 : w[i]);
+        wmin = min(wmin, w[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) T |= (w[i] == wmin ? 1u : 0u) << i;
+    const bool single = __popc(m1) == 1;
+    unsigned pick;
+    if (single) {
+        unsigned m2 = 0u;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) m2 |= (w[i] == a2 ? 1u : 0u) << i;
+        const unsigned mp = m2 & pos;
+        pick = m1 | (mp ? (mp & (0u - mp)) : (1u << (31 - __clz(m2))));
+    } else {
+        a2 = a1;
+        const unsigned jp = m1 & pos, jn = m1 & negm;
+        const int np = __popc(jp);
+        if (np >= 2) {
+            const unsigned f = jp & (0u - jp), r = jp & ~f;
+            pick = f | (r & (0u - r));
+        } else if (np == 1) {
+            pick = jp | (1u << (31 - __clz(jn)));
+        } else {
+            const unsigned l = 1u << (31 - __clz(jn));
+            pick = l | (1u << (31 - __clz(jn & ~l)));
+        }
+    }
+    const int vI = 2 * (a1 + a2);
+    unsigned hneg = negm;
+    if (__popc(negm) & 1) {
+        if (zer) {
+            hneg |= 1u << (31 - __clz(zer));
+        } else {
+            const unsigned tn = T & negm;
+            hneg ^= tn ? (tn & (0u - tn)) : (1u << (31 - __clz(T)));
+            vH -= 2 * wmin;
+        }
+    }
+    const int ri0 = (pick & 1u) ? ((pos & 1u) ? 2 : -2) : 0;
+    const int rh0 = (hneg & 1u) ? -1 : 1;
+    const bool useI = (vI > vH) || (vI == vH && ri0 > rh0);
+    if (useI) {
+        const int i = __ffs(pick) - 1, j = 31 - __clz(pick);
+        const int ni = ((pos >> i) & 1u) ? 0 : 1, nj = ((pos >> j) & 1u) ? 0 : 1;
+        key = (i << 5) | (j << 2) | (ni << 1) | nj;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) Q[k] = P[k] - (((pick >> k) & 1u) ? (((pos >> k) & 1u) ? 2 : -2) : 0);
+        return vI;
+    }
+    key = 256 | static_cast<int>(hneg);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) Q[k] = P[k] - (((hneg >> k) & 1u) ? -1 : 1);
+    return vH;
+}
+
+// core_rank with |Q|^2 supplied by the caller
+__device__ __forceinline__ int core_rank_n2(const int (&P)[8], int n2, const uint16_t* __restrict__ t1,
+                                            const uint16_t* __restrict__ t2) {
+    if (n2 > 48) return -1;
+    const int type = P[0] & 1;
+    int hk = 0, lk = 0;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+        hk = hk * 7 + ((P[i] + 6) >> 1);
+        lk = lk * 7 + ((P[i + 4] + 6) >> 1);
+    }
+    const int a = t1[(type * 2401 + hk) * 7 + (n2 >> 3)];
+    const int b = t2[type * 2401 + lk];
+    const int r = a + b;
+    return (a != 0xFFFF && r < 65536) ? r : -1;
+}
+
+}  // namespace e8q

@@ -62,6 +62,27 @@ bool build(HostTables& t) {
         if (p.n2 == 8)
             for (int i = 0; i < 8; ++i) t.roots.push_back(p.c[i]);
     if (t.roots.size() != static_cast<size_t>(kNumRoots) * 8) return false;
+    t.root_of_key.assign(512, 0xFF);
+    for (int k = 0; k < kNumRoots; ++k) {
+        const int8_t* r = &t.roots[8 * k];
+        int key = 0, nz = 0, first = -1, second = -1;
+        for (int i = 0; i < 8; ++i)
+            if (r[i] != 0) {
+                ++nz;
+                if (first < 0) first = i;
+                else second = i;
+            }
+        if (nz == 2) {
+            key = (first << 5) | (second << 2) | ((r[first] < 0) << 1) | (r[second] < 0);
+        } else if (nz == 8) {
+            key = 256;
+            for (int i = 0; i < 8; ++i) key |= (r[i] < 0) << i;
+        } else {
+            return false;
+        }
+        if (t.root_of_key[key] != 0xFF) return false;
+        t.root_of_key[key] = static_cast<uint8_t>(k);
+    }
 
     // T2: position of a 4-vector among same-type 4-vectors with equal norm
     // and equal sum mod 4, in lexicographic order (= increasing key).

@@ -36,9 +36,13 @@ struct HostTables {
     std::vector<uint16_t> t2;     // [2][2401]
     std::vector<int8_t> core;     // [65536][8] doubled coordinates
     std::vector<int8_t> roots;    // [240][8]
+    std::vector<uint8_t> root_of_key;  // [512] root index by construction key (see root_key)
     bool ok = false;
 };
 
+// Root construction key: +-2 at positions i < j (signs si, sj, 1 = minus):
+// (i << 5) | (j << 2) | (si << 1) | sj; +-1 everywhere with minus mask m:
+// 256 | m.
 // Builds the tables once (thread-safe); returns nullptr if a consistency
 // check failed.
 const HostTables* host_tables();
