@@ -64,7 +64,7 @@ def measured_peaks() -> dict:
 def profile_traffic(kernel: str):
     """Per-launch DRAM bytes from a committed ncu summary, if it was taken
     on the current kernel sources; otherwise None."""
-    path = os.path.join(ROOT, "profiles", f"{kernel}_mlp_14336.md")
+    path = os.path.join(ROOT, "profiles", f"{kernel}_mlp_14336.md")  # written from an ncu capture
     if not os.path.exists(path):
         return None
     vals = {}
@@ -217,6 +217,7 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--eager", action="store_true", help="time eager launches instead of one captured graph")
     args = ap.parse_args()
     batches = [int(b) for b in args.batches.split(",") if b]
     if args.impl == "reference":
@@ -225,9 +226,9 @@ def main():
     import torch
     import torch.distributed as dist
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local = int(os.environ.get("LOCAL_RANK", "0"))
+    from bit_e8_lattice_b200.dist import max_over_ranks, rank_info
+
+    rank, world, local = rank_info()
     if world > 1:
         from datetime import timedelta
 
@@ -294,6 +295,8 @@ def main():
     graph = None
     mode = "cuda_graph"
     try:
+        if args.eager:
+            raise RuntimeError("eager timing requested")
         ev, t_start, t_end = make_events(True)
         graph = torch.cuda.CUDAGraph()
         cap = torch.cuda.Stream()
@@ -304,7 +307,8 @@ def main():
         graph.replay()  # upload + warm
         torch.cuda.synchronize()
     except Exception as exc:  # capture refused: time eager launches instead
-        print(f"# graph capture unavailable ({exc}); timing eager launches", file=sys.stderr)
+        if not args.eager:
+            print(f"# graph capture unavailable ({exc}); timing eager launches", file=sys.stderr)
         graph, mode = None, "eager"
         torch.cuda.synchronize()
         ev, t_start, t_end = make_events(False)
@@ -319,11 +323,7 @@ def main():
         torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
-    ms = t_start.elapsed_time(t_end)
-    if world > 1:
-        tt = torch.tensor([ms], device=dev, dtype=torch.float64)
-        dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-        ms = float(tt.item())
+    ms = max_over_ranks(t_start.elapsed_time(t_end), dev)
     value = world * G * K / (ms * 1e-3) / 1e9
 
     enc_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
@@ -386,11 +386,7 @@ def main():
             e2e_step()
         z.record(stream)
         torch.cuda.synchronize()
-        ems = a.elapsed_time(z)
-        if world > 1:
-            tt = torch.tensor([ems], device=dev, dtype=torch.float64)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ems = float(tt.item())
+        ems = max_over_ranks(a.elapsed_time(z), dev)
         e2e = {"value": world * G * args.e2e_steps / (ems * 1e-3) / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
@@ -404,7 +400,7 @@ def main():
     if world > 1:
         dist.barrier()
     if rank == 0:
-        traffic = profile_traffic("k_encode")
+        traffic = profile_traffic("k_encode_fast")
         line = {
             "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": K, "warmup": args.warmup,
             "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -414,7 +410,7 @@ def main():
                        "escape_fraction": n_esc / G, "overflow_fraction": n_ovf / G,
                        "payload_bits_pages_formula": 2 + 20 * (n_esc + n_ovf) / G,
                        "parallelism": f"replicas x{world} (rows are independent; no collective)"},
-            "roofline": {"bound": "hbm", "kernel": "k_encode", "achieved": enc_gbs, "peak": peaks["hbm_gbs"],
+            "roofline": {"bound": "hbm", "kernel": "k_encode_fast", "achieved": enc_gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": enc_gbs / peaks["hbm_gbs"], "traffic": traffic,
                          "peak_source": peaks["source"], "algorithmic_bytes_per_launch": enc_bytes},
             "kernels": kernels,
