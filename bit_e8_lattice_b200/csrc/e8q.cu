@@ -55,8 +55,41 @@ e8q_status ensure_device(int* dev_out) {
                                               kFastSmemBytes));
         if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileMaxElems * 4));
+        if (st == E8Q_OK) {
+            // GEMV codeword words: nibble i = P_i + 8
+            std::vector<uint32_t> words(65536);
+            for (int k = 0; k < 65536; ++k) {
+                uint32_t wd = 0;
+                for (int i = 0; i < 8; ++i) wd |= static_cast<uint32_t>((t->core[8 * k + i] + 8) & 0xF) << (4 * i);
+                words[k] = wd;
+            }
+            st = cuda_ok(cudaMemcpyToSymbol(g_gv_tab, words.data(), words.size() * sizeof(uint32_t)));
+        }
         if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_rht_x, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxCols * 4));
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
+        // prep and finalize leave the SM configured for the main kernel's shared
+        // memory, so that its CTAs can start while they are still running
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_prep, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                              cudaSharedmemCarveoutMaxShared));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_fin<1>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                              cudaSharedmemCarveoutMaxShared));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_fin<2>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                              cudaSharedmemCarveoutMaxShared));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_fin<4>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                              cudaSharedmemCarveoutMaxShared));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_fin<8>, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                              cudaSharedmemCarveoutMaxShared));
         if (st == E8Q_OK) st = cuda_ok(cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev));
         if (st != E8Q_OK) return st;
         g_ready[dev] = true;
@@ -66,6 +99,24 @@ e8q_status ensure_device(int* dev_out) {
 }
 
 bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+// Launch with programmatic stream serialisation: the kernel may start while
+// the previous kernel on the stream is finishing; it waits for that
+// kernel's results with griddepcontrol.wait.
+template <typename P>
+e8q_status launch_pdl(void (*kernel)(P), int grid, int threads, size_t smem, cudaStream_t s, const P& params) {
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(static_cast<unsigned>(grid));
+    cfg.blockDim = dim3(static_cast<unsigned>(threads));
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    return cuda_ok(cudaLaunchKernelEx(&cfg, kernel, params));
+}
 
 // log2 of the effective RHT block, or -1 if invalid
 int resolve_logb(int64_t cols, int32_t block) {
@@ -316,9 +367,9 @@ e8q_status e8q_decode(const e8q_encoded* m, int32_t basis, void* out_bf16, e8q_s
 }
 
 size_t e8q_gemv_workspace_bytes(const e8q_encoded* m, int32_t batch) {
-    if (!m || m->cols <= 0 || batch <= 0) return 256;
-    const size_t bytes = static_cast<size_t>(batch) * static_cast<size_t>(m->cols) * 4;
-    return (bytes + 255) / 256 * 256;
+    if (!m || m->rows < 0 || m->cols <= 0 || m->cols > kMaxCols || batch <= 0 || batch > 256) return 256;
+    const GvGeom g = gv_geometry(m->rows, m->cols, batch, 0, kGvMaxCtas);
+    return gv_workspace(g).total;
 }
 
 e8q_status e8q_dequant_gemv(const e8q_encoded* m, const void* x_bf16, int32_t batch, void* y_bf16, void* ws,
@@ -328,42 +379,75 @@ e8q_status e8q_dequant_gemv(const e8q_encoded* m, const void* x_bf16, int32_t ba
     if (st != E8Q_OK) return st;
     if (batch < 1 || batch > 256) return E8Q_ERR_INVALID_ARG;
     if (!x_bf16 || !y_bf16 || !m->signs || !aligned(x_bf16, 16) || !aligned(y_bf16, 2)) return E8Q_ERR_INVALID_ARG;
+    if (m->esc_row_ptr && !aligned(m->esc, 8)) return E8Q_ERR_INVALID_ARG;
     const size_t need = e8q_gemv_workspace_bytes(m, batch);
-    if (!ws || ws_bytes < need || !aligned(ws, 16)) return E8Q_ERR_WORKSPACE;
+    if (!ws || ws_bytes < need || !aligned(ws, 256)) return E8Q_ERR_WORKSPACE;
     if (m->rows == 0) return E8Q_OK;
     int dev;
     st = ensure_device(&dev);
     if (st != E8Q_OK) return st;
     cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-    RhtParams rp;
-    rp.x = static_cast<const uint16_t*>(x_bf16);
-    rp.signs = m->signs;
-    rp.xr = static_cast<float*>(ws);
-    rp.cols = static_cast<int32_t>(m->cols);
-    rp.logb = logb;
-    k_rht_x<<<batch, kRhtThreads, static_cast<size_t>(m->cols) * 4, s>>>(rp);
+    const int ctas = g_sms[dev] < kGvMaxCtas ? g_sms[dev] : kGvMaxCtas;
+    const GvGeom g = gv_geometry(m->rows, m->cols, batch, logb, ctas);
+    const GvWs L = gv_workspace(g);
+    unsigned char* w = static_cast<unsigned char*>(ws);
+    const bool has_esc = m->esc_row_ptr != nullptr;
+
+    GvPrepParams pp;
+    pp.x = static_cast<const uint16_t*>(x_bf16);
+    pp.signs = m->signs;
+    pp.x32 = reinterpret_cast<float*>(w + L.x32);
+    pp.x16 = reinterpret_cast<uint4*>(w + L.x16);
+    pp.xe = reinterpret_cast<float*>(w + L.xe);
+    pp.esc = m->esc;
+    pp.esc_rp = m->esc_row_ptr;
+    pp.map = reinterpret_cast<uint8_t*>(w + L.map);
+    pp.esc_n = has_esc ? m->esc_count : 0;
+    pp.group_base = m->group_base;
+    pp.g = g;
+    pp.n_xcta = g.nseg * batch;
+    const int n_ecta = has_esc ? (g.rows + 7) / 8 : 0;
+    k_gv_prep<<<pp.n_xcta + n_ecta, 256, 0, s>>>(pp);
     st = cuda_ok(cudaGetLastError());
     if (st != E8Q_OK) return st;
-    GemvParams gp;
-    gp.idx = m->idx;
-    gp.scale = m->scale;
-    gp.esc = m->esc;
-    gp.esc_rp = m->esc_row_ptr;
-    gp.ovf = m->ovf;
-    gp.ovf_rp = m->ovf_row_ptr;
-    gp.esc_n = m->esc_row_ptr ? m->esc_count : 0;
-    gp.ovf_n = m->ovf_row_ptr ? m->ovf_count : 0;
-    gp.xr = static_cast<const float*>(ws);
-    gp.y = static_cast<uint16_t*>(y_bf16);
-    gp.group_base = m->group_base;
-    gp.rows = static_cast<int32_t>(m->rows);
-    gp.cols = static_cast<int32_t>(m->cols);
-    gp.batch = batch;
-    const int warps_per_cta = kGemvThreads / 32;
-    int grid = static_cast<int>((m->rows + warps_per_cta - 1) / warps_per_cta);
-    if (grid > 8 * g_sms[dev]) grid = 8 * g_sms[dev];
-    k_gemv<<<grid, kGemvThreads, 0, s>>>(gp);
-    return cuda_ok(cudaGetLastError());
+
+    GvMainParams mp;
+    mp.idx = m->idx;
+    mp.x16 = pp.x16;
+    mp.map = has_esc ? pp.map : nullptr;
+    mp.part = reinterpret_cast<float*>(w + L.part);
+    mp.g = g;
+    mp.vec_idx = (g.gpr % 8 == 0 && aligned(m->idx, 16)) ? 1 : 0;
+    const int grid = g.nctas;
+    for (int v0 = 0; v0 < g.nbt; v0 += kGvPassTiles) {
+        const int nt = g.nbt - v0 < kGvPassTiles ? g.nbt - v0 : kGvPassTiles;
+        mp.v0 = v0;
+        if (nt == 1) st = launch_pdl(k_gv_main<1>, grid, kGvThreads, kGvSmemBytes, s, mp);
+        else if (nt == 2) st = launch_pdl(k_gv_main<2>, grid, kGvThreads, kGvSmemBytes, s, mp);
+        else if (nt <= 4) st = launch_pdl(k_gv_main<4>, grid, kGvThreads, kGvSmemBytes, s, mp);
+        else st = launch_pdl(k_gv_main<8>, grid, kGvThreads, kGvSmemBytes, s, mp);
+        if (st != E8Q_OK) return st;
+    }
+
+    GvFinParams fp;
+    fp.part = mp.part;
+    fp.xe = pp.xe;
+    fp.x32 = pp.x32;
+    fp.scale = m->scale;
+    fp.ovf = m->ovf;
+    fp.ovf_rp = m->ovf_row_ptr;
+    fp.y = static_cast<uint16_t*>(y_bf16);
+    fp.ovf_n = m->ovf_row_ptr ? m->ovf_count : 0;
+    fp.group_base = m->group_base;
+    fp.g = g;
+    fp.bl_log = 0;
+    while ((1 << fp.bl_log) < batch && fp.bl_log < 5) ++fp.bl_log;
+    const int kb = (batch + 31) / 32;  // batch rows per lane
+    const int fgrid = (g.rows + 7) / 8;
+    if (kb == 1) return launch_pdl(k_gv_fin<1>, fgrid, 256, 0, s, fp);
+    if (kb == 2) return launch_pdl(k_gv_fin<2>, fgrid, 256, 0, s, fp);
+    if (kb <= 4) return launch_pdl(k_gv_fin<4>, fgrid, 256, 0, s, fp);
+    return launch_pdl(k_gv_fin<8>, fgrid, 256, 0, s, fp);
 }
 
 }  // extern "C"

@@ -1,129 +1,632 @@
 // K4 + K5: dequant-GEMV from the 2-bit form ("E8-QAT", abstract: decoding
 // throughput of the 2-bit representation).
 //
-//   y[b][r] = s_r / 2 * ( sum_g <P_core[idx_rg], xr_bg>
-//                       + sum_{escapes of row r} <R_root, xr_bg>
-//                       + sum_{overflows of row r} <P_record, xr_bg> ),
-//   xr_b = H_B (d (.) x_b) / sqrt(B)   (blockwise, fp32),
-// which equals sum_c w~[r][c] x[b][c] with w~ the original-basis weights.
+//   y[b][r] = s_r / 2 * sum_g < P_rg , xr_b[8g .. 8g+7] >,
+//   xr_b   = H_B (d (.) x_b) / sqrt(B)          (blockwise),
+//   P_rg   = core[idx_rg] (+ root, for an escaped group; = record, for an
+//            overflow group),
+// which equals sum_c w~[r][c] x[b][c] with w~ the original-basis weights
+// (the doubled coordinates P = 2p account for the 1/2).
+//
+// Three launches:
+//  k_gv_prep  (a) per activation row and 2048-column segment: xr in fp32
+//             (natural order) and in fp16 scaled by a power of two chosen
+//             from the row's largest |x| so that no value can overflow fp16,
+//             stored in the order in which the MMA B fragments are read;
+//             (b) per weight row: a dense byte map group -> root + 1 (0: no
+//             escape) from the escape records, in any record order.
+//  k_gv_main  tensor cores: mma.sync m16n8k16, A = codewords (16 weight rows
+//             x 16 coordinates), B = activations (16 coordinates x 8 batch
+//             rows), fp32 accumulate.  The work -- 256-row blocks times
+//             256-column chunks times 8 k-steps -- is split into equal
+//             contiguous k-step ranges, one per CTA (one resident CTA per
+//             SM); the 8 warps of a CTA take 32 rows each of the same range,
+//             so they read the same activation fragments (L1 hits).  The first
+//             49,152 codeword words live in shared memory (a shared-memory
+//             gather costs a few wavefronts per warp, a global one up to one
+//             per lane); the rest are read through L1.  Indices and root-map
+//             bytes of the next chunk are loaded while the current one is
+//             multiplied.  Escape roots are added to the codeword bytes before
+//             the fp16 conversion.  Partial sums go to a per-(row block, CTA)
+//             slot of the workspace.
+//  k_gv_fin   per weight row: the partial slots in a fixed order, the
+//             overflow records (CUDA cores, fp32 activations; lanes split
+//             over records and batch rows), the scale, bf16 output.
 #pragma once
+#include <cuda_fp16.h>
+
 #include "common.cuh"
-#include "lattice.cuh"
+#include "ptx.cuh"
 
 namespace e8q {
 
-constexpr int kRhtThreads = 256;
-constexpr int kGemvThreads = 256;
+// Core codeword k as 8 nibbles: nibble i (bits 4i..4i+3) = P_i + 8.
+__device__ __align__(16) uint32_t g_gv_tab[65536];
 
-struct RhtParams {
-    const uint16_t* x;  // bf16 [batch][cols]
-    const int8_t* signs;
-    float* xr;          // fp32 [batch][cols]
-    int32_t cols;
+constexpr int kGvThreads = 256;
+constexpr int kGvWarps = kGvThreads / 32;
+constexpr int kGvWarpRows = 32;    // rows per warp: two 16-row MMA tiles
+constexpr int kGvBlockRows = kGvWarps * kGvWarpRows;  // rows per row block (one CTA's rows)
+constexpr int kGvChunkCols = 256;  // columns per chunk: 32 groups, 8 k-steps
+constexpr int kGvTabN = 49152;     // codeword words held in shared memory
+constexpr int kGvMaxCtas = 160;    // upper bound on main-kernel CTAs (workspace sizing)
+constexpr int kGvSegCols = 2048;   // activation columns per prep CTA
+constexpr int kGvPassTiles = 8;    // batch tiles of 8 per main-kernel pass
+constexpr size_t kGvTabBytes = size_t{kGvTabN} * 4;
+constexpr size_t kGvRootBytes = 256 * 8;
+constexpr size_t kGvSmemBytes = kGvTabBytes + kGvRootBytes;
+
+struct GvGeom {
+    int32_t rows, cols, gpr, batch;
+    int32_t nbt;       // batch tiles of 8
+    int32_t nchunks;   // 256-column chunks (last one may be partial)
+    int32_t nrb;       // 32-row blocks
+    int32_t nctas;     // main-kernel CTAs with work
+    int32_t maxslots;  // partial slots per row block
+    int32_t mstride;   // root-map bytes per row (32 * nchunks)
+    int32_t seg_cols;  // prep segment
+    int32_t nseg;
     int32_t logb;
+    int64_t ksteps;    // nrb * nchunks * 8
 };
 
-__global__ void __launch_bounds__(kRhtThreads) k_rht_x(const __grid_constant__ RhtParams p) {
-    extern __shared__ __align__(16) unsigned char smem[];
-    float* buf = reinterpret_cast<float*>(smem);
-    const int b = blockIdx.x, C = p.cols;
-    const uint16_t* xb = p.x + static_cast<size_t>(b) * C;
-    for (int c = threadIdx.x; c < C; c += kRhtThreads) {
-        const float v = __uint_as_float(static_cast<unsigned>(xb[c]) << 16);
-        buf[c] = p.signs[c] < 0 ? -v : v;
-    }
-    __syncthreads();
-    if (p.logb > 0) fwht_smem(buf, C, p.logb);
-    const float inv = 1.0f / sqrtf(static_cast<float>(1 << p.logb));
-    for (int c = threadIdx.x; c < C; c += kRhtThreads) p.xr[static_cast<size_t>(b) * C + c] = buf[c] * inv;
+inline GvGeom gv_geometry(int64_t rows, int64_t cols, int batch, int logb, int ctas) {
+    GvGeom g;
+    g.rows = static_cast<int32_t>(rows);
+    g.cols = static_cast<int32_t>(cols);
+    g.gpr = g.cols / 8;
+    g.batch = batch;
+    g.nbt = (batch + 7) / 8;
+    g.nchunks = (g.cols + kGvChunkCols - 1) / kGvChunkCols;
+    g.nrb = (g.rows + kGvBlockRows - 1) / kGvBlockRows;
+    g.ksteps = static_cast<int64_t>(g.nrb) * g.nchunks * 8;
+    g.nctas = static_cast<int32_t>(g.ksteps < ctas ? g.ksteps : ctas);
+    if (g.nctas < 1) g.nctas = 1;
+    // a row block's k-steps meet at most ceil(KS / per) + 1 CTA ranges
+    const int64_t per = g.ksteps / g.nctas > 0 ? g.ksteps / g.nctas : 1;
+    const int64_t ks = static_cast<int64_t>(g.nchunks) * 8;
+    int64_t slots = (ks + per - 1) / per + 1;
+    if (slots > g.nctas) slots = g.nctas;
+    g.maxslots = static_cast<int32_t>(slots);
+    g.mstride = 32 * g.nchunks;
+    g.seg_cols = g.cols < kGvSegCols ? g.cols : kGvSegCols;
+    g.nseg = g.seg_cols > 0 ? (g.cols + g.seg_cols - 1) / g.seg_cols : 0;
+    g.logb = logb;
+    return g;
 }
 
-struct GemvParams {
-    const uint16_t* idx;
-    const float* scale;
+struct GvWs {
+    size_t x32, x16, xe, map, part, total;
+};
+inline size_t gv_round(size_t x) { return (x + 255) / 256 * 256; }
+inline GvWs gv_workspace(const GvGeom& g) {
+    GvWs w;
+    w.x32 = 0;
+    w.x16 = w.x32 + gv_round(static_cast<size_t>(g.batch) * g.cols * 4);
+    w.xe = w.x16 + gv_round(static_cast<size_t>(g.nchunks) * g.nbt * 8 * 32 * 16);
+    w.map = w.xe + gv_round(static_cast<size_t>(g.nbt) * 8 * 4);
+    w.part = w.map + gv_round(static_cast<size_t>(g.rows) * g.mstride);
+    w.total = w.part + gv_round(static_cast<size_t>(g.nrb) * g.maxslots * g.batch * kGvBlockRows * 4);
+    return w;
+}
+
+// The CTA whose k-step range holds k-step u (ranges: [floor(wT/W), floor((w+1)T/W))).
+__host__ __device__ __forceinline__ int64_t gv_cta_of(int64_t u, int64_t T, int64_t W) {
+    return ((u + 1) * W - 1) / T;
+}
+
+// ---------------------------------------------------------------------------
+// prep
+// ---------------------------------------------------------------------------
+struct GvPrepParams {
+    const uint16_t* x;  // bf16 [batch][cols]
+    const int8_t* signs;
+    float* x32;         // [cols][batch] (column-major: one group's batch rows contiguous)
+    uint4* x16;         // [nchunks][nbt][8 k-steps][32 lanes] x 8 halves
+    float* xe;          // [batch]: 2^e, x16 = xr * 2^-e
     const e8q_escape* esc;
     const int64_t* esc_rp;
-    const e8q_overflow* ovf;
-    const int64_t* ovf_rp;
-    const float* xr;  // fp32 [batch][cols]
-    uint16_t* y;      // bf16 [batch][rows]
+    uint8_t* map;       // [rows][mstride]: root + 1 of an escaped group, else 0
     long long esc_n;
-    long long ovf_n;
     long long group_base;
-    int32_t rows;
-    int32_t cols;
-    int32_t batch;
+    GvGeom g;
+    int32_t n_xcta;     // CTAs of part (a)
 };
 
-__global__ void __launch_bounds__(kGemvThreads) k_gemv(const __grid_constant__ GemvParams p) {
+__device__ __forceinline__ long long gv_clamp(long long v, long long lo, long long hi) {
+    return v < lo ? lo : (v > hi ? hi : v);
+}
+
+__device__ __forceinline__ unsigned pack_half2(float a, float b) {
+    const __half2 h = __floats2half2_rn(a, b);
+    return *reinterpret_cast<const unsigned*>(&h);
+}
+
+__global__ void __launch_bounds__(256) k_gv_prep(const __grid_constant__ GvPrepParams p) {
+    __shared__ __align__(16) float buf[kGvSegCols];
+    __shared__ unsigned s_red[8];
+    pdl_launch_dependents();
+    const GvGeom& G = p.g;
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    if (static_cast<int>(blockIdx.x) < p.n_xcta) {
+        const int b = blockIdx.x / G.nseg, seg = blockIdx.x % G.nseg;
+        const int C = G.cols;
+        const uint16_t* xb = p.x + static_cast<size_t>(b) * C;
+        // largest |x| of the row, as bf16 magnitude bits (integer order = value order)
+        unsigned m = 0;
+        for (int i = threadIdx.x; i < C / 8; i += 256) {
+            const uint4 v = __ldg(reinterpret_cast<const uint4*>(xb) + i);
+            const unsigned w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int k = 0; k < 4; ++k) m = max(m, max(w4[k] & 0x7FFFu, (w4[k] >> 16) & 0x7FFFu));
+        }
+        m = __reduce_max_sync(0xFFFFFFFFu, m);
+        if (lane == 0) s_red[warp] = m;
+        __syncthreads();
+        m = s_red[0];
+#pragma unroll
+        for (int k = 1; k < 8; ++k) m = max(m, s_red[k]);
+        // |xr_i| <= sqrt(B) max|x|: pick e with sqrt(B) max|x| 2^-e < 2^15
+        int e = 0;
+        if (m != 0 && m < 0x7F80u) {
+            const float bound = __uint_as_float(m << 16) * sqrtf(static_cast<float>(1 << G.logb)) * 1.0001f;
+            int k;
+            frexpf(bound, &k);
+            e = k - 15;
+            e = e < -126 ? -126 : (e > 126 ? 126 : e);
+        }
+        const float down = __uint_as_float(static_cast<unsigned>(127 - e) << 23);  // 2^-e
+        const int c0 = seg * G.seg_cols;
+        const int n = min(G.seg_cols, C - c0);
+        for (int i = threadIdx.x; i < n; i += 256) {
+            const float v = __uint_as_float(static_cast<unsigned>(xb[c0 + i]) << 16);
+            buf[i] = p.signs[c0 + i] < 0 ? -v : v;
+        }
+        __syncthreads();
+        if (G.logb > 0) fwht_smem(buf, n, G.logb);
+        const float inv = 1.0f / sqrtf(static_cast<float>(1 << G.logb));
+        for (int i = threadIdx.x; i < n; i += 256) p.x32[static_cast<size_t>(c0 + i) * G.batch + b] = buf[i] * inv;
+        for (int t = threadIdx.x; t < n / 8; t += 256) {
+            const int col = c0 + 8 * t;
+            const int c = col >> 8, gc = (col & 255) >> 3, q = gc >> 3, j = gc & 7;
+            const int L = 4 * (b & 7) + q;
+            float v[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) v[i] = buf[8 * t + i] * inv * down;
+            uint4 o;
+            o.x = pack_half2(v[0], v[1]);
+            o.y = pack_half2(v[2], v[3]);
+            o.z = pack_half2(v[4], v[5]);
+            o.w = pack_half2(v[6], v[7]);
+            p.x16[((static_cast<size_t>(c) * G.nbt + (b >> 3)) * 8 + j) * 32 + L] = o;
+        }
+        if (seg == 0 && threadIdx.x == 0) p.xe[b] = __uint_as_float(static_cast<unsigned>(127 + e) << 23);
+        return;
+    }
+    // (b) root map of one weight row per warp: clear, then scatter the row's records
+    if (!p.esc_rp) return;
+    const int r = (blockIdx.x - p.n_xcta) * 8 + warp;
+    if (r >= G.rows) return;
+    uint8_t* mrow = p.map + static_cast<size_t>(r) * G.mstride;
+    for (int i = lane; i < G.mstride / 16; i += 32) reinterpret_cast<uint4*>(mrow)[i] = make_uint4(0, 0, 0, 0);
+    __syncwarp();
+    const long long e0 = gv_clamp(p.esc_rp[r], 0, p.esc_n);
+    const long long e1 = gv_clamp(p.esc_rp[r + 1], e0, p.esc_n);
+    const long long g0 = p.group_base + static_cast<long long>(r) * G.gpr;
+    // records in rounds of 8 per lane: all loads of a round before its stores
+    for (long long k0 = e0; k0 < e1; k0 += 8 * 32) {
+        uint2 rec[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const long long k = k0 + lane + 32 * i;
+            rec[i] = k < e1 ? __ldcs(reinterpret_cast<const uint2*>(p.esc + k)) : make_uint2(0xFFFFFFFFu, 0u);
+        }
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const long long gl = static_cast<long long>(rec[i].x) - g0;  // group
+            const unsigned root = (rec[i].y >> 16) & 0xFFu;
+            if (gl >= 0 && gl < G.gpr && root < 240) mrow[gl] = static_cast<uint8_t>(root + 1);
+        }
+    }
+}
+
+// ---------------------------------------------------------------------------
+// main
+// ---------------------------------------------------------------------------
+struct GvMainParams {
+    const uint16_t* idx;
+    const uint4* x16;
+    const uint8_t* map;  // null: no escapes
+    float* part;         // [nrb][maxslots][256 rows][batch]
+    GvGeom g;
+    int32_t v0;          // first batch tile of this pass
+    int32_t vec_idx;     // index rows 16-byte aligned (gpr % 8 == 0, aligned base)
+};
+
+__device__ __forceinline__ void mma_f16(float (&d)[4], unsigned a0, unsigned a1, unsigned a2, unsigned a3, unsigned b0,
+                                        unsigned b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+        "{%0,%1,%2,%3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ unsigned hsub2_bits(unsigned a, unsigned b) {
+    unsigned r;
+    asm("sub.rn.f16x2 %0, %1, %2;" : "=r"(r) : "r"(a), "r"(b));
+    return r;
+}
+
+// 8 indices of one row: groups gs .. gs+7 (0 past the row end).
+__device__ __forceinline__ uint4 gv_idx8(const uint16_t* rowp, int gs, int gpr, bool vec) {
+    if (vec && gs + 8 <= gpr) return __ldcs(reinterpret_cast<const uint4*>(rowp + gs));
+    unsigned h[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) h[i] = (gs + i < gpr) ? static_cast<unsigned>(rowp[gs + i]) : 0u;
+    return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
+}
+
+// row (within the warp's 32) of codeword slot r (0..3): tile r>>1, +8 for odd r
+__device__ __forceinline__ int gv_row_in_warp(int r, int g) { return 16 * (r >> 1) + 8 * (r & 1) + g; }
+
+struct GvVisit {
+    uint4 idx[4];  // 8 indices per codeword row
+    uint2 map[4];  // 8 root-map bytes per codeword row
+};
+
+__device__ __forceinline__ void gv_load_idx(const GvMainParams& p, int rb, int c, int warp, int g, int q, GvVisit& d) {
+    const GvGeom& G = p.g;
+    const int gs = 32 * c + 8 * q;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int row = rb * kGvBlockRows + warp * kGvWarpRows + gv_row_in_warp(r, g);
+        d.idx[r] = row < G.rows ? gv_idx8(p.idx + static_cast<size_t>(row) * G.gpr, gs, G.gpr, p.vec_idx != 0)
+                                : make_uint4(0, 0, 0, 0);
+    }
+}
+
+__device__ __forceinline__ void gv_load_map(const GvMainParams& p, int rb, int c, int warp, int g, int q, GvVisit& d) {
+    const GvGeom& G = p.g;
+    const int gs = 32 * c + 8 * q;
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const int row = rb * kGvBlockRows + warp * kGvWarpRows + gv_row_in_warp(r, g);
+        d.map[r] = (row < G.rows && p.map)
+                       ? __ldcg(reinterpret_cast<const uint2*>(p.map + static_cast<size_t>(row) * G.mstride + gs))
+                       : make_uint2(0, 0);
+    }
+}
+
+__device__ __forceinline__ unsigned gv_comp(const uint4& v, int k) {
+    return k == 0 ? v.x : (k == 1 ? v.y : (k == 2 ? v.z : v.w));
+}
+
+// Codeword word of codeword row r at k-step j (shared table, else L1).
+__device__ __forceinline__ unsigned gv_word(const GvVisit& cv, const uint32_t* s_tab, int r, int j) {
+    const unsigned comp = gv_comp(cv.idx[r], j >> 1);
+    const unsigned id = (j & 1) ? (comp >> 16) : (comp & 0xFFFFu);
+    return id < static_cast<unsigned>(kGvTabN) ? s_tab[id] : __ldg(g_gv_tab + id);
+}
+
+// Codeword pairs (P_2k, P_2k+1) in fp16 of the 4 codeword rows at k-step j.
+template <bool ESC>
+__device__ __forceinline__ void gv_decode(const GvVisit& cv, const unsigned (&wd)[4], const uint2* s_root, int j,
+                                          unsigned (&pr)[4][4]) {
+#pragma unroll
+    for (int r = 0; r < 4; ++r) {
+        const unsigned w = wd[r];
+        unsigned lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu, bias;
+        if (ESC) {
+            const unsigned root = ((j < 4 ? cv.map[r].x : cv.map[r].y) >> (8 * (j & 3))) & 0xFFu;
+            const uint2 rb = s_root[root];
+            lo += rb.x;
+            hi += rb.y;
+            bias = 0x640A640Au;  // 1034 = 1024 + 8 + 2
+        } else {
+            bias = 0x64086408u;  // 1032 = 1024 + 8
+        }
+        pr[r][0] = hsub2_bits(prmt(lo, hi, 0x8480u) | 0x64006400u, bias);
+        pr[r][1] = hsub2_bits(prmt(lo, hi, 0x8581u) | 0x64006400u, bias);
+        pr[r][2] = hsub2_bits(prmt(lo, hi, 0x8682u) | 0x64006400u, bias);
+        pr[r][3] = hsub2_bits(prmt(lo, hi, 0x8783u) | 0x64006400u, bias);
+    }
+}
+
+template <int NBP>
+__device__ __forceinline__ void gv_mma(float (&acc)[2][NBP][4], const unsigned (&pr)[4][4], const uint4 (&xb)[NBP]) {
+#pragma unroll
+    for (int u = 0; u < NBP; ++u)
+#pragma unroll
+        for (int t = 0; t < 2; ++t) {
+            mma_f16(acc[t][u], pr[2 * t][0], pr[2 * t + 1][0], pr[2 * t][1], pr[2 * t + 1][1], xb[u].x, xb[u].y);
+            mma_f16(acc[t][u], pr[2 * t][2], pr[2 * t + 1][2], pr[2 * t][3], pr[2 * t + 1][3], xb[u].z, xb[u].w);
+        }
+}
+
+// Activation fragments of k-step j for the pass's batch tiles (0 where the
+// batch row or the group does not exist).
+template <int NBP>
+__device__ __forceinline__ void gv_load_x(const uint4* xs, const bool (&bok)[NBP], bool jok, int j, int lane,
+                                          uint4 (&xb)[NBP]) {
+#pragma unroll
+    for (int u = 0; u < NBP; ++u)
+        xb[u] = (bok[u] && jok) ? __ldg(xs + static_cast<size_t>(u) * 256 + j * 32 + lane) : make_uint4(0, 0, 0, 0);
+}
+
+template <int NBP, bool ESC>
+__device__ __forceinline__ void gv_visit(float (&acc)[2][NBP][4], const GvVisit& cv, const uint32_t* s_tab,
+                                         const uint2* s_root, const uint4* xs, const bool (&bok)[NBP], int lim, int j0,
+                                         int j1, int lane) {
+    if (NBP <= 2) {
+        // every codeword word and activation fragment of the chunk up front:
+        // one exposed latency per chunk
+        unsigned wd[8][4];
+        uint4 xa[8][NBP];
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+#pragma unroll
+            for (int r = 0; r < 4; ++r) wd[j][r] = (j >= j0 && j < j1) ? gv_word(cv, s_tab, r, j) : 0u;
+#pragma unroll
+        for (int j = 0; j < 8; ++j) gv_load_x<NBP>(xs, bok, j < lim && j >= j0 && j < j1, j, lane, xa[j]);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j >= j0 && j < j1) {
+                unsigned pr[4][4];
+                gv_decode<ESC>(cv, wd[j], s_root, j, pr);
+                gv_mma<NBP>(acc, pr, xa[j]);
+            }
+    } else if (NBP >= 8) {
+        // no room for a second set of fragments: load at the k-step
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j >= j0 && j < j1) {
+                uint4 xb[NBP];
+                unsigned wd[4];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) wd[r] = gv_word(cv, s_tab, r, j);
+                gv_load_x<NBP>(xs, bok, j < lim, j, lane, xb);
+                unsigned pr[4][4];
+                gv_decode<ESC>(cv, wd, s_root, j, pr);
+                gv_mma<NBP>(acc, pr, xb);
+            }
+    } else {
+        uint4 xb[NBP], xn[NBP];
+        unsigned wd[4], wn[4];
+#pragma unroll
+        for (int r = 0; r < 4; ++r) wd[r] = gv_word(cv, s_tab, r, j0);
+        gv_load_x<NBP>(xs, bok, j0 < lim, j0, lane, xb);
+#pragma unroll
+        for (int j = 0; j < 8; ++j)
+            if (j >= j0 && j < j1) {
+                if (j + 1 < j1) {
+                    gv_load_x<NBP>(xs, bok, j + 1 < lim, j + 1, lane, xn);
+#pragma unroll
+                    for (int r = 0; r < 4; ++r) wn[r] = gv_word(cv, s_tab, r, j + 1);
+                }
+                unsigned pr[4][4];
+                gv_decode<ESC>(cv, wd, s_root, j, pr);
+                gv_mma<NBP>(acc, pr, xb);
+#pragma unroll
+                for (int u = 0; u < NBP; ++u) xb[u] = xn[u];
+#pragma unroll
+                for (int r = 0; r < 4; ++r) wd[r] = wn[r];
+            }
+    }
+}
+
+template <int NBP>
+__device__ __forceinline__ void gv_flush(const GvMainParams& p, float (&acc)[2][NBP][4], int rb, int warp, int g,
+                                         int q) {
+    const GvGeom& G = p.g;
+    const long long ks = static_cast<long long>(G.nchunks) * 8;
+    const long long slot = static_cast<long long>(blockIdx.x) - gv_cta_of(static_cast<long long>(rb) * ks, G.ksteps, G.nctas);
+    if (slot >= 0 && slot < G.maxslots) {
+        float* base = p.part + ((static_cast<size_t>(rb) * G.maxslots + slot) * kGvBlockRows + warp * kGvWarpRows) *
+                                   G.batch;
+#pragma unroll
+        for (int t = 0; t < 2; ++t)
+#pragma unroll
+            for (int u = 0; u < NBP; ++u)
+#pragma unroll
+                for (int k = 0; k < 4; ++k) {
+                    const int b = 8 * (p.v0 + u) + 2 * q + (k & 1);
+                    const int ri = 16 * t + g + 8 * (k >> 1);
+                    if (b < G.batch) base[static_cast<size_t>(ri) * G.batch + b] = acc[t][u][k];
+                }
+    }
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int u = 0; u < NBP; ++u)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[t][u][k] = 0.f;
+}
+
+// Root byte vectors: entry 0 = no root, entry 1 + i = root i; bytes R + 2,
+// even coordinates in .x, odd coordinates in .y.
+__device__ __forceinline__ uint2 gv_root_entry(int i) {
+    if (i == 0) return make_uint2(0x02020202u, 0x02020202u);
+    if (i > 240) return make_uint2(0u, 0u);
+    const uint2 rw = g_root8[i - 1];
+    unsigned lo = 0, hi = 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+        const int c_even = static_cast<int8_t>(((k < 2 ? rw.x : rw.y) >> (16 * (k & 1))) & 0xFF);
+        const int c_odd = static_cast<int8_t>(((k < 2 ? rw.x : rw.y) >> (16 * (k & 1) + 8)) & 0xFF);
+        lo |= static_cast<unsigned>(c_even + 2) << (8 * k);
+        hi |= static_cast<unsigned>(c_odd + 2) << (8 * k);
+    }
+    return make_uint2(lo, hi);
+}
+
+template <int NBP>
+__global__ void __launch_bounds__(kGvThreads, 1) k_gv_main(const __grid_constant__ GvMainParams p) {
+    extern __shared__ __align__(16) unsigned char smem[];
+    uint32_t* s_tab = reinterpret_cast<uint32_t*>(smem);
+    uint2* s_root = reinterpret_cast<uint2*>(smem + kGvTabBytes);
+    const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, g = lane >> 2, q = lane & 3;
+    const GvGeom& G = p.g;
+    const long long cta = blockIdx.x;
+    const long long lo = cta * G.ksteps / G.nctas, hi = (cta + 1) * G.ksteps / G.nctas;
+    const long long vbeg = lo >> 3, vend = (hi + 7) >> 3;
+    int rb = static_cast<int>(vbeg / G.nchunks), c = static_cast<int>(vbeg % G.nchunks);
+    pdl_launch_dependents();
+    // prologue independent of the prep kernel: first indices, shared tables
+    GvVisit cur;
+    if (lo < hi) gv_load_idx(p, rb, c, warp, g, q, cur);
+    for (int i = threadIdx.x; i < kGvTabN / 4; i += kGvThreads)
+        reinterpret_cast<uint4*>(s_tab)[i] = __ldg(reinterpret_cast<const uint4*>(g_gv_tab) + i);
+    for (int i = threadIdx.x; i < 256; i += kGvThreads) s_root[i] = gv_root_entry(i);
+    __syncthreads();
+    pdl_wait();  // activations and root map written by the prep kernel
+    if (lo >= hi) return;
+    gv_load_map(p, rb, c, warp, g, q, cur);
+
+    bool bok[NBP];
+#pragma unroll
+    for (int u = 0; u < NBP; ++u) bok[u] = 8 * (p.v0 + u) + g < G.batch;
+
+    float acc[2][NBP][4];
+#pragma unroll
+    for (int t = 0; t < 2; ++t)
+#pragma unroll
+        for (int u = 0; u < NBP; ++u)
+#pragma unroll
+            for (int k = 0; k < 4; ++k) acc[t][u][k] = 0.f;
+
+    int cur_rb = rb;
+    for (long long v = vbeg; v < vend; ++v) {
+        GvVisit nxt;
+        int nrb = rb, nc = c + 1;
+        if (nc == G.nchunks) {
+            nc = 0;
+            ++nrb;
+        }
+        if (v + 1 < vend) {
+            gv_load_idx(p, nrb, nc, warp, g, q, nxt);
+            gv_load_map(p, nrb, nc, warp, g, q, nxt);
+        }
+        if (rb != cur_rb) {
+            gv_flush<NBP>(p, acc, cur_rb, warp, g, q);
+            cur_rb = rb;
+        }
+        const int j0 = v == vbeg ? static_cast<int>(lo & 7) : 0;
+        const int j1 = v == vend - 1 ? static_cast<int>(((hi - 1) & 7) + 1) : 8;
+        const int vg = G.gpr - 32 * c < 32 ? G.gpr - 32 * c : 32;  // valid groups in this chunk
+        const int lim = vg - 8 * q;
+        const uint4* xs = p.x16 + (static_cast<size_t>(c) * G.nbt + p.v0) * 256;
+        unsigned any = 0;
+#pragma unroll
+        for (int r = 0; r < 4; ++r) any |= cur.map[r].x | cur.map[r].y;
+        if (__any_sync(0xFFFFFFFFu, any != 0))
+            gv_visit<NBP, true>(acc, cur, s_tab, s_root, xs, bok, lim, j0, j1, lane);
+        else
+            gv_visit<NBP, false>(acc, cur, s_tab, s_root, xs, bok, lim, j0, j1, lane);
+        cur = nxt;
+        rb = nrb;
+        c = nc;
+    }
+    gv_flush<NBP>(p, acc, cur_rb, warp, g, q);
+}
+
+// ---------------------------------------------------------------------------
+// finalize
+// ---------------------------------------------------------------------------
+struct GvFinParams {
+    const float* part;
+    const float* xe;
+    const float* x32;
+    const float* scale;
+    const e8q_overflow* ovf;
+    const int64_t* ovf_rp;
+    uint16_t* y;  // bf16 [batch][rows]
+    long long ovf_n;
+    long long group_base;
+    GvGeom g;
+    int32_t bl_log;  // log2 of the batch lanes: lanes = record lane * BL + batch lane
+};
+
+// Lanes = record lane rl (slots / overflow records) x batch lane bl; each
+// lane holds KB batch rows bl, bl + BL, ...; one shuffle reduction over rl.
+template <int KB>
+__global__ void __launch_bounds__(256) k_gv_fin(const __grid_constant__ GvFinParams p) {
+    pdl_wait();  // partial sums of the main kernel
+    const GvGeom& G = p.g;
     const int lane = threadIdx.x & 31;
-    const int warps = gridDim.x * (kGemvThreads / 32);
-    const int C = p.cols, gpr = C >> 3;
-    for (int r = blockIdx.x * (kGemvThreads / 32) + (threadIdx.x >> 5); r < p.rows; r += warps) {
-        const float s = p.scale[r];
-        const size_t g0 = static_cast<size_t>(r) * gpr;
-        for (int bc = 0; bc < p.batch; bc += 8) {
-            const int nb = min(8, p.batch - bc);
-            float acc[8];
+    const int r = blockIdx.x * 8 + (threadIdx.x >> 5);
+    if (r >= G.rows) return;
+    const int BL = 1 << p.bl_log, RL = 32 >> p.bl_log;
+    const int bl = lane & (BL - 1), rl = lane >> p.bl_log;
+    const int rb = r / kGvBlockRows, ri = r % kGvBlockRows;
+    const long long ks = static_cast<long long>(G.nchunks) * 8;
+    const long long c0 = gv_cta_of(static_cast<long long>(rb) * ks, G.ksteps, G.nctas);
+    const long long c1 = gv_cta_of(static_cast<long long>(rb) * ks + ks - 1, G.ksteps, G.nctas);
+    const int nsl = static_cast<int>(c1 - c0 + 1 < G.maxslots ? c1 - c0 + 1 : G.maxslots);
+    const float* pb = p.part + (static_cast<size_t>(rb) * G.maxslots * kGvBlockRows + ri) * G.batch;
+    const size_t sstride = static_cast<size_t>(kGvBlockRows) * G.batch;
+    float acc[KB];
 #pragma unroll
-            for (int b = 0; b < 8; ++b) acc[b] = 0.f;
-            for (int g = lane; g < gpr; g += 32) {
-                const uint2 cw = g_core8[p.idx[g0 + g]];
-                float P[8];
+    for (int k = 0; k < KB; ++k) {
+        const int b = bl + BL * k;
+        float v = 0.f;
+        if (b < G.batch) {
+#pragma unroll 4
+            for (int sl = rl; sl < nsl; sl += RL) v += __ldcg(pb + sl * sstride + b);
+            v *= p.xe[b];
+        }
+        acc[k] = v;
+    }
+    if (p.ovf_rp) {
+        const long long o0 = gv_clamp(p.ovf_rp[r], 0, p.ovf_n);
+        const long long o1 = gv_clamp(p.ovf_rp[r + 1], o0, p.ovf_n);
+        const long long g0 = p.group_base + static_cast<long long>(r) * G.gpr;
+        for (long long oc = o0; oc < o1; oc += 4 * RL) {
+            // up to 4 records per lane: records first, then activations
+            int gls[4];
+            int cw[4][4];  // coordinate pairs as packed int16
 #pragma unroll
-                for (int i = 0; i < 8; ++i) P[i] = coord_of(cw, i);
+            for (int i = 0; i < 4; ++i) {
+                const long long o = oc + rl + static_cast<long long>(RL) * i;
+                gls[i] = -1;
+                if (o < o1) {
+                    const unsigned* rp = reinterpret_cast<const unsigned*>(p.ovf + o);
+                    const long long gl = static_cast<long long>(__ldg(rp)) - g0;
+                    if (gl >= 0 && gl < G.gpr) gls[i] = static_cast<int>(gl);
 #pragma unroll
-                for (int b = 0; b < 8; ++b)
-                    if (b < nb) {
-                        const float4* x = reinterpret_cast<const float4*>(p.xr + static_cast<size_t>(bc + b) * C) + 2 * g;
-                        const float4 u = x[0], v = x[1];
-                        acc[b] = fmaf(P[0], u.x, fmaf(P[1], u.y, fmaf(P[2], u.z, fmaf(P[3], u.w, acc[b]))));
-                        acc[b] = fmaf(P[4], v.x, fmaf(P[5], v.y, fmaf(P[6], v.z, fmaf(P[7], v.w, acc[b]))));
+                    for (int k = 0; k < 4; ++k) cw[i][k] = static_cast<int>(__ldg(rp + 1 + k));
+                }
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                if (gls[i] < 0) continue;
+                const float* xc = p.x32 + static_cast<size_t>(gls[i]) * 8 * G.batch;
+#pragma unroll
+                for (int k = 0; k < KB; ++k) {
+                    const int b = bl + BL * k;
+                    if (b < G.batch) {
+                        float a = acc[k];
+#pragma unroll
+                        for (int c = 0; c < 8; ++c) {
+                            const int v = (c & 1) ? (cw[i][c >> 1] >> 16) : static_cast<int>(static_cast<int16_t>(cw[i][c >> 1] & 0xFFFF));
+                            a = fmaf(static_cast<float>(v), __ldg(xc + static_cast<size_t>(c) * G.batch + b), a);
+                        }
+                        acc[k] = a;
                     }
-            }
-            if (p.esc_rp) {
-                const long long e1 = min(static_cast<long long>(p.esc_rp[r + 1]), p.esc_n);
-                for (long long e = max(static_cast<long long>(p.esc_rp[r]), 0ll) + lane; e < e1; e += 32) {
-                    const e8q_escape rec = p.esc[e];
-                    const long long gl = static_cast<long long>(rec.group) - p.group_base - static_cast<long long>(g0);
-                    if (gl < 0 || gl >= gpr || rec.root >= 240) continue;
-                    const uint2 rw = g_root8[rec.root];
-#pragma unroll
-                    for (int b = 0; b < 8; ++b)
-                        if (b < nb) {
-                            const float* x = p.xr + static_cast<size_t>(bc + b) * C + 8 * gl;
-#pragma unroll
-                            for (int i = 0; i < 8; ++i) acc[b] = fmaf(static_cast<float>(coord_of(rw, i)), x[i], acc[b]);
-                        }
                 }
             }
-            if (p.ovf_rp) {
-                const long long o1 = min(static_cast<long long>(p.ovf_rp[r + 1]), p.ovf_n);
-                for (long long o = max(static_cast<long long>(p.ovf_rp[r]), 0ll) + lane; o < o1; o += 32) {
-                    const e8q_overflow rec = p.ovf[o];
-                    const long long gl = static_cast<long long>(rec.group) - p.group_base - static_cast<long long>(g0);
-                    if (gl < 0 || gl >= gpr) continue;
+        }
+    }
 #pragma unroll
-                    for (int b = 0; b < 8; ++b)
-                        if (b < nb) {
-                            const float* x = p.xr + static_cast<size_t>(bc + b) * C + 8 * gl;
+    for (int k = 0; k < KB; ++k)
+        for (int off = BL; off < 32; off <<= 1) acc[k] += __shfl_xor_sync(0xFFFFFFFFu, acc[k], off);
+    if (rl == 0) {
+        const float s = 0.5f * p.scale[r];
 #pragma unroll
-                            for (int i = 0; i < 8; ++i) acc[b] = fmaf(static_cast<float>(rec.coord2[i]), x[i], acc[b]);
-                        }
-                }
-            }
-#pragma unroll
-            for (int b = 0; b < 8; ++b) {
-#pragma unroll
-                for (int off = 16; off > 0; off >>= 1) acc[b] += __shfl_xor_sync(0xFFFFFFFFu, acc[b], off);
-            }
-            if (lane < nb) {
-                float v = acc[0];
-#pragma unroll
-                for (int b = 1; b < 8; ++b)
-                    if (lane == b) v = acc[b];
-                p.y[static_cast<size_t>(bc + lane) * p.rows + r] = __bfloat16_as_ushort(__float2bfloat16_rn(0.5f * s * v));
-            }
+        for (int k = 0; k < KB; ++k) {
+            const int b = bl + BL * k;
+            if (b < G.batch)
+                p.y[static_cast<size_t>(b) * G.rows + r] = __bfloat16_as_ushort(__float2bfloat16_rn(s * acc[k]));
         }
     }
 }

@@ -205,7 +205,11 @@ e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_
  */
 e8q_status e8q_decode(const e8q_encoded* m /* host */, int32_t basis, void* out_bf16, e8q_stream stream);
 
-/* Workspace bytes e8q_dequant_gemv needs for this matrix and batch. */
+/*
+ * Workspace bytes e8q_dequant_gemv needs for this matrix and batch (an upper
+ * bound valid on any device; 256 for arguments the GEMV would reject).
+ * Needs no GPU.
+ */
 size_t e8q_gemv_workspace_bytes(const e8q_encoded* m /* host */, int32_t batch);
 
 /*
@@ -213,8 +217,25 @@ size_t e8q_gemv_workspace_bytes(const e8q_encoded* m /* host */, int32_t batch);
  * 2-bit representation):
  *   y[b][r] = sum_c w~[r][c] x[b][c],  w~ = d (.) H_B (s_r p) / sqrt(B)
  *           = s_r * sum_g < p_rg , (H_B (d (.) x_b) / sqrt(B))_g >,
- * fp32 accumulation, bf16 output.  x: [batch][cols] bf16; y: [batch][rows]
- * bf16; 1 <= batch <= 256.  ws: at least e8q_gemv_workspace_bytes().
+ * with p_rg = core[idx] (+ the root of an escape record, or the point of an
+ * overflow record).  x: [batch][cols] bf16, 16-byte aligned; y: [batch][rows]
+ * bf16; 1 <= batch <= 256; m->signs required; m->esc 8-byte aligned.  ws: device memory of at least
+ * e8q_gemv_workspace_bytes(m, batch) bytes, 256-byte aligned, owned by the
+ * caller, overwritten.
+ *
+ * Escape and overflow records must be listed per row through the CSR row
+ * pointers and sorted by group within each row (e8q_project_encode writes
+ * them so); records outside their row are ignored and record counts are
+ * clamped to esc_count / ovf_count, so malformed records give wrong values
+ * but no out-of-bounds access.
+ *
+ * Arithmetic: the rotated activations are formed in fp32, then, for the
+ * tensor-core product with the exact integer coordinates, rounded to fp16
+ * after a per-row power-of-two scaling chosen from the row's largest |x| (no
+ * overflow is possible); fp32 accumulation; overflow records use the fp32
+ * values; bf16 output (round to nearest even).  Expected relative error
+ * about 1e-4 of the output norm.  Asynchronous on `stream`; errors:
+ * INVALID_ARG, UNSUPPORTED (cols > 16384), WORKSPACE, CUDA.
  */
 e8q_status e8q_dequant_gemv(const e8q_encoded* m /* host */, const void* x_bf16, int32_t batch, void* y_bf16,
                             void* ws, size_t ws_bytes, e8q_stream stream);

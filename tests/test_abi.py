@@ -136,6 +136,8 @@ def test_decode_and_gemv_reject_bad_args(lib):
     assert lib.e8q_dequant_gemv(ctypes.byref(m), ctypes.c_void_p(0x100000), 0, ctypes.c_void_p(0x100000),
                                 ctypes.c_void_p(0x100000), 1 << 20, None) == 1  # batch 0
     need = lib.e8q_gemv_workspace_bytes(ctypes.byref(m), 4)
-    assert need == 1024
+    # fp32 and fp16 rotated activations, scale exponents, chunk offsets, partial sums
+    assert need % 256 == 0 and need >= 4 * 64 * 4 + 4 * 64 * 2
+    assert lib.e8q_gemv_workspace_bytes(ctypes.byref(m), 257) == 256
     assert lib.e8q_dequant_gemv(ctypes.byref(m), ctypes.c_void_p(0x100000), 4, ctypes.c_void_p(0x100000),
                                 ctypes.c_void_p(0x100000), need - 1, None) == 4

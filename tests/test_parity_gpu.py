@@ -342,6 +342,58 @@ def test_gemv_small(e8q, batch):
     check_gemv(y.cpu().view(torch.int16).numpy(), y_ref, f"gemv b={batch}")
 
 
+@pytest.mark.parametrize("rows,cols,batch,kappa", [
+    (37, 264, 3, 1.0),      # one partial 256-column chunk + RHT block 8, rows not a multiple of 32
+    (129, 8, 1, 1.0),       # one group per row
+    (70, 64, 9, 1.0),       # two batch tiles, ragged second tile
+    (5, 768, 100, 1.0),     # two passes over batch tiles (8 + 5)
+    (33, 2056, 256, 1.0),   # largest batch, 9 chunks, block 8
+    (300, 1536, 17, 2.5),   # many escapes and overflow records
+])
+def test_gemv_shapes(e8q, rows, cols, batch, kappa):
+    rng = np.random.default_rng(rows * 7 + cols)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((rows, cols)) * 0.02)
+    d = synth.signs(rows, cols)
+    B = oracle.default_block(cols)
+    enc, res = run_encode(e8q, [w], [d], 0, kappa=kappa)
+    st = compare_all(e8q, res, [w], [d], [B], kappa=kappa, label="gemv_shape")[0]
+    if kappa > 2:
+        ctr = res.read_counters()
+        assert ctr["n_escape"] > rows and ctr["n_overflow"] > 0, ctr
+    xb = synth.gemv_x(batch, cols)
+    y = e8q.Gemv(res.encoded[0], batch)(dev_bf16(xb))
+    torch.cuda.synchronize()
+    y_ref = oracle.gemv(st["points"], res.scale[0].cpu().numpy().astype(np.float64), d, B,
+                        synth.bf16_bits_to_f64(xb))
+    check_gemv(y.cpu().view(torch.int16).numpy(), y_ref, f"gemv {rows}x{cols} b={batch}")
+
+
+def test_gemv_large_activations(e8q):
+    """Activations near the bf16 range limit: the per-row power-of-two
+    scaling keeps the fp16 operand finite."""
+    rng = np.random.default_rng(11)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((64, 2048)) * 0.02)
+    d = synth.signs(3, 2048)
+    enc, res = run_encode(e8q, [w], [d], 0)
+    st = compare_all(e8q, res, [w], [d], [2048], label="gemv_big_x")[0]
+    x = rng.standard_normal((4, 2048))
+    x[0] *= 1e30
+    x[1] *= 1e-30
+    x[2, 5] = 3e33  # one outlier
+    xb = synth.f64_to_bf16_bits(x)
+    y = e8q.Gemv(res.encoded[0], 4)(dev_bf16(xb))
+    torch.cuda.synchronize()
+    y_ref = oracle.gemv(st["points"], res.scale[0].cpu().numpy().astype(np.float64), d, 2048,
+                        synth.bf16_bits_to_f64(xb))
+    got = synth.bf16_bits_to_f64(y.cpu().view(torch.int16).numpy().view(np.uint16))
+    assert np.isfinite(got).all()
+    for b in (0, 1, 3):
+        check_gemv(y.cpu().view(torch.int16).numpy()[b:b + 1], y_ref[b:b + 1], f"gemv big x row {b}")
+    # row 2: one huge entry dominates; compare normwise only
+    rel = np.linalg.norm(got[2] - y_ref[2]) / np.linalg.norm(y_ref[2])
+    assert rel < 1e-2, rel
+
+
 # ----------------------------------------------------------------------
 # full-size workloads, in the launch configuration bench.py times
 # ----------------------------------------------------------------------
