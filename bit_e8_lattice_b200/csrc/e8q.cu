@@ -66,13 +66,13 @@ e8q_status ensure_device(int* dev_out) {
             st = cuda_ok(cudaMemcpyToSymbol(g_gv_tab, words.data(), words.size() * sizeof(uint32_t)));
         }
         if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<1, 1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
         if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
         if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
         if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<2, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
         // prep and finalize leave the SM configured for the main kernel's shared
         // memory, so that its CTAs can start while they are still running
         if (st == E8Q_OK)
@@ -165,7 +165,7 @@ TileCounts count_tiles(const e8q_matrix* mats, int n) {
 size_t status_bytes(const TileCounts& tc) { return align256(16 + 8 * static_cast<size_t>(tc.generic)); }
 size_t scratch_bytes(const TileCounts& tc) {
     const int64_t ctas = tc.fast < kFastMaxCtas ? tc.fast : kFastMaxCtas;
-    return static_cast<size_t>(ctas) * 3 * kFastTileGroups * 16;
+    return static_cast<size_t>(ctas) * kFastSlots * kFastTileGroups * 16;
 }
 
 e8q_status check_encoded(const e8q_encoded* m, int* logb) {
@@ -224,7 +224,8 @@ e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_
     if (n_mats > kMaxMats) return E8Q_ERR_UNSUPPORTED;
     if (!a->counters || !(a->kappa > 0.f) || !std::isfinite(a->kappa)) return E8Q_ERR_INVALID_ARG;
     if (a->dequant < E8Q_DEQUANT_NONE || a->dequant > E8Q_DEQUANT_ORIGINAL) return E8Q_ERR_INVALID_ARG;
-    if (a->esc_cap < 0 || a->ovf_cap < 0 || (a->esc_cap > 0 && !a->esc) || (a->ovf_cap > 0 && !a->ovf))
+    if (a->esc_cap < 0 || a->ovf_cap < 0 || (a->esc_cap > 0 && (!a->esc || !aligned(a->esc, 8))) ||
+        (a->ovf_cap > 0 && (!a->ovf || !aligned(a->ovf, 4))))
         return E8Q_ERR_INVALID_ARG;
     if (a->scale_in != 0 && a->scale_in != 1) return E8Q_ERR_INVALID_ARG;
 
@@ -422,10 +423,11 @@ e8q_status e8q_dequant_gemv(const e8q_encoded* m, const void* x_bf16, int32_t ba
     for (int v0 = 0; v0 < g.nbt; v0 += kGvPassTiles) {
         const int nt = g.nbt - v0 < kGvPassTiles ? g.nbt - v0 : kGvPassTiles;
         mp.v0 = v0;
-        if (nt == 1) st = launch_pdl(k_gv_main<1>, grid, kGvThreads, kGvSmemBytes, s, mp);
-        else if (nt == 2) st = launch_pdl(k_gv_main<2>, grid, kGvThreads, kGvSmemBytes, s, mp);
-        else if (nt <= 4) st = launch_pdl(k_gv_main<4>, grid, kGvThreads, kGvSmemBytes, s, mp);
-        else st = launch_pdl(k_gv_main<8>, grid, kGvThreads, kGvSmemBytes, s, mp);
+        // batch tiles <= 2: one 16-row tile per warp, 16 warps; else two tiles, 8 warps
+        if (nt == 1) st = launch_pdl(k_gv_main<1, 1>, grid, 512, kGvSmemBytes, s, mp);
+        else if (nt == 2) st = launch_pdl(k_gv_main<1, 2>, grid, 512, kGvSmemBytes, s, mp);
+        else if (nt <= 4) st = launch_pdl(k_gv_main<2, 4>, grid, 256, kGvSmemBytes, s, mp);
+        else st = launch_pdl(k_gv_main<2, 8>, grid, 256, kGvSmemBytes, s, mp);
         if (st != E8Q_OK) return st;
     }
 
@@ -473,7 +475,8 @@ extern "C" e8q_status e8q_project_encode_noalloc(const e8q_matrix* mats, int32_t
     if (n_mats > kMaxMats) return E8Q_ERR_UNSUPPORTED;
     if (!a->counters || !(a->kappa > 0.f) || !std::isfinite(a->kappa)) return E8Q_ERR_INVALID_ARG;
     if (a->dequant < E8Q_DEQUANT_NONE || a->dequant > E8Q_DEQUANT_ORIGINAL) return E8Q_ERR_INVALID_ARG;
-    if (a->esc_cap < 0 || a->ovf_cap < 0 || (a->esc_cap > 0 && !a->esc) || (a->ovf_cap > 0 && !a->ovf))
+    if (a->esc_cap < 0 || a->ovf_cap < 0 || (a->esc_cap > 0 && (!a->esc || !aligned(a->esc, 8))) ||
+        (a->ovf_cap > 0 && (!a->ovf || !aligned(a->ovf, 4))))
         return E8Q_ERR_INVALID_ARG;
     if (a->scale_in != 0 && a->scale_in != 1) return E8Q_ERR_INVALID_ARG;
 

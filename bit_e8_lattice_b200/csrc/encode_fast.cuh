@@ -27,7 +27,7 @@
 namespace e8q {
 
 constexpr int kFastWarps = 8;
-constexpr int kFastThreads = (kFastWarps + 1) * 32;
+constexpr int kFastThreads = (kFastWarps + 1) * 32;  // compute warps, service warp
 constexpr int kFastTileElems = 16384;
 constexpr int kFastTileGroups = kFastTileElems / 8;
 constexpr int kFastMaxCtas = 160;
@@ -38,15 +38,18 @@ __host__ __device__ inline int fast_rows_per_tile(int cols) {
     return r < 1 ? 1 : (r > kMaxTileRows ? kMaxTileRows : r);
 }
 
+// Pipeline depth: a tile's map, chunk counts and overflow scratch live for
+// four iterations (computed, counted, placed, emitted).
+constexpr int kFastSlots = 4;
+
 // shared-memory layout (bytes)
-constexpr int kFsIn = 0;                                      // bf16 [2][16384]
-constexpr int kFsT1 = kFsIn + 2 * kFastTileElems * 2;         // 65536
+constexpr int kFsIn = 0;                                              // bf16 [2][16384]
+constexpr int kFsT1 = kFsIn + 2 * kFastTileElems * 2;                 // 65536
 constexpr int kFsT2 = kFsT1 + kEncT1Bytes;
-constexpr int kFsMap = kFsT2 + kEncT2Bytes;                   // u32 [3][2048]
-constexpr int kFsIdx = kFsMap + 3 * kFastTileGroups * 4;      // u16 [2][2048]
-constexpr int kFsGss = kFsIdx + 2 * kFastTileGroups * 2;      // f32 [2048]
-constexpr int kFsChunk = kFsGss + kFastTileGroups * 4;        // u32 [3][2][65]
-constexpr int kFsRootKey = kFsChunk + 3 * 2 * 65 * 4 + 8;      // u8 [512]
+constexpr int kFsMap = kFsT2 + kEncT2Bytes;                           // u32 [4][2048]
+constexpr int kFsIdx = kFsMap + kFastSlots * kFastTileGroups * 4;     // u16 [2][2048]
+constexpr int kFsChunk = kFsIdx + 2 * kFastTileGroups * 2;            // u32 [4][2][65]
+constexpr int kFsRootKey = kFsChunk + kFastSlots * 2 * 65 * 4 + 8;    // u8 [512]
 constexpr int kFastSmemBytes = kFsRootKey + 512;
 
 struct FastTile {
@@ -221,37 +224,53 @@ __device__ __forceinline__ void load_window_raw(unsigned (&raw)[8][4], const uin
     }
 }
 
-// Escape search for one queued group (entry: group | P0, P1 | P2, ... P7 | flag).
-__device__ __forceinline__ void resolve_entry(const uint32_t* e, const uint16_t* st1, const uint16_t* st2,
-                                              const uint8_t* rootkey, uint32_t* map, int16_t* ovf_scratch,
-                                              unsigned long long& clamped) {
-    const int g = static_cast<int>(e[0] & 0xFFFFu);
-    int P[8];
-    P[0] = static_cast<int16_t>(e[0] >> 16);
-    P[1] = static_cast<int16_t>(e[1] & 0xFFFFu);
-    P[2] = static_cast<int16_t>(e[1] >> 16);
-    P[3] = static_cast<int16_t>(e[2] & 0xFFFFu);
-    P[4] = static_cast<int16_t>(e[2] >> 16);
-    P[5] = static_cast<int16_t>(e[3] & 0xFFFFu);
-    P[6] = static_cast<int16_t>(e[3] >> 16);
-    P[7] = static_cast<int16_t>(e[4] & 0xFFFFu);
-    int Q[8], key, n2 = 0;
+// Escape search for queued groups (entry: group | P0, P1 | P2, ... P7 | flag),
+// N per lane: all entries are read before any result is stored, so the
+// independent searches overlap.
+template <int N>
+__device__ __forceinline__ void resolve_entries(const uint32_t* q, const int (&slot)[N], const bool (&ok)[N],
+                                                const uint16_t* st1, const uint16_t* st2, const uint8_t* rootkey,
+                                                uint32_t* map, int16_t* ovf_scratch, unsigned long long& clamped) {
+    uint32_t e[N][5];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) n2 += P[i] * P[i];
-    const int v = escape_search(P, Q, key);
-    const int rq = core_rank_n2(Q, n2 - 2 * v + 8, st1, st2);  // |P - R|^2 = |P|^2 - 2 <P, R> + |R|^2
-    if (rq >= 0) {
-        const uint32_t rr = rootkey[key];
-        map[map_slot(g)] = static_cast<uint32_t>(rq) | (rr << 16) | (1u << 24);
-    } else {
-        map[map_slot(g)] = 2u << 24;
-        uint4 o;
-        o.x = (e[0] >> 16) | (e[1] << 16);
-        o.y = (e[1] >> 16) | (e[2] << 16);
-        o.z = (e[2] >> 16) | (e[3] << 16);
-        o.w = (e[3] >> 16) | (e[4] << 16);
-        *reinterpret_cast<uint4*>(ovf_scratch + 8 * g) = o;
-        if (e[4] & 0x10000u) ++clamped;
+    for (int n = 0; n < N; ++n)
+#pragma unroll
+        for (int k = 0; k < 5; ++k) e[n][k] = ok[n] ? q[5 * slot[n] + k] : 0u;
+    uint32_t out[N];
+    int rq[N];
+#pragma unroll
+    for (int n = 0; n < N; ++n) {
+        int P[8];
+        P[0] = static_cast<int16_t>(e[n][0] >> 16);
+        P[1] = static_cast<int16_t>(e[n][1] & 0xFFFFu);
+        P[2] = static_cast<int16_t>(e[n][1] >> 16);
+        P[3] = static_cast<int16_t>(e[n][2] & 0xFFFFu);
+        P[4] = static_cast<int16_t>(e[n][2] >> 16);
+        P[5] = static_cast<int16_t>(e[n][3] & 0xFFFFu);
+        P[6] = static_cast<int16_t>(e[n][3] >> 16);
+        P[7] = static_cast<int16_t>(e[n][4] & 0xFFFFu);
+        int Q[8], key, n2 = 0;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) n2 += P[i] * P[i];
+        const int v = escape_search_keys(P, Q, key);
+        rq[n] = core_rank_n2(Q, n2 - 2 * v + 8, st1, st2);  // |P - R|^2 = |P|^2 - 2 <P, R> + |R|^2
+        out[n] = rq[n] >= 0 ? (static_cast<uint32_t>(rq[n]) | (static_cast<uint32_t>(rootkey[key]) << 16) | (1u << 24))
+                            : (2u << 24);
+    }
+#pragma unroll
+    for (int n = 0; n < N; ++n) {
+        if (!ok[n]) continue;
+        const int g = static_cast<int>(e[n][0] & 0xFFFFu);
+        map[map_slot(g)] = out[n];
+        if (rq[n] < 0) {
+            uint4 o;
+            o.x = (e[n][0] >> 16) | (e[n][1] << 16);
+            o.y = (e[n][1] >> 16) | (e[n][2] << 16);
+            o.z = (e[n][2] >> 16) | (e[n][3] << 16);
+            o.w = (e[n][3] >> 16) | (e[n][4] << 16);
+            *reinterpret_cast<uint4*>(ovf_scratch + 8 * g) = o;
+            if (e[n][4] & 0x10000u) ++clamped;
+        }
     }
 }
 
@@ -274,6 +293,71 @@ __device__ __forceinline__ FastTile make_tile(const EncodeParams<MAXM>& p, int t
     return ft;
 }
 
+// Row scales of a tile, from its input: the blockwise RHT is orthonormal,
+// so the rotated row's sum of squares is the (sign-flipped) input row's.
+// One warp, rows in turn, fixed summation order; a row whose sum is not
+// finite is summed again with non-finite inputs read as 0, as the transform
+// reads them.  s_r = sqrt(sum / C) / kappa (or the given scale).
+template <int MAXM>
+__device__ __forceinline__ void tile_scales(const EncodeParams<MAXM>& p, const FastTile& ft, const uint16_t* tb,
+                                            float* rows, float* rowc, float* rowm, int lane) {
+    const MatDesc& M = p.m[ft.mat];
+    const int C = M.cols;
+    const float sqb = sqrtf(static_cast<float>(1 << meta_logb(M.meta)));
+    for (int r = 0; r < ft.nr; ++r) {
+        const uint4* row = reinterpret_cast<const uint4*>(tb + r * C);
+        float ss = 0.f;
+        if (!p.scale_in) {
+            float2 acc = make_float2(0.f, 0.f);
+            for (int k = lane; k < C / 8; k += 32) {
+                const uint4 v = row[k];
+                const unsigned w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const float2 t = make_float2(__uint_as_float(w[j] << 16), __uint_as_float(w[j] & 0xFFFF0000u));
+                    acc = __ffma2_rn(t, t, acc);
+                }
+            }
+            ss = acc.x + acc.y;
+#pragma unroll
+            for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
+            ss = __shfl_sync(0xFFFFFFFFu, ss, 0);
+            if (!isfinite(ss)) {
+                acc = make_float2(0.f, 0.f);
+                for (int k = lane; k < C / 8; k += 32) {
+                    const uint4 v = row[k];
+                    const unsigned w[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+                    for (int j = 0; j < 4; ++j) {
+                        unsigned x = w[j];
+                        if ((x & 0x7F80u) == 0x7F80u) x &= 0xFFFF0000u;
+                        if ((x & 0x7F800000u) == 0x7F800000u) x &= 0x0000FFFFu;
+                        const float2 t = make_float2(__uint_as_float(x << 16), __uint_as_float(x & 0xFFFF0000u));
+                        acc = __ffma2_rn(t, t, acc);
+                    }
+                }
+                ss = acc.x + acc.y;
+#pragma unroll
+                for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
+                ss = __shfl_sync(0xFFFFFFFFu, ss, 0);
+            }
+        }
+        if (lane == 0) {
+            float sc;
+            if (p.scale_in) {
+                sc = M.scale[ft.r0 + r];
+                if (!(sc > 0.f) || !isfinite(sc)) sc = 0.f;
+            } else {
+                sc = sqrtf(ss / static_cast<float>(C)) / p.kappa;
+                M.scale[ft.r0 + r] = sc;
+            }
+            rows[r] = sc;
+            rowc[r] = sc > 0.f ? 2.0f / (sc * sqb) : 0.f;
+            rowm[r] = sc / sqb;
+        }
+    }
+}
+
 template <int MAXM>
 __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_constant__ EncodeParams<MAXM> p,
                                                                   int16_t* __restrict__ ovf_scratch_all) {
@@ -283,19 +367,18 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
     uint16_t* st2 = reinterpret_cast<uint16_t*>(smem + kFsT2);
     uint32_t* smap = reinterpret_cast<uint32_t*>(smem + kFsMap);
     uint16_t* sidx = reinterpret_cast<uint16_t*>(smem + kFsIdx);
-    float* sgss = reinterpret_cast<float*>(smem + kFsGss);
     uint32_t* schunk = reinterpret_cast<uint32_t*>(smem + kFsChunk);
     uint8_t* srootkey = smem + kFsRootKey;
 
     __shared__ __align__(8) uint64_t s_full[2];
-    __shared__ FastTile s_info[4];
-    __shared__ float s_rss[kMaxTileRows], s_rows[kMaxTileRows], s_rowc[kMaxTileRows], s_rowm[kMaxTileRows];
-    __shared__ float s_wss[kFastWarps];
-    __shared__ unsigned s_ex[3][2];
+    __shared__ FastTile s_info[8];  // tile of iteration i at i & 7
+    __shared__ float s_rows[2][kMaxTileRows], s_rowc[2][kMaxTileRows], s_rowm[2][kMaxTileRows];
+    __shared__ unsigned s_tot[kFastSlots][2];  // a tile's escape / overflow record counts
+    __shared__ unsigned s_ex[kFastSlots][2];   // records of all earlier tiles
 
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const bool service = warp == kFastWarps;
-    int16_t* ovf_scratch = ovf_scratch_all + static_cast<size_t>(blockIdx.x) * 3 * kFastTileGroups * 8;
+    int16_t* ovf_scratch = ovf_scratch_all + static_cast<size_t>(blockIdx.x) * kFastSlots * kFastTileGroups * 8;
     unsigned long long* status = p.ws + 2;
 
     {  // constant tables
@@ -310,7 +393,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
         fence_mbar_init();
-        for (int s = 0; s < 4; ++s) s_info[s] = make_tile(p, 0x7FFFFFFF);
+        for (int s = 0; s < 8; ++s) s_info[s] = make_tile(p, 0x7FFFFFFF);
         const int t0 = static_cast<int>(atomicAdd(&p.ws[0], 1ull));
         s_info[0] = make_tile(p, t0);
         if (t0 < p.n_tiles) {
@@ -323,18 +406,35 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
         }
     }
     __syncthreads();
+    if (service && s_info[0].t < p.n_tiles) {  // row scales of the first tile
+        int spins = 0;
+        while (!mbar_try_wait(&s_full[0], 0)) {
+            if (++spins > kWaitLimit) {
+                if (lane == 0) atomicOr(&p.ctr->err, 2ull);
+                break;
+            }
+        }
+        tile_scales(p, s_info[0], inbuf, s_rows[0], s_rowc[0], s_rowm[0], lane);
+    }
+    __syncthreads();
 
     const HFrag hf = make_hfrag(lane);
     unsigned long long nonfinite = 0, clamped = 0;
 
+    // Iteration i: compute warps transform, project and count tile i and emit
+    // the records of tile i - 3; the service warp claims and loads tile i + 1,
+    // publishes tile i - 1's record counts and stores its indices, places
+    // tile i - 2 among all earlier tiles, and computes tile i + 1's row
+    // scales.  One barrier per iteration.
     for (int i = 0;; ++i) {
-        const FastTile cur = s_info[i & 3];
-        const FastTile prev1 = s_info[(i + 3) & 3];
-        const FastTile prev2 = s_info[(i + 2) & 3];
+        const FastTile cur = s_info[i & 7];
+        const FastTile prev1 = s_info[(i + 7) & 7];
+        const FastTile prev2 = s_info[(i + 6) & 7];
+        const FastTile prev3 = s_info[(i + 5) & 7];
         const bool cur_ok = cur.t < p.n_tiles, p1_ok = i >= 1 && prev1.t < p.n_tiles,
-                   p2_ok = i >= 2 && prev2.t < p.n_tiles;
-        if (!cur_ok && !p1_ok && !p2_ok) break;
-        const int b = i & 1, msl = i % 3, msl2 = (i + 1) % 3;
+                   p2_ok = i >= 2 && prev2.t < p.n_tiles, p3_ok = i >= 3 && prev3.t < p.n_tiles;
+        if (!cur_ok && !p1_ok && !p2_ok && !p3_ok) break;
+        const int b = i & 1, sl = i & 3, sl1 = (i + 3) & 3, sl2 = (i + 2) & 3, sl3 = (i + 1) & 3;
 
         if (!service) {
             // ================================================ compute warps
@@ -344,15 +444,9 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                 const int n = cur.nr * C, G = cur.nr * gpr;
                 const int nwin = (n + 2047) >> 11;
                 const bool win_rows = (C & 2047) == 0;  // every window inside one row
-                {  // wait for the tile's bytes (bounded)
-                    int spins = 0;
-                    while (!mbar_try_wait(&s_full[b], (i >> 1) & 1)) {
-                        if (++spins > kWaitLimit) {
-                            if (lane == 0) atomicOr(&p.ctr->err, 2ull);
-                            break;
-                        }
-                    }
-                }
+                const float* rows_b = s_rows[b];
+                const float* rowc_b = s_rowc[b];
+                const float* rowm_b = s_rowm[b];
                 float v[8][8];
                 const int w = warp;
                 const int wbase = 2048 * w;
@@ -360,70 +454,30 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                 uint16_t* win = inbuf + b * kFastTileElems + wbase;
                 float4* scratch = reinterpret_cast<float4*>(win);
                 if (w < nwin) {
+                    {  // wait for the tile's bytes (bounded)
+                        int spins = 0;
+                        while (!mbar_try_wait(&s_full[b], (i >> 1) & 1)) {
+                            if (++spins > kWaitLimit) {
+                                if (lane == 0) atomicOr(&p.ctr->err, 2ull);
+                                break;
+                            }
+                        }
+                    }
                     unsigned raw[8][4];
                     load_window_raw(raw, win, false, M.signs, C, wbase, nchunks, lane, nonfinite);
                     __syncwarp();
-                    float ss = window_forward(v, raw, logb, nchunks, scratch, lane, hf);
+                    const float ss = window_forward(v, raw, logb, nchunks, scratch, lane, hf);
                     if (__any_sync(0xFFFFFFFFu, !isfinite(ss))) {  // non-finite input: redo from global, sanitised
                         const uint16_t* g = static_cast<const uint16_t*>(M.w) + static_cast<size_t>(cur.r0) * C + wbase;
                         load_window_raw(raw, g, true, M.signs, C, wbase, nchunks, lane, nonfinite);
                         __syncwarp();
-                        ss = window_forward(v, raw, logb, nchunks, scratch, lane, hf);
-                    }
-                    if (win_rows) {
-#pragma unroll
-                        for (int off = 16; off > 0; off >>= 1) ss += __shfl_xor_sync(0xFFFFFFFFu, ss, off);
-                        if (lane == 0) s_wss[w] = ss;
-                    } else {
-                        const int a = lane >> 2, q = lane & 3;
-#pragma unroll
-                        for (int h = 0; h < 8; ++h) {
-                            float gs = 0.f;
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) gs = fmaf(v[h][e], v[h][e], gs);
-                            if (a < nchunks) sgss[256 * w + 32 * a + 4 * h + q] = gs;
-                        }
+                        window_forward(v, raw, logb, nchunks, scratch, lane, hf);
                     }
                 }
-                named_bar_sync(1, kFastWarps * 32);
-                // row scales
-                const float Bf = static_cast<float>(1 << logb);
-                if (win_rows) {
-                    if (tid < cur.nr) {
-                        const int wpr = C >> 11;
-                        float ssr = 0.f;
-                        for (int k = 0; k < wpr; ++k) ssr += s_wss[tid * wpr + k];
-                        s_rss[tid] = ssr;
-                    }
-                } else {
-                    for (int r = warp; r < cur.nr; r += kFastWarps) {
-                        float a = 0.f;
-                        for (int g = lane; g < gpr; g += 32) a += sgss[r * gpr + g];
-#pragma unroll
-                        for (int off = 16; off > 0; off >>= 1) a += __shfl_xor_sync(0xFFFFFFFFu, a, off);
-                        if (lane == 0) s_rss[r] = a;
-                    }
-                }
-                named_bar_sync(1, kFastWarps * 32);
-                if (tid < cur.nr) {
-                    float s;
-                    if (p.scale_in) {
-                        s = M.scale[cur.r0 + tid];
-                        if (!(s > 0.f) || !isfinite(s)) s = 0.f;
-                    } else {
-                        s = sqrtf(s_rss[tid] / (Bf * static_cast<float>(C))) / p.kappa;
-                        M.scale[cur.r0 + tid] = s;
-                    }
-                    s_rows[tid] = s;
-                    s_rowc[tid] = (s > 0.f) ? 2.0f / (s * sqrtf(Bf)) : 0.f;
-                    s_rowm[tid] = s / sqrtf(Bf);
-                }
-                named_bar_sync(1, kFastWarps * 32);
-
                 // projection + encoding of the warp's 8 x 32 groups
-                uint32_t* map = smap + msl * kFastTileGroups;
+                uint32_t* map = smap + sl * kFastTileGroups;
                 uint16_t* idxs = sidx + b * kFastTileGroups;
-                int16_t* oscr = ovf_scratch + static_cast<size_t>(msl) * kFastTileGroups * 8;
+                int16_t* oscr = ovf_scratch + static_cast<size_t>(sl) * kFastTileGroups * 8;
                 if (w < nwin) {
                     const int a = lane >> 2, q = lane & 3;
                     const bool lane_ok = a < nchunks;
@@ -436,11 +490,13 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     // original-basis dequant): 5 words per entry, at most 159 live entries
                     uint32_t* qbuf = reinterpret_cast<uint32_t*>(win);
                     int qn = 0;
+                    // the lane's 8 groups are independent: project all of them, then
+                    // rank all of them, then queue, so that the chains overlap
+                    unsigned oddm = 0u;
 #pragma unroll
                     for (int h = 0; h < 8; ++h) {
-                        const int gt = 256 * w + 32 * a + 4 * h + q;
                         const int row = win_rows ? row_w : r0l + (h >= hcut ? 1 : 0);
-                        const float c = s_rowc[lane_ok ? row : 0];
+                        const float c = rowc_b[lane_ok ? row : 0];
                         float X[8];
 #pragma unroll
                         for (int j = 0; j < 4; ++j) {
@@ -453,10 +509,18 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                             for (int e = 0; e < 8; ++e) X[e] = fminf(fmaxf(X[e], -1048576.f), 1048576.f);
                         }
                         float Pf[8];
-                        const bool odd = e8_nearest_lean(X, Pf);
+                        oddm |= (e8_nearest_lean(X, Pf) ? 1u : 0u) << h;
 #pragma unroll
                         for (int e = 0; e < 8; ++e) v[h][e] = Pf[e];  // keep p for the dequant
-                        const int rk = lane_ok ? core_rank_f(Pf, odd, st1, st2) : 0;
+                    }
+                    int rks[8];
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) rks[h] = lane_ok ? core_rank_f(v[h], (oddm >> h) & 1u, st1, st2) : 0;
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) {
+                        const int gt = 256 * w + 32 * a + 4 * h + q;
+                        const float (&Pf)[8] = v[h];
+                        const int rk = rks[h];
                         const bool pend = lane_ok && rk < 0;
                         if (lane_ok && !pend) map[map_slot(gt)] = static_cast<uint32_t>(rk);
                         const unsigned bal = __ballot_sync(0xFFFFFFFFu, pend);
@@ -484,9 +548,12 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                             __syncwarp();
                             int qh = 0;
                             const int until = (h == 7) ? qn : (qn & ~31);
-                            for (; qh < until; qh += 32)
-                                if (qh + lane < qn)
-                                    resolve_entry(qbuf + 5 * (qh + lane), st1, st2, srootkey, map, oscr, clamped);
+                            for (; qh < until; qh += 64) {
+                                const int sl[2] = {qh + lane, qh + 32 + lane};
+                                const bool okk[2] = {qh + lane < until, qh + 32 + lane < until};
+                                resolve_entries<2>(qbuf, sl, okk, st1, st2, srootkey, map, oscr, clamped);
+                            }
+                            qh = until;
                             __syncwarp();
                             if (h == 3 && qh > 0) {  // move the partial batch to the front
                                 const int left = qn - qh;
@@ -511,7 +578,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         for (int h = 0; h < 8; ++h) {
                             if (!lane_ok) continue;
                             const int gt = 256 * w + 32 * a + 4 * h + q;
-                            const float s = s_rows[win_rows ? row_w : r0l + (h >= hcut ? 1 : 0)];
+                            const float s = rows_b[win_rows ? row_w : r0l + (h >= hcut ? 1 : 0)];
                             uint4 o;
                             o.x = pack_bf16x2(bf16_of_product(s, 0.5f * v[h][0]), bf16_of_product(s, 0.5f * v[h][1]));
                             o.y = pack_bf16x2(bf16_of_product(s, 0.5f * v[h][2]), bf16_of_product(s, 0.5f * v[h][3]));
@@ -581,7 +648,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                             if (tc >= C) { tc -= C; ++tr; }
                             if (k >= nchunks) continue;
                             const int te = wbase + 256 * k + 8 * lane;  // tile element of the 8-run
-                            const float m = s_rowm[win_rows ? row_w : rowk];
+                            const float m = rowm_b[win_rows ? row_w : rowk];
                             unsigned o[4];
 #pragma unroll
                             for (int j = 0; j < 4; ++j) {
@@ -593,88 +660,81 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         }
                     }
                 }
-                named_bar_sync(1, kFastWarps * 32);
-                // per-chunk record counts and their prefix (group order)
-                uint32_t* cnt = schunk + msl * 130;
-                const int nch = (G + 31) >> 5;
-                for (int c = warp; c < nch; c += kFastWarps) {
-                    const int g = 32 * c + lane;
-                    const uint32_t m = g < G ? map[map_slot(g)] : 0u;
-                    const uint32_t k = m >> 24;
-                    if (g < G) idxs[g] = static_cast<uint16_t>(k == 2 ? 0u : (m & 0xFFFFu));
-                    const unsigned be = __ballot_sync(0xFFFFFFFFu, k == 1), bo = __ballot_sync(0xFFFFFFFFu, k == 2);
-                    if (lane == 0) {
-                        cnt[c] = __popc(be);
-                        cnt[65 + c] = __popc(bo);
-                    }
-                }
-                named_bar_sync(1, kFastWarps * 32);
-                if (warp == 0) {
-                    unsigned ce0 = lane < nch ? cnt[lane] : 0u, ce1 = lane + 32 < nch ? cnt[lane + 32] : 0u;
-                    unsigned co0 = lane < nch ? cnt[65 + lane] : 0u, co1 = lane + 32 < nch ? cnt[65 + lane + 32] : 0u;
-                    unsigned se0 = ce0, se1 = ce1, so0 = co0, so1 = co1;  // inclusive scans
+                if (w < nwin) {
+                    // the window's record counts per 32-group chunk, and its indices
+                    uint32_t* cnt = schunk + sl * 130;
+                    __syncwarp();
 #pragma unroll
-                    for (int off = 1; off < 32; off <<= 1) {
-                        const unsigned a0 = __shfl_up_sync(0xFFFFFFFFu, se0, off), a1 = __shfl_up_sync(0xFFFFFFFFu, se1, off);
-                        const unsigned b0 = __shfl_up_sync(0xFFFFFFFFu, so0, off), b1 = __shfl_up_sync(0xFFFFFFFFu, so1, off);
-                        if (lane >= off) { se0 += a0; se1 += a1; so0 += b0; so1 += b1; }
-                    }
-                    const unsigned te0 = __shfl_sync(0xFFFFFFFFu, se0, 31), to0 = __shfl_sync(0xFFFFFFFFu, so0, 31);
-                    const unsigned te1 = __shfl_sync(0xFFFFFFFFu, se1, 31), to1 = __shfl_sync(0xFFFFFFFFu, so1, 31);
-                    cnt[lane] = se0 - ce0;
-                    cnt[lane + 32] = te0 + se1 - ce1;
-                    cnt[65 + lane] = so0 - co0;
-                    cnt[65 + lane + 32] = to0 + so1 - co1;
-                    if (lane == 0) {
-                        cnt[64] = te0 + te1;
-                        cnt[65 + 64] = to0 + to1;
-                        s_info[i & 3].ne = te0 + te1;
-                        s_info[i & 3].no = to0 + to1;
+                    for (int k = 0; k < 8; ++k) {
+                        const int c = 8 * w + k;
+                        if (32 * c >= G) break;
+                        const int g = 32 * c + lane;
+                        const uint32_t m = g < G ? map[map_slot(g)] : 0u;
+                        const uint32_t kind = m >> 24;
+                        if (g < G) idxs[g] = static_cast<uint16_t>(kind == 2 ? 0u : (m & 0xFFFFu));
+                        const unsigned be = __ballot_sync(0xFFFFFFFFu, kind == 1), bo = __ballot_sync(0xFFFFFFFFu, kind == 2);
+                        if (lane == 0) {
+                            cnt[c] = __popc(be);
+                            cnt[65 + c] = __popc(bo);
+                        }
                     }
                 }
             }
-            // emit the records of the tile finished two iterations ago, once
-            // the service warp has placed it
-            named_bar_sync(2, kFastThreads);
-            if (p2_ok) {
-                const MatDesc& M = p.m[prev2.mat];
-                const int gpr = M.cols >> 3, G = prev2.nr * gpr, nch = (G + 31) >> 5;
-                const uint32_t* map = smap + msl2 * kFastTileGroups;
-                const uint32_t* cnt = schunk + msl2 * 130;
-                const int16_t* oscr = ovf_scratch + static_cast<size_t>(msl2) * kFastTileGroups * 8;
-                const long long ex_e = s_ex[msl2][0], ex_o = s_ex[msl2][1];
-                const uint32_t gid0 = M.group_base + static_cast<uint32_t>(prev2.r0) * gpr;
-                for (int c = warp; c < nch; c += kFastWarps) {
-                    const int g = 32 * c + lane;
-                    const uint32_t m = g < G ? map[map_slot(g)] : 0u;
-                    const uint32_t k = m >> 24;
-                    const unsigned be = __ballot_sync(0xFFFFFFFFu, k == 1), bo = __ballot_sync(0xFFFFFFFFu, k == 2);
-                    if (k == 1) {
-                        const long long pos = ex_e + cnt[c] + __popc(be & lanemask_lt());
-                        if (pos < p.esc_cap) {
-                            e8q_escape r;
-                            r.group = gid0 + g;
-                            r.core = static_cast<uint16_t>(m & 0xFFFFu);
-                            r.root = static_cast<uint8_t>((m >> 16) & 0xFFu);
-                            r.reserved = 0;
-                            p.esc[pos] = r;
-                        }
-                    } else if (k == 2) {
-                        const long long pos = ex_o + cnt[65 + c] + __popc(bo & lanemask_lt());
-                        if (pos < p.ovf_cap) {
-                            const uint4 cw = *reinterpret_cast<const uint4*>(oscr + 8 * g);
-                            uint32_t* dst = reinterpret_cast<uint32_t*>(p.ovf + pos);
-                            dst[0] = gid0 + g;
-                            dst[1] = cw.x; dst[2] = cw.y; dst[3] = cw.z; dst[4] = cw.w;
+            // emit the records of tile i - 3, placed by the service warp during
+            // the previous iteration: each warp its own window's 8 chunks, all
+            // loads before the ballots and stores
+            if (p3_ok) {
+                const MatDesc& M = p.m[prev3.mat];
+                const int gpr = M.cols >> 3, G = prev3.nr * gpr, nch = (G + 31) >> 5;
+                const uint32_t* map = smap + sl3 * kFastTileGroups;
+                const uint32_t* cnt = schunk + sl3 * 130;
+                const int16_t* oscr = ovf_scratch + static_cast<size_t>(sl3) * kFastTileGroups * 8;
+                const long long ex_e = s_ex[sl3][0], ex_o = s_ex[sl3][1];
+                const uint32_t gid0 = M.group_base + static_cast<uint32_t>(prev3.r0) * gpr;
+                for (int c0 = 8 * warp; c0 < nch && c0 < 8 * warp + 8; c0 += 8) {
+                    uint32_t m[8];
+                    uint4 cw[8];
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int g = 32 * (c0 + k) + lane;
+                        m[k] = (c0 + k < nch && g < G) ? map[map_slot(g)] : 0u;
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int g = 32 * (c0 + k) + lane;
+                        cw[k] = (m[k] >> 24) == 2 ? *reinterpret_cast<const uint4*>(oscr + 8 * g) : make_uint4(0, 0, 0, 0);
+                    }
+#pragma unroll
+                    for (int k = 0; k < 8; ++k) {
+                        const int c = c0 + k;
+                        if (c >= nch) break;
+                        const int g = 32 * c + lane;
+                        const uint32_t kind = m[k] >> 24;
+                        const unsigned be = __ballot_sync(0xFFFFFFFFu, kind == 1), bo = __ballot_sync(0xFFFFFFFFu, kind == 2);
+                        if (kind == 1) {
+                            const long long pos = ex_e + cnt[c] + __popc(be & lanemask_lt());
+                            if (pos < p.esc_cap) {
+                                uint2 r;
+                                r.x = gid0 + g;
+                                r.y = (m[k] & 0xFFFFu) | (((m[k] >> 16) & 0xFFu) << 16);
+                                *reinterpret_cast<uint2*>(p.esc + pos) = r;
+                            }
+                        } else if (kind == 2) {
+                            const long long pos = ex_o + cnt[65 + c] + __popc(bo & lanemask_lt());
+                            if (pos < p.ovf_cap) {
+                                uint32_t* dst = reinterpret_cast<uint32_t*>(p.ovf + pos);
+                                dst[0] = gid0 + g;
+                                dst[1] = cw[k].x; dst[2] = cw[k].y; dst[3] = cw[k].z; dst[4] = cw[k].w;
+                            }
                         }
                     }
                 }
-                if (tid < prev2.nr) {
-                    const int c = (tid * gpr) >> 5;  // rows start on chunk boundaries (gpr % 32 == 0)
-                    if (p.esc_rp) p.esc_rp[M.row_base + prev2.r0 + tid] = ex_e + cnt[c];
-                    if (p.ovf_rp) p.ovf_rp[M.row_base + prev2.r0 + tid] = ex_o + cnt[65 + c];
+                for (int r = tid; r < prev3.nr; r += kFastWarps * 32) {
+                    const int c = (r * gpr) >> 5;  // rows start on chunk boundaries (gpr % 32 == 0)
+                    if (p.esc_rp) p.esc_rp[M.row_base + prev3.r0 + r] = ex_e + cnt[c];
+                    if (p.ovf_rp) p.ovf_rp[M.row_base + prev3.r0 + r] = ex_o + cnt[65 + c];
                 }
-                if (prev2.t == p.n_tiles - 1 && tid == 0) {
+                if (prev3.t == p.n_tiles - 1 && tid == 0) {
                     const long long te = ex_e + cnt[64], to = ex_o + cnt[65 + 64];
                     if (p.esc_rp) p.esc_rp[p.total_rows] = te;
                     if (p.ovf_rp) p.ovf_rp[p.total_rows] = to;
@@ -684,13 +744,13 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                 }
             }
             fence_proxy_async_smem();
-        } else {
+        } else if (service) {
             // ================================================= service warp
             if (lane == 0) {
                 int tn = 0x7FFFFFFF;
                 if (cur_ok) tn = static_cast<int>(atomicAdd(&p.ws[0], 1ull));
                 const FastTile nt = make_tile(p, tn);
-                s_info[(i + 1) & 3] = nt;
+                s_info[(i + 1) & 7] = nt;
                 if (tn < p.n_tiles) {
                     const MatDesc& M = p.m[nt.mat];
                     const unsigned bytes = static_cast<unsigned>(nt.nr) * M.cols * 2u;
@@ -699,11 +759,34 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     bulk_load(inbuf + ((i + 1) & 1) * kFastTileElems,
                               static_cast<const uint16_t*>(M.w) + static_cast<size_t>(nt.r0) * M.cols, bytes, bar);
                 }
-                if (p1_ok) {
-                    const MatDesc& M = p.m[prev1.mat];
-                    const int gpr = M.cols >> 3;
-                    const unsigned long long own =
-                        (static_cast<unsigned long long>(prev1.ne) << 31) | prev1.no;
+            }
+            __syncwarp();
+            if (p1_ok) {  // tile i - 1: chunk prefix (group order), publish its counts, store its indices
+                const MatDesc& M = p.m[prev1.mat];
+                const int gpr = M.cols >> 3, nch = (prev1.nr * gpr + 31) >> 5;
+                uint32_t* cnt = schunk + sl1 * 130;
+                const unsigned ce0 = lane < nch ? cnt[lane] : 0u, ce1 = lane + 32 < nch ? cnt[lane + 32] : 0u;
+                const unsigned co0 = lane < nch ? cnt[65 + lane] : 0u, co1 = lane + 32 < nch ? cnt[65 + lane + 32] : 0u;
+                unsigned se0 = ce0, se1 = ce1, so0 = co0, so1 = co1;  // inclusive scans
+#pragma unroll
+                for (int off = 1; off < 32; off <<= 1) {
+                    const unsigned a0 = __shfl_up_sync(0xFFFFFFFFu, se0, off), a1 = __shfl_up_sync(0xFFFFFFFFu, se1, off);
+                    const unsigned b0 = __shfl_up_sync(0xFFFFFFFFu, so0, off), b1 = __shfl_up_sync(0xFFFFFFFFu, so1, off);
+                    if (lane >= off) { se0 += a0; se1 += a1; so0 += b0; so1 += b1; }
+                }
+                const unsigned te0 = __shfl_sync(0xFFFFFFFFu, se0, 31), to0 = __shfl_sync(0xFFFFFFFFu, so0, 31);
+                const unsigned te1 = __shfl_sync(0xFFFFFFFFu, se1, 31), to1 = __shfl_sync(0xFFFFFFFFu, so1, 31);
+                cnt[lane] = se0 - ce0;
+                cnt[lane + 32] = te0 + se1 - ce1;
+                cnt[65 + lane] = so0 - co0;
+                cnt[65 + lane + 32] = to0 + so1 - co1;
+                if (lane == 0) {
+                    const unsigned ne = te0 + te1, no = to0 + to1;
+                    cnt[64] = ne;
+                    cnt[65 + 64] = no;
+                    s_tot[sl1][0] = ne;
+                    s_tot[sl1][1] = no;
+                    const unsigned long long own = (static_cast<unsigned long long>(ne) << 31) | no;
                     st_volatile_u64(&status[prev1.t], (prev1.t == 0 ? (2ull << 62) : (1ull << 62)) | own);
                     bulk_store(M.idx + static_cast<size_t>(prev1.r0) * gpr, sidx + ((i + 1) & 1) * kFastTileGroups,
                                static_cast<unsigned>(prev1.nr) * gpr * 2u);
@@ -711,15 +794,15 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                 }
             }
             __syncwarp();
-            if (p2_ok) {
+            if (p2_ok) {  // tile i - 2: its place among all earlier tiles' records
                 unsigned ex_e = 0, ex_o = 0;
                 if (prev2.t > 0) {
                     unsigned acc_e = 0, acc_o = 0;
                     int j = prev2.t - 1, spins = 0;
                     while (true) {
                         const int k = j - lane;
-                        const unsigned long long s = (k >= 0) ? ld_volatile_u64(&status[k]) : (2ull << 62);
-                        const unsigned flag = static_cast<unsigned>(s >> 62);
+                        const unsigned long long st = (k >= 0) ? ld_volatile_u64(&status[k]) : (2ull << 62);
+                        const unsigned flag = static_cast<unsigned>(st >> 62);
                         const unsigned notready = __ballot_sync(0xFFFFFFFFu, flag == 0);
                         const unsigned ispre = __ballot_sync(0xFFFFFFFFu, flag == 2);
                         const unsigned window = ispre ? (((ispre & (0u - ispre)) << 1) - 1u) : 0xFFFFFFFFu;
@@ -732,8 +815,8 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                             continue;
                         }
                         const bool in = (window >> lane) & 1u;
-                        unsigned ve = in ? static_cast<unsigned>((s >> 31) & 0x7FFFFFFFu) : 0u;
-                        unsigned vo = in ? static_cast<unsigned>(s & 0x7FFFFFFFu) : 0u;
+                        unsigned ve = in ? static_cast<unsigned>((st >> 31) & 0x7FFFFFFFu) : 0u;
+                        unsigned vo = in ? static_cast<unsigned>(st & 0x7FFFFFFFu) : 0u;
 #pragma unroll
                         for (int off = 16; off > 0; off >>= 1) {
                             ve += __shfl_xor_sync(0xFFFFFFFFu, ve, off);
@@ -749,15 +832,28 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     if (lane == 0)
                         st_volatile_u64(&status[prev2.t],
                                         (2ull << 62) |
-                                            (static_cast<unsigned long long>((ex_e + prev2.ne) & 0x7FFFFFFFu) << 31) |
-                                            ((ex_o + prev2.no) & 0x7FFFFFFFu));
+                                            (static_cast<unsigned long long>((ex_e + s_tot[sl2][0]) & 0x7FFFFFFFu) << 31) |
+                                            ((ex_o + s_tot[sl2][1]) & 0x7FFFFFFFu));
                 }
                 if (lane == 0) {
-                    s_ex[msl2][0] = ex_e;
-                    s_ex[msl2][1] = ex_o;
+                    s_ex[sl2][0] = ex_e;
+                    s_ex[sl2][1] = ex_o;
                 }
             }
-            named_bar_sync(2, kFastThreads);
+            {  // row scales of tile i + 1 once its bytes are in
+                const FastTile nt = s_info[(i + 1) & 7];
+                if (nt.t < p.n_tiles) {
+                    int spins = 0;
+                    while (!mbar_try_wait(&s_full[(i + 1) & 1], ((i + 1) >> 1) & 1)) {
+                        if (++spins > kWaitLimit) {
+                            if (lane == 0) atomicOr(&p.ctr->err, 2ull);
+                            break;
+                        }
+                    }
+                    tile_scales(p, nt, inbuf + ((i + 1) & 1) * kFastTileElems, s_rows[(i + 1) & 1],
+                                s_rowc[(i + 1) & 1], s_rowm[(i + 1) & 1], lane);
+                }
+            }
             if (lane == 0) bulk_wait_read_all();
             __syncwarp();
         }

@@ -43,10 +43,7 @@ namespace e8q {
 // Core codeword k as 8 nibbles: nibble i (bits 4i..4i+3) = P_i + 8.
 __device__ __align__(16) uint32_t g_gv_tab[65536];
 
-constexpr int kGvThreads = 256;
-constexpr int kGvWarps = kGvThreads / 32;
-constexpr int kGvWarpRows = 32;    // rows per warp: two 16-row MMA tiles
-constexpr int kGvBlockRows = kGvWarps * kGvWarpRows;  // rows per row block (one CTA's rows)
+constexpr int kGvBlockRows = 256;  // rows per row block (one CTA's rows): 16-row MMA tiles over the warps
 constexpr int kGvChunkCols = 256;  // columns per chunk: 32 groups, 8 k-steps
 constexpr int kGvTabN = 49152;     // codeword words held in shared memory
 constexpr int kGvMaxCtas = 160;    // upper bound on main-kernel CTAs (workspace sizing)
@@ -154,11 +151,19 @@ __global__ void __launch_bounds__(256) k_gv_prep(const __grid_constant__ GvPrepP
         const uint16_t* xb = p.x + static_cast<size_t>(b) * C;
         // largest |x| of the row, as bf16 magnitude bits (integer order = value order)
         unsigned m = 0;
-        for (int i = threadIdx.x; i < C / 8; i += 256) {
-            const uint4 v = __ldg(reinterpret_cast<const uint4*>(xb) + i);
-            const unsigned w4[4] = {v.x, v.y, v.z, v.w};
+        for (int i0 = 0; i0 < C / 8; i0 += 8 * 256) {
+            uint4 v[8];  // all loads of a round before their use
 #pragma unroll
-            for (int k = 0; k < 4; ++k) m = max(m, max(w4[k] & 0x7FFFu, (w4[k] >> 16) & 0x7FFFu));
+            for (int k = 0; k < 8; ++k) {
+                const int i = i0 + threadIdx.x + 256 * k;
+                v[k] = i < C / 8 ? __ldg(reinterpret_cast<const uint4*>(xb) + i) : make_uint4(0, 0, 0, 0);
+            }
+#pragma unroll
+            for (int k = 0; k < 8; ++k) {
+                const unsigned w4[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+                for (int e = 0; e < 4; ++e) m = max(m, max(w4[e] & 0x7FFFu, (w4[e] >> 16) & 0x7FFFu));
+            }
         }
         m = __reduce_max_sync(0xFFFFFFFFu, m);
         if (lane == 0) s_red[warp] = m;
@@ -267,31 +272,36 @@ __device__ __forceinline__ uint4 gv_idx8(const uint16_t* rowp, int gs, int gpr, 
     return make_uint4(h[0] | (h[1] << 16), h[2] | (h[3] << 16), h[4] | (h[5] << 16), h[6] | (h[7] << 16));
 }
 
-// row (within the warp's 32) of codeword slot r (0..3): tile r>>1, +8 for odd r
+// Rows of codeword slot r (0 .. 2RT-1) inside the warp: tile r>>1, +8 for odd r.
 __device__ __forceinline__ int gv_row_in_warp(int r, int g) { return 16 * (r >> 1) + 8 * (r & 1) + g; }
 
+template <int RT>
 struct GvVisit {
-    uint4 idx[4];  // 8 indices per codeword row
-    uint2 map[4];  // 8 root-map bytes per codeword row
+    uint4 idx[2 * RT];  // 8 indices per codeword row
+    uint2 map[2 * RT];  // 8 root-map bytes per codeword row
 };
 
-__device__ __forceinline__ void gv_load_idx(const GvMainParams& p, int rb, int c, int warp, int g, int q, GvVisit& d) {
+template <int RT>
+__device__ __forceinline__ void gv_load_idx(const GvMainParams& p, int rb, int c, int warp, int g, int q,
+                                            GvVisit<RT>& d) {
     const GvGeom& G = p.g;
     const int gs = 32 * c + 8 * q;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int row = rb * kGvBlockRows + warp * kGvWarpRows + gv_row_in_warp(r, g);
+    for (int r = 0; r < 2 * RT; ++r) {
+        const int row = rb * kGvBlockRows + warp * 16 * RT + gv_row_in_warp(r, g);
         d.idx[r] = row < G.rows ? gv_idx8(p.idx + static_cast<size_t>(row) * G.gpr, gs, G.gpr, p.vec_idx != 0)
                                 : make_uint4(0, 0, 0, 0);
     }
 }
 
-__device__ __forceinline__ void gv_load_map(const GvMainParams& p, int rb, int c, int warp, int g, int q, GvVisit& d) {
+template <int RT>
+__device__ __forceinline__ void gv_load_map(const GvMainParams& p, int rb, int c, int warp, int g, int q,
+                                            GvVisit<RT>& d) {
     const GvGeom& G = p.g;
     const int gs = 32 * c + 8 * q;
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
-        const int row = rb * kGvBlockRows + warp * kGvWarpRows + gv_row_in_warp(r, g);
+    for (int r = 0; r < 2 * RT; ++r) {
+        const int row = rb * kGvBlockRows + warp * 16 * RT + gv_row_in_warp(r, g);
         d.map[r] = (row < G.rows && p.map)
                        ? __ldcg(reinterpret_cast<const uint2*>(p.map + static_cast<size_t>(row) * G.mstride + gs))
                        : make_uint2(0, 0);
@@ -303,18 +313,19 @@ __device__ __forceinline__ unsigned gv_comp(const uint4& v, int k) {
 }
 
 // Codeword word of codeword row r at k-step j (shared table, else L1).
-__device__ __forceinline__ unsigned gv_word(const GvVisit& cv, const uint32_t* s_tab, int r, int j) {
+template <int RT>
+__device__ __forceinline__ unsigned gv_word(const GvVisit<RT>& cv, const uint32_t* s_tab, int r, int j) {
     const unsigned comp = gv_comp(cv.idx[r], j >> 1);
     const unsigned id = (j & 1) ? (comp >> 16) : (comp & 0xFFFFu);
     return id < static_cast<unsigned>(kGvTabN) ? s_tab[id] : __ldg(g_gv_tab + id);
 }
 
-// Codeword pairs (P_2k, P_2k+1) in fp16 of the 4 codeword rows at k-step j.
-template <bool ESC>
-__device__ __forceinline__ void gv_decode(const GvVisit& cv, const unsigned (&wd)[4], const uint2* s_root, int j,
-                                          unsigned (&pr)[4][4]) {
+// Codeword pairs (P_2k, P_2k+1) in fp16 of the codeword rows at k-step j.
+template <int RT, bool ESC>
+__device__ __forceinline__ void gv_decode(const GvVisit<RT>& cv, const unsigned (&wd)[2 * RT], const uint2* s_root,
+                                          int j, unsigned (&pr)[2 * RT][4]) {
 #pragma unroll
-    for (int r = 0; r < 4; ++r) {
+    for (int r = 0; r < 2 * RT; ++r) {
         const unsigned w = wd[r];
         unsigned lo = w & 0x0F0F0F0Fu, hi = (w >> 4) & 0x0F0F0F0Fu, bias;
         if (ESC) {
@@ -333,12 +344,13 @@ __device__ __forceinline__ void gv_decode(const GvVisit& cv, const unsigned (&wd
     }
 }
 
-template <int NBP>
-__device__ __forceinline__ void gv_mma(float (&acc)[2][NBP][4], const unsigned (&pr)[4][4], const uint4 (&xb)[NBP]) {
+template <int RT, int NBP>
+__device__ __forceinline__ void gv_mma(float (&acc)[RT][NBP][4], const unsigned (&pr)[2 * RT][4],
+                                       const uint4 (&xb)[NBP]) {
 #pragma unroll
     for (int u = 0; u < NBP; ++u)
 #pragma unroll
-        for (int t = 0; t < 2; ++t) {
+        for (int t = 0; t < RT; ++t) {
             mma_f16(acc[t][u], pr[2 * t][0], pr[2 * t + 1][0], pr[2 * t][1], pr[2 * t + 1][1], xb[u].x, xb[u].y);
             mma_f16(acc[t][u], pr[2 * t][2], pr[2 * t + 1][2], pr[2 * t][3], pr[2 * t + 1][3], xb[u].z, xb[u].w);
         }
@@ -354,27 +366,27 @@ __device__ __forceinline__ void gv_load_x(const uint4* xs, const bool (&bok)[NBP
         xb[u] = (bok[u] && jok) ? __ldg(xs + static_cast<size_t>(u) * 256 + j * 32 + lane) : make_uint4(0, 0, 0, 0);
 }
 
-template <int NBP, bool ESC>
-__device__ __forceinline__ void gv_visit(float (&acc)[2][NBP][4], const GvVisit& cv, const uint32_t* s_tab,
+template <int RT, int NBP, bool ESC>
+__device__ __forceinline__ void gv_visit(float (&acc)[RT][NBP][4], const GvVisit<RT>& cv, const uint32_t* s_tab,
                                          const uint2* s_root, const uint4* xs, const bool (&bok)[NBP], int lim, int j0,
                                          int j1, int lane) {
-    if (NBP <= 2) {
+    if (RT * NBP <= 2) {
         // every codeword word and activation fragment of the chunk up front:
         // one exposed latency per chunk
-        unsigned wd[8][4];
+        unsigned wd[8][2 * RT];
         uint4 xa[8][NBP];
 #pragma unroll
         for (int j = 0; j < 8; ++j)
 #pragma unroll
-            for (int r = 0; r < 4; ++r) wd[j][r] = (j >= j0 && j < j1) ? gv_word(cv, s_tab, r, j) : 0u;
+            for (int r = 0; r < 2 * RT; ++r) wd[j][r] = (j >= j0 && j < j1) ? gv_word<RT>(cv, s_tab, r, j) : 0u;
 #pragma unroll
         for (int j = 0; j < 8; ++j) gv_load_x<NBP>(xs, bok, j < lim && j >= j0 && j < j1, j, lane, xa[j]);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
             if (j >= j0 && j < j1) {
-                unsigned pr[4][4];
-                gv_decode<ESC>(cv, wd[j], s_root, j, pr);
-                gv_mma<NBP>(acc, pr, xa[j]);
+                unsigned pr[2 * RT][4];
+                gv_decode<RT, ESC>(cv, wd[j], s_root, j, pr);
+                gv_mma<RT, NBP>(acc, pr, xa[j]);
             }
     } else if (NBP >= 8) {
         // no room for a second set of fragments: load at the k-step
@@ -382,19 +394,19 @@ __device__ __forceinline__ void gv_visit(float (&acc)[2][NBP][4], const GvVisit&
         for (int j = 0; j < 8; ++j)
             if (j >= j0 && j < j1) {
                 uint4 xb[NBP];
-                unsigned wd[4];
+                unsigned wd[2 * RT];
 #pragma unroll
-                for (int r = 0; r < 4; ++r) wd[r] = gv_word(cv, s_tab, r, j);
+                for (int r = 0; r < 2 * RT; ++r) wd[r] = gv_word<RT>(cv, s_tab, r, j);
                 gv_load_x<NBP>(xs, bok, j < lim, j, lane, xb);
-                unsigned pr[4][4];
-                gv_decode<ESC>(cv, wd, s_root, j, pr);
-                gv_mma<NBP>(acc, pr, xb);
+                unsigned pr[2 * RT][4];
+                gv_decode<RT, ESC>(cv, wd, s_root, j, pr);
+                gv_mma<RT, NBP>(acc, pr, xb);
             }
     } else {
         uint4 xb[NBP], xn[NBP];
-        unsigned wd[4], wn[4];
+        unsigned wd[2 * RT], wn[2 * RT];
 #pragma unroll
-        for (int r = 0; r < 4; ++r) wd[r] = gv_word(cv, s_tab, r, j0);
+        for (int r = 0; r < 2 * RT; ++r) wd[r] = gv_word<RT>(cv, s_tab, r, j0);
         gv_load_x<NBP>(xs, bok, j0 < lim, j0, lane, xb);
 #pragma unroll
         for (int j = 0; j < 8; ++j)
@@ -402,30 +414,30 @@ __device__ __forceinline__ void gv_visit(float (&acc)[2][NBP][4], const GvVisit&
                 if (j + 1 < j1) {
                     gv_load_x<NBP>(xs, bok, j + 1 < lim, j + 1, lane, xn);
 #pragma unroll
-                    for (int r = 0; r < 4; ++r) wn[r] = gv_word(cv, s_tab, r, j + 1);
+                    for (int r = 0; r < 2 * RT; ++r) wn[r] = gv_word<RT>(cv, s_tab, r, j + 1);
                 }
-                unsigned pr[4][4];
-                gv_decode<ESC>(cv, wd, s_root, j, pr);
-                gv_mma<NBP>(acc, pr, xb);
+                unsigned pr[2 * RT][4];
+                gv_decode<RT, ESC>(cv, wd, s_root, j, pr);
+                gv_mma<RT, NBP>(acc, pr, xb);
 #pragma unroll
                 for (int u = 0; u < NBP; ++u) xb[u] = xn[u];
 #pragma unroll
-                for (int r = 0; r < 4; ++r) wd[r] = wn[r];
+                for (int r = 0; r < 2 * RT; ++r) wd[r] = wn[r];
             }
     }
 }
 
-template <int NBP>
-__device__ __forceinline__ void gv_flush(const GvMainParams& p, float (&acc)[2][NBP][4], int rb, int warp, int g,
+template <int RT, int NBP>
+__device__ __forceinline__ void gv_flush(const GvMainParams& p, float (&acc)[RT][NBP][4], int rb, int warp, int g,
                                          int q) {
     const GvGeom& G = p.g;
     const long long ks = static_cast<long long>(G.nchunks) * 8;
     const long long slot = static_cast<long long>(blockIdx.x) - gv_cta_of(static_cast<long long>(rb) * ks, G.ksteps, G.nctas);
     if (slot >= 0 && slot < G.maxslots) {
-        float* base = p.part + ((static_cast<size_t>(rb) * G.maxslots + slot) * kGvBlockRows + warp * kGvWarpRows) *
+        float* base = p.part + ((static_cast<size_t>(rb) * G.maxslots + slot) * kGvBlockRows + warp * 16 * RT) *
                                    G.batch;
 #pragma unroll
-        for (int t = 0; t < 2; ++t)
+        for (int t = 0; t < RT; ++t)
 #pragma unroll
             for (int u = 0; u < NBP; ++u)
 #pragma unroll
@@ -436,7 +448,7 @@ __device__ __forceinline__ void gv_flush(const GvMainParams& p, float (&acc)[2][
                 }
     }
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
+    for (int t = 0; t < RT; ++t)
 #pragma unroll
         for (int u = 0; u < NBP; ++u)
 #pragma unroll
@@ -460,8 +472,10 @@ __device__ __forceinline__ uint2 gv_root_entry(int i) {
     return make_uint2(lo, hi);
 }
 
-template <int NBP>
-__global__ void __launch_bounds__(kGvThreads, 1) k_gv_main(const __grid_constant__ GvMainParams p) {
+// RT 16-row tiles per warp, 16 / RT warps per CTA (256 rows); NBP batch tiles of 8.
+template <int RT, int NBP>
+__global__ void __launch_bounds__(512 / RT, 1) k_gv_main(const __grid_constant__ GvMainParams p) {
+    constexpr int kThreads = 512 / RT;
     extern __shared__ __align__(16) unsigned char smem[];
     uint32_t* s_tab = reinterpret_cast<uint32_t*>(smem);
     uint2* s_root = reinterpret_cast<uint2*>(smem + kGvTabBytes);
@@ -473,23 +487,23 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gv_main(const __grid_constant
     int rb = static_cast<int>(vbeg / G.nchunks), c = static_cast<int>(vbeg % G.nchunks);
     pdl_launch_dependents();
     // prologue independent of the prep kernel: first indices, shared tables
-    GvVisit cur;
-    if (lo < hi) gv_load_idx(p, rb, c, warp, g, q, cur);
-    for (int i = threadIdx.x; i < kGvTabN / 4; i += kGvThreads)
+    GvVisit<RT> cur;
+    if (lo < hi) gv_load_idx<RT>(p, rb, c, warp, g, q, cur);
+    for (int i = threadIdx.x; i < kGvTabN / 4; i += kThreads)
         reinterpret_cast<uint4*>(s_tab)[i] = __ldg(reinterpret_cast<const uint4*>(g_gv_tab) + i);
-    for (int i = threadIdx.x; i < 256; i += kGvThreads) s_root[i] = gv_root_entry(i);
+    for (int i = threadIdx.x; i < 256; i += kThreads) s_root[i] = gv_root_entry(i);
     __syncthreads();
     pdl_wait();  // activations and root map written by the prep kernel
     if (lo >= hi) return;
-    gv_load_map(p, rb, c, warp, g, q, cur);
+    gv_load_map<RT>(p, rb, c, warp, g, q, cur);
 
     bool bok[NBP];
 #pragma unroll
     for (int u = 0; u < NBP; ++u) bok[u] = 8 * (p.v0 + u) + g < G.batch;
 
-    float acc[2][NBP][4];
+    float acc[RT][NBP][4];
 #pragma unroll
-    for (int t = 0; t < 2; ++t)
+    for (int t = 0; t < RT; ++t)
 #pragma unroll
         for (int u = 0; u < NBP; ++u)
 #pragma unroll
@@ -497,18 +511,18 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gv_main(const __grid_constant
 
     int cur_rb = rb;
     for (long long v = vbeg; v < vend; ++v) {
-        GvVisit nxt;
+        GvVisit<RT> nxt;
         int nrb = rb, nc = c + 1;
         if (nc == G.nchunks) {
             nc = 0;
             ++nrb;
         }
         if (v + 1 < vend) {
-            gv_load_idx(p, nrb, nc, warp, g, q, nxt);
-            gv_load_map(p, nrb, nc, warp, g, q, nxt);
+            gv_load_idx<RT>(p, nrb, nc, warp, g, q, nxt);
+            gv_load_map<RT>(p, nrb, nc, warp, g, q, nxt);
         }
         if (rb != cur_rb) {
-            gv_flush<NBP>(p, acc, cur_rb, warp, g, q);
+            gv_flush<RT, NBP>(p, acc, cur_rb, warp, g, q);
             cur_rb = rb;
         }
         const int j0 = v == vbeg ? static_cast<int>(lo & 7) : 0;
@@ -518,16 +532,16 @@ __global__ void __launch_bounds__(kGvThreads, 1) k_gv_main(const __grid_constant
         const uint4* xs = p.x16 + (static_cast<size_t>(c) * G.nbt + p.v0) * 256;
         unsigned any = 0;
 #pragma unroll
-        for (int r = 0; r < 4; ++r) any |= cur.map[r].x | cur.map[r].y;
+        for (int r = 0; r < 2 * RT; ++r) any |= cur.map[r].x | cur.map[r].y;
         if (__any_sync(0xFFFFFFFFu, any != 0))
-            gv_visit<NBP, true>(acc, cur, s_tab, s_root, xs, bok, lim, j0, j1, lane);
+            gv_visit<RT, NBP, true>(acc, cur, s_tab, s_root, xs, bok, lim, j0, j1, lane);
         else
-            gv_visit<NBP, false>(acc, cur, s_tab, s_root, xs, bok, lim, j0, j1, lane);
+            gv_visit<RT, NBP, false>(acc, cur, s_tab, s_root, xs, bok, lim, j0, j1, lane);
         cur = nxt;
         rb = nrb;
         c = nc;
     }
-    gv_flush<NBP>(p, acc, cur_rb, warp, g, q);
+    gv_flush<RT, NBP>(p, acc, cur_rb, warp, g, q);
 }
 
 // ---------------------------------------------------------------------------
@@ -608,7 +622,8 @@ __global__ void __launch_bounds__(256) k_gv_fin(const __grid_constant__ GvFinPar
                         float a = acc[k];
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
-                            const int v = (c & 1) ? (cw[i][c >> 1] >> 16) : static_cast<int>(static_cast<int16_t>(cw[i][c >> 1] & 0xFFFF));
+                            const int v = (c & 1) ? (cw[i][c >> 1] >> 16)
+                                                  : static_cast<int>(static_cast<int16_t>(cw[i][c >> 1] & 0xFFFF));
                             a = fmaf(static_cast<float>(v), __ldg(xc + static_cast<size_t>(c) * G.batch + b), a);
                         }
                         acc[k] = a;

@@ -361,79 +361,57 @@ __device__ __forceinline__ void best_escape_root_lean(const int (&P)[8], int (&R
 
 namespace e8q {
 
-// The escape choice of best_escape_root, returned as the core candidate
-// Q = P - R, the root's construction key (tables.h) and <P, R>.
-__device__ __forceinline__ int escape_search(const int (&P)[8], int (&Q)[8], int& key) {
-    int w[8];
-    unsigned pos = 0u, zer = 0u;
-    int a1 = 0, vH = 0;
+// The escape choice of best_escape_root without branches, returned as the
+// core candidate Q = P - R, the root's construction key (tables.h) and
+// <P, R>.  One key per
+// coordinate, k_i = (|P_i| << 5) | (P_i < 0 ? i : 23 - i), orders the
+// coordinates by magnitude and breaks ties the way the lexicographic rule
+// does: a non-negative coordinate earlier, a negative one later, is the
+// better place for a +-2 of the integer-type root.  Its two largest keys
+// are that root's positions; its smallest key is the coordinate whose sign
+// the half-type root flips when P has an odd number of negative
+// coordinates (the last zero coordinate if there is one, which costs
+// nothing).
+__device__ __forceinline__ int escape_search_keys(const int (&P)[8], int (&Q)[8], int& key) {
+    int k[8], sumw = 0;
+    unsigned negm = 0u;
 #pragma unroll
     for (int i = 0; i < 8; ++i) {
-        w[i] = abs(P[i]);
-        a1 = max(a1, w[i]);
-        vH += w[i];
-        pos |= (P[i] >= 0 ? 1u : 0u) << i;
-        zer |= (P[i] == 0 ? 1u : 0u) << i;
+        const bool neg = P[i] < 0;
+        const int w = abs(P[i]);
+        sumw += w;
+        negm |= (neg ? 1u : 0u) << i;
+        k[i] = (w << 5) | (neg ? i : 23 - i);
     }
-    const unsigned negm = ~pos & 0xFFu;
-    unsigned m1 = 0u, T = 0u;
-    int a2 = -1, wmin = w[0];
+    int m1 = k[0], mn = k[0];
 #pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        m1 |= (w[i] == a1 ? 1u : 0u) << i;
-        a2 = max(a2, w[i] == a1 ? -1 : w[i]);
-        wmin = min(wmin, w[i]);
+    for (int i = 1; i < 8; ++i) {
+        m1 = max(m1, k[i]);
+        mn = min(mn, k[i]);
     }
+    int m2 = 0;  // every key is >= 16 (non-negative coordinate) or >= 32 (negative one)
 #pragma unroll
-    for (int i = 0; i < 8; ++i) T |= (w[i] == wmin ? 1u : 0u) << i;
-    const bool single = __popc(m1) == 1;
-    unsigned pick;
-    if (single) {
-        unsigned m2 = 0u;
-#pragma unroll
-        for (int i = 0; i < 8; ++i) m2 |= (w[i] == a2 ? 1u : 0u) << i;
-        const unsigned mp = m2 & pos;
-        pick = m1 | (mp ? (mp & (0u - mp)) : (1u << (31 - __clz(m2))));
-    } else {
-        a2 = a1;
-        const unsigned jp = m1 & pos, jn = m1 & negm;
-        const int np = __popc(jp);
-        if (np >= 2) {
-            const unsigned f = jp & (0u - jp), r = jp & ~f;
-            pick = f | (r & (0u - r));
-        } else if (np == 1) {
-            pick = jp | (1u << (31 - __clz(jn)));
-        } else {
-            const unsigned l = 1u << (31 - __clz(jn));
-            pick = l | (1u << (31 - __clz(jn & ~l)));
-        }
-    }
-    const int vI = 2 * (a1 + a2);
-    unsigned hneg = negm;
-    if (__popc(negm) & 1) {
-        if (zer) {
-            hneg |= 1u << (31 - __clz(zer));
-        } else {
-            const unsigned tn = T & negm;
-            hneg ^= tn ? (tn & (0u - tn)) : (1u << (31 - __clz(T)));
-            vH -= 2 * wmin;
-        }
-    }
-    const int ri0 = (pick & 1u) ? ((pos & 1u) ? 2 : -2) : 0;
+    for (int i = 0; i < 8; ++i) m2 = max(m2, k[i] == m1 ? 0 : k[i]);
+    const int t1 = m1 & 31, t2 = m2 & 31, tn = mn & 31;
+    const int p1 = t1 >= 16 ? 23 - t1 : t1, p2 = t2 >= 16 ? 23 - t2 : t2, pf = tn >= 16 ? 23 - tn : tn;
+    const int vI = 2 * ((m1 >> 5) + (m2 >> 5));
+    const unsigned par = __popc(negm) & 1u;
+    const unsigned hneg = negm ^ (par << pf);
+    const int vH = sumw - (par ? 2 * (mn >> 5) : 0);
+    const int s1 = t1 >= 16 ? 2 : -2, s2 = t2 >= 16 ? 2 : -2;
+    const int ri0 = p1 == 0 ? s1 : (p2 == 0 ? s2 : 0);
     const int rh0 = (hneg & 1u) ? -1 : 1;
     const bool useI = (vI > vH) || (vI == vH && ri0 > rh0);
-    if (useI) {
-        const int i = __ffs(pick) - 1, j = 31 - __clz(pick);
-        const int ni = ((pos >> i) & 1u) ? 0 : 1, nj = ((pos >> j) & 1u) ? 0 : 1;
-        key = (i << 5) | (j << 2) | (ni << 1) | nj;
 #pragma unroll
-        for (int k = 0; k < 8; ++k) Q[k] = P[k] - (((pick >> k) & 1u) ? (((pos >> k) & 1u) ? 2 : -2) : 0);
-        return vI;
+    for (int i = 0; i < 8; ++i) {
+        const int ri = (i == p1 ? s1 : 0) + (i == p2 ? s2 : 0);
+        const int rh = ((hneg >> i) & 1u) ? -1 : 1;
+        Q[i] = P[i] - (useI ? ri : rh);
     }
-    key = 256 | static_cast<int>(hneg);
-#pragma unroll
-    for (int k = 0; k < 8; ++k) Q[k] = P[k] - (((hneg >> k) & 1u) ? -1 : 1);
-    return vH;
+    const int lo = min(p1, p2), hi = max(p1, p2);
+    const int nlo = (lo == p1 ? s1 : s2) < 0 ? 1 : 0, nhi = (hi == p1 ? s1 : s2) < 0 ? 1 : 0;
+    key = useI ? ((lo << 5) | (hi << 2) | (nlo << 1) | nhi) : (256 | static_cast<int>(hneg));
+    return useI ? vI : vH;
 }
 
 // core_rank with |Q|^2 supplied by the caller

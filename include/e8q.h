@@ -128,9 +128,9 @@ typedef struct e8q_encode_args {
     int32_t scale_in;          /* 0: compute s_r and write mats[].scale; 1: read s_r from
                                   mats[].scale (fixed reconstruction scales; a value that is
                                   not finite and > 0 reads as 0, giving x = 0) */
-    e8q_escape* esc;           /* out: escape records sorted by group, capacity esc_cap */
+    e8q_escape* esc;           /* out: escape records sorted by group, capacity esc_cap; 8-byte aligned */
     int64_t esc_cap;
-    e8q_overflow* ovf;         /* out: overflow records sorted by group, capacity ovf_cap */
+    e8q_overflow* ovf;         /* out: overflow records sorted by group, capacity ovf_cap; 4-byte aligned */
     int64_t ovf_cap;
     int64_t* esc_row_ptr;      /* out: [total_rows + 1] CSR offsets into esc, or NULL */
     int64_t* ovf_row_ptr;      /* out: [total_rows + 1] CSR offsets into ovf, or NULL */
