@@ -20,6 +20,12 @@ __device__ __align__(16) uint16_t g_t2[2 * 2401];
 __device__ __align__(16) uint2 g_core8[65536];  // 8 int8 doubled coordinates per core index
 __device__ __align__(16) uint2 g_root8[240];
 __device__ __align__(16) uint8_t g_rootkey[512];  // root index by construction key
+// Escape lookup over every E8 point with |P|^2 <= 88 (host tables.h): the
+// two-table extended rank and the encoding word of each extended point.
+constexpr int kExtPoints = 1113841;
+__device__ __align__(16) uint32_t g_t1e[2 * 10000 * 12];
+__device__ __align__(16) uint32_t g_t2e[2 * 10000];
+__device__ __align__(16) uint32_t g_res[kExtPoints];
 
 // Rows per tile: enough rows that a tile holds about 4K elements.
 __host__ __device__ inline int rows_per_tile(int cols) {

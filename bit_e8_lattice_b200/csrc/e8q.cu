@@ -42,6 +42,12 @@ e8q_status ensure_device(int* dev_out) {
         if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_core8, core.data(), core.size() * sizeof(uint2)));
         if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_root8, roots.data(), roots.size() * sizeof(uint2)));
         if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_rootkey, t->root_of_key.data(), 512));
+        if (st == E8Q_OK && (t->res.size() != static_cast<size_t>(kExtPoints) || t->t1e.size() != 2 * 10000 * 12 ||
+                             t->t2e.size() != 2 * 10000))
+            st = E8Q_ERR_UNSUPPORTED;
+        if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_t1e, t->t1e.data(), t->t1e.size() * 4));
+        if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_t2e, t->t2e.data(), t->t2e.size() * 4));
+        if (st == E8Q_OK) st = cuda_ok(cudaMemcpyToSymbol(g_res, t->res.data(), t->res.size() * 4));
         if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_encode<1>, cudaFuncAttributeMaxDynamicSharedMemorySize, kEncSmemBytes));
         if (st == E8Q_OK)
@@ -209,6 +215,19 @@ e8q_status e8q_core_table(int8_t* out_coord2) {
     const HostTables* t = host_tables();
     if (!t) return E8Q_ERR_UNSUPPORTED;
     std::memcpy(out_coord2, t->core.data(), t->core.size());
+    return E8Q_OK;
+}
+
+e8q_status e8q_escape_lookup(const int8_t* coord2, int64_t n, uint32_t* out) {
+    if (n < 0 || (n > 0 && (!coord2 || !out))) return E8Q_ERR_INVALID_ARG;
+    const HostTables* t = host_tables();
+    if (!t) return E8Q_ERR_UNSUPPORTED;
+    for (int64_t k = 0; k < n; ++k) {
+        int P[8];
+        for (int i = 0; i < 8; ++i) P[i] = coord2[8 * k + i];
+        const uint32_t r = ext_rank(*t, P);
+        out[k] = r == kExtNone ? (2u << 24) : t->res[r];
+    }
     return E8Q_OK;
 }
 

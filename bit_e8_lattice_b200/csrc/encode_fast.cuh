@@ -49,8 +49,7 @@ constexpr int kFsT2 = kFsT1 + kEncT1Bytes;
 constexpr int kFsMap = kFsT2 + kEncT2Bytes;                           // u32 [4][2048]
 constexpr int kFsIdx = kFsMap + kFastSlots * kFastTileGroups * 4;     // u16 [2][2048]
 constexpr int kFsChunk = kFsIdx + 2 * kFastTileGroups * 2;            // u32 [4][2][65]
-constexpr int kFsRootKey = kFsChunk + kFastSlots * 2 * 65 * 4 + 8;    // u8 [512]
-constexpr int kFastSmemBytes = kFsRootKey + 512;
+constexpr int kFastSmemBytes = kFsChunk + kFastSlots * 2 * 65 * 4 + 8;
 
 struct FastTile {
     int t;        // ticket (>= n_tiles: none)
@@ -224,20 +223,23 @@ __device__ __forceinline__ void load_window_raw(unsigned (&raw)[8][4], const uin
     }
 }
 
-// Escape search for queued groups (entry: group | P0, P1 | P2, ... P7 | flag),
-// N per lane: all entries are read before any result is stored, so the
-// independent searches overlap.
+// Encoding of queued groups outside the core (entry: group | P0, P1 | P2,
+// ... P7 | flag), N per lane, by table: the extended rank of P (every E8
+// point with |P|^2 <= 88, two-table decomposition with digits
+// (P_i + 9) >> 1) indexes the encoding word -- rank(P - R) | root << 16 |
+// 1 << 24 for an escape, 2 << 24 for an overflow record; points beyond the
+// table are overflow records.  All entries are read, then all table words
+// gathered, then the results stored.
 template <int N>
 __device__ __forceinline__ void resolve_entries(const uint32_t* q, const int (&slot)[N], const bool (&ok)[N],
-                                                const uint16_t* st1, const uint16_t* st2, const uint8_t* rootkey,
                                                 uint32_t* map, int16_t* ovf_scratch, unsigned long long& clamped) {
     uint32_t e[N][5];
 #pragma unroll
     for (int n = 0; n < N; ++n)
 #pragma unroll
         for (int k = 0; k < 5; ++k) e[n][k] = ok[n] ? q[5 * slot[n] + k] : 0u;
-    uint32_t out[N];
-    int rq[N];
+    uint32_t ia[N], ib[N];
+    bool inr[N];
 #pragma unroll
     for (int n = 0; n < N; ++n) {
         int P[8];
@@ -249,20 +251,37 @@ __device__ __forceinline__ void resolve_entries(const uint32_t* q, const int (&s
         P[5] = static_cast<int16_t>(e[n][3] & 0xFFFFu);
         P[6] = static_cast<int16_t>(e[n][3] >> 16);
         P[7] = static_cast<int16_t>(e[n][4] & 0xFFFFu);
-        int Q[8], key, n2 = 0;
+        int n2 = 0, hk = 0, lk = 0;
+        bool in = ok[n];
 #pragma unroll
-        for (int i = 0; i < 8; ++i) n2 += P[i] * P[i];
-        const int v = escape_search_keys(P, Q, key);
-        rq[n] = core_rank_n2(Q, n2 - 2 * v + 8, st1, st2);  // |P - R|^2 = |P|^2 - 2 <P, R> + |R|^2
-        out[n] = rq[n] >= 0 ? (static_cast<uint32_t>(rq[n]) | (static_cast<uint32_t>(rootkey[key]) << 16) | (1u << 24))
-                            : (2u << 24);
+        for (int i = 0; i < 8; ++i) {
+            n2 += P[i] * P[i];
+            in = in && static_cast<unsigned>(P[i] + 9) <= 18u;
+        }
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+            hk = hk * 10 + ((P[i] + 9) >> 1);
+            lk = lk * 10 + ((P[i + 4] + 9) >> 1);
+        }
+        in = in && n2 <= 88;
+        const int type = P[0] & 1;
+        inr[n] = in;
+        ia[n] = in ? __ldg(g_t1e + (type * 10000 + hk) * 12 + (n2 >> 3)) : 0u;
+        ib[n] = in ? __ldg(g_t2e + type * 10000 + lk) : 0u;
+    }
+    uint32_t out[N];
+#pragma unroll
+    for (int n = 0; n < N; ++n) {
+        const uint32_t r = ia[n] + ib[n];
+        const bool hit = inr[n] && ia[n] != 0xFFFFFFFFu && ib[n] != 0xFFFFFFFFu && r < static_cast<uint32_t>(kExtPoints);
+        out[n] = hit ? __ldg(g_res + r) : (2u << 24);
     }
 #pragma unroll
     for (int n = 0; n < N; ++n) {
         if (!ok[n]) continue;
         const int g = static_cast<int>(e[n][0] & 0xFFFFu);
         map[map_slot(g)] = out[n];
-        if (rq[n] < 0) {
+        if ((out[n] >> 24) == 2) {
             uint4 o;
             o.x = (e[n][0] >> 16) | (e[n][1] << 16);
             o.y = (e[n][1] >> 16) | (e[n][2] << 16);
@@ -368,7 +387,6 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
     uint32_t* smap = reinterpret_cast<uint32_t*>(smem + kFsMap);
     uint16_t* sidx = reinterpret_cast<uint16_t*>(smem + kFsIdx);
     uint32_t* schunk = reinterpret_cast<uint32_t*>(smem + kFsChunk);
-    uint8_t* srootkey = smem + kFsRootKey;
 
     __shared__ __align__(8) uint64_t s_full[2];
     __shared__ FastTile s_info[8];  // tile of iteration i at i & 7
@@ -387,7 +405,6 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
         for (int i = tid; i < (2 * 2401 * 7 * 2) / 16; i += kFastThreads) b[i] = a[i];
         for (int i = ((2 * 2401 * 7 * 2) / 16) * 8 + tid; i < 2 * 2401 * 7; i += kFastThreads) st1[i] = g_t1[i];
         for (int i = tid; i < 2 * 2401; i += kFastThreads) st2[i] = g_t2[i];
-        for (int i = tid; i < 512; i += kFastThreads) srootkey[i] = g_rootkey[i];
     }
     if (tid == 0) {
         mbar_init(&s_full[0], 1);
@@ -551,7 +568,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                             for (; qh < until; qh += 64) {
                                 const int sl[2] = {qh + lane, qh + 32 + lane};
                                 const bool okk[2] = {qh + lane < until, qh + 32 + lane < until};
-                                resolve_entries<2>(qbuf, sl, okk, st1, st2, srootkey, map, oscr, clamped);
+                                resolve_entries<2>(qbuf, sl, okk, map, oscr, clamped);
                             }
                             qh = until;
                             __syncwarp();

@@ -361,59 +361,6 @@ __device__ __forceinline__ void best_escape_root_lean(const int (&P)[8], int (&R
 
 namespace e8q {
 
-// The escape choice of best_escape_root without branches, returned as the
-// core candidate Q = P - R, the root's construction key (tables.h) and
-// <P, R>.  One key per
-// coordinate, k_i = (|P_i| << 5) | (P_i < 0 ? i : 23 - i), orders the
-// coordinates by magnitude and breaks ties the way the lexicographic rule
-// does: a non-negative coordinate earlier, a negative one later, is the
-// better place for a +-2 of the integer-type root.  Its two largest keys
-// are that root's positions; its smallest key is the coordinate whose sign
-// the half-type root flips when P has an odd number of negative
-// coordinates (the last zero coordinate if there is one, which costs
-// nothing).
-__device__ __forceinline__ int escape_search_keys(const int (&P)[8], int (&Q)[8], int& key) {
-    int k[8], sumw = 0;
-    unsigned negm = 0u;
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const bool neg = P[i] < 0;
-        const int w = abs(P[i]);
-        sumw += w;
-        negm |= (neg ? 1u : 0u) << i;
-        k[i] = (w << 5) | (neg ? i : 23 - i);
-    }
-    int m1 = k[0], mn = k[0];
-#pragma unroll
-    for (int i = 1; i < 8; ++i) {
-        m1 = max(m1, k[i]);
-        mn = min(mn, k[i]);
-    }
-    int m2 = 0;  // every key is >= 16 (non-negative coordinate) or >= 32 (negative one)
-#pragma unroll
-    for (int i = 0; i < 8; ++i) m2 = max(m2, k[i] == m1 ? 0 : k[i]);
-    const int t1 = m1 & 31, t2 = m2 & 31, tn = mn & 31;
-    const int p1 = t1 >= 16 ? 23 - t1 : t1, p2 = t2 >= 16 ? 23 - t2 : t2, pf = tn >= 16 ? 23 - tn : tn;
-    const int vI = 2 * ((m1 >> 5) + (m2 >> 5));
-    const unsigned par = __popc(negm) & 1u;
-    const unsigned hneg = negm ^ (par << pf);
-    const int vH = sumw - (par ? 2 * (mn >> 5) : 0);
-    const int s1 = t1 >= 16 ? 2 : -2, s2 = t2 >= 16 ? 2 : -2;
-    const int ri0 = p1 == 0 ? s1 : (p2 == 0 ? s2 : 0);
-    const int rh0 = (hneg & 1u) ? -1 : 1;
-    const bool useI = (vI > vH) || (vI == vH && ri0 > rh0);
-#pragma unroll
-    for (int i = 0; i < 8; ++i) {
-        const int ri = (i == p1 ? s1 : 0) + (i == p2 ? s2 : 0);
-        const int rh = ((hneg >> i) & 1u) ? -1 : 1;
-        Q[i] = P[i] - (useI ? ri : rh);
-    }
-    const int lo = min(p1, p2), hi = max(p1, p2);
-    const int nlo = (lo == p1 ? s1 : s2) < 0 ? 1 : 0, nhi = (hi == p1 ? s1 : s2) < 0 ? 1 : 0;
-    key = useI ? ((lo << 5) | (hi << 2) | (nlo << 1) | nhi) : (256 | static_cast<int>(hneg));
-    return useI ? vI : vH;
-}
-
 // core_rank with |Q|^2 supplied by the caller
 __device__ __forceinline__ int core_rank_n2(const int (&P)[8], int n2, const uint16_t* __restrict__ t1,
                                             const uint16_t* __restrict__ t2) {

@@ -69,6 +69,8 @@ def lib():
         L.e8q_init.restype = ctypes.c_int
         L.e8q_core_table.argtypes = [vp]
         L.e8q_core_table.restype = ctypes.c_int
+        L.e8q_escape_lookup.argtypes = [vp, i64, vp]
+        L.e8q_escape_lookup.restype = ctypes.c_int
         L.e8q_encode_workspace_bytes.argtypes = [ctypes.POINTER(Matrix), i32]
         L.e8q_encode_workspace_bytes.restype = sz
         L.e8q_project_encode.argtypes = [ctypes.POINTER(Matrix), i32, ctypes.POINTER(EncodeArgs), vp, sz, vp]
@@ -110,6 +112,16 @@ def core_table() -> np.ndarray:
     """The library's host-built core table (doubled coordinates), [65536][8]."""
     out = np.zeros((65536, 8), np.int8)
     _check(lib().e8q_core_table(out.ctypes.data_as(ctypes.c_void_p)), "e8q_core_table")
+    return out
+
+
+def escape_lookup(P: np.ndarray) -> np.ndarray:
+    """The encode kernels' encoding word of given doubled E8 points [n][8]
+    (host table; see e8q_escape_lookup in e8q.h)."""
+    P = np.ascontiguousarray(np.asarray(P).reshape(-1, 8).astype(np.int8))
+    out = np.zeros(P.shape[0], np.uint32)
+    _check(lib().e8q_escape_lookup(P.ctypes.data_as(ctypes.c_void_p), P.shape[0], out.ctypes.data_as(ctypes.c_void_p)),
+           "e8q_escape_lookup")
     return out
 
 

@@ -167,6 +167,17 @@ e8q_status e8q_init(void);
  * decoders (Table 3, "core decoding agreement"). */
 e8q_status e8q_core_table(int8_t* out_coord2);
 
+/* Host only: how the encode kernels encode given doubled E8 points
+ * (coord2: host [n][8], each a point of E8; out: host [n]).  A core point
+ * gives its core index; a point outside the core gives, by the escape rule
+ * (the root r maximising <p, r>, ties to the lexicographically largest r;
+ * E8-QAT appendix Table 3, single-root membership), rank(p - r) |
+ * (index of r << 16) | (1 << 24), or 2 << 24 (overflow record) when p - r
+ * is not in the core.  The kernels read the same table (every point with
+ * |p|^2 <= 22; farther points are always overflow records).  Lets a CPU test
+ * compare the table with other encoders. */
+e8q_status e8q_escape_lookup(const int8_t* coord2, int64_t n, uint32_t* out);
+
 /* Workspace bytes e8q_project_encode needs for these matrices (>= 16). */
 size_t e8q_encode_workspace_bytes(const e8q_matrix* mats /* host [n_mats] */, int32_t n_mats);
 

@@ -141,3 +141,26 @@ def test_decode_and_gemv_reject_bad_args(lib):
     assert lib.e8q_gemv_workspace_bytes(ctypes.byref(m), 257) == 256
     assert lib.e8q_dequant_gemv(ctypes.byref(m), ctypes.c_void_p(0x100000), 4, ctypes.c_void_p(0x100000),
                                 ctypes.c_void_p(0x100000), need - 1, None) == 4
+
+
+def test_escape_table_matches_oracle(lib):
+    """Every E8 point with |p|^2 <= 22 (1,113,841 points), plus a shell
+    beyond: the kernels' lookup table gives the oracle's encoding (core
+    index; escape core index and root; overflow).  E8-QAT appendix Table 3,
+    single-root membership."""
+    import lattice_np
+    import oracle
+    from bit_e8_lattice_b200 import e8q
+
+    P, n2 = lattice_np.e8_points(88)
+    assert len(P) == 1113841
+    far, _ = lattice_np.e8_points(96, 96)
+    P = np.concatenate([P, far[::7]], 0)
+    words = e8q.escape_lookup(P)
+    out = oracle.project_encode_vectors(P / 2.0)
+    kind, idx, root = out["kind"], out["idx"], out["root"]
+    assert (out["P"] == P).all()
+    expect = np.where(kind == 0, idx, np.where(kind == 1, idx | (root << 16) | (1 << 24), 2 << 24)).astype(np.uint32)
+    bad = np.nonzero(words != expect)[0]
+    assert len(bad) == 0, (len(bad), P[bad[:3]], words[bad[:3]], expect[bad[:3]])
+    assert (kind[-len(far[::7]):] == 2).all()
