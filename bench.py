@@ -21,6 +21,7 @@ from __future__ import annotations
 
 import argparse
 import hashlib
+import re
 import json
 import os
 import statistics
@@ -39,17 +40,21 @@ WORKLOAD = ("mlp_14336 QAT step: project+encode+STE-dequant of up 4096x14336 and
             "(one launch), identity-STE backward, then 2-bit dequant-GEMV of up at batch 1,4,16,64")
 D_MODEL, D_FF = 4096, 14336
 NOMINAL_HBM_GBS = 8000.0
-KERNEL_SOURCES = ["bit_e8_lattice_b200/csrc/" + f for f in
-                  ("e8q.cu", "encode.cuh", "lattice.cuh", "common.cuh", "gemv.cuh", "decode.cuh", "tables.cpp",
-                   "tables.h")]
+CSRC = os.path.join("bit_e8_lattice_b200", "csrc")
 
 
 def source_sha() -> str:
+    """Hash of the code of every kernel source file, comments and blank
+    space removed (a profile taken on other code does not describe the
+    current kernels)."""
     h = hashlib.sha256()
-    for f in KERNEL_SOURCES:
-        p = os.path.join(ROOT, f)
-        if os.path.exists(p):
-            h.update(open(p, "rb").read())
+    for f in sorted(os.listdir(os.path.join(ROOT, CSRC))):
+        if f.endswith((".cu", ".cuh", ".cpp", ".h")):
+            text = open(os.path.join(ROOT, CSRC, f), encoding="utf-8").read()
+            text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
+            text = re.sub(r"//[^\n]*", " ", text)
+            h.update(f.encode())
+            h.update(" ".join(text.split()).encode())
     return h.hexdigest()[:16]
 
 

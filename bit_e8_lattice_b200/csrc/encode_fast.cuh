@@ -3,20 +3,22 @@
 // of 256 and whose RHT block is 256..2048 ("E8-QAT", Figure 2 (a)-(c)).
 //
 // CTA = 8 compute warps + 1 service warp, persistent over row tiles of up
-// to 16K elements taken from an atomic ticket.
-//   service warp: claims the next tile and prefetches it with a 1-D bulk
-//     copy (TMA engine) into the other shared-memory buffer; publishes the
-//     finished tile's record counts; stores its 16-bit indices with a bulk
-//     copy; resolves, one tile later still, the tile's place among all
-//     earlier tiles' records (decoupled look-back, bounded waits).
-//   compute warps: one 2048-element window each.  Hadamard in registers:
-//     bits {0,1,3,4} of the element index by one bf16 m16n8k16 tensor-core
-//     MMA against H_16 straight from the (sign-flipped) bf16 input, bit 2
-//     and bits 8..10 as fp32 butterflies, then an in-warp transpose through
-//     shared memory and bits 5..7.  Row scales from per-window sums of
-//     squares; projection, core rank and escape search in registers; groups
-//     outside the core go to a per-warp queue so the root search runs with
-//     all lanes busy.  Records are emitted in group order two tiles later.
+// to 16K elements taken from an atomic ticket; one barrier per iteration.
+//   service warp, iteration i: claims tile i+1 and prefetches it with a
+//     1-D bulk copy (TMA engine) into the other shared-memory buffer; forms
+//     the chunk prefix of tile i-1's record counts, publishes them and
+//     stores its 16-bit indices with a bulk copy; places tile i-2 among all
+//     earlier tiles' records (decoupled look-back, bounded waits); computes
+//     tile i+1's row scales from its input (the RHT is orthonormal).
+//   compute warps: one 2048-element window each of tile i.  Hadamard in
+//     registers: bits {0,1,3,4} of the element index by one bf16 m16n8k16
+//     tensor-core MMA against H_16 straight from the (sign-flipped) bf16
+//     input, bit 2 and bits 8..10 as fp32 butterflies, then an in-warp
+//     transpose through shared memory and bits 5..7.  Projection and core
+//     rank in registers; groups outside the core go to a per-warp queue,
+//     drained with all lanes busy through the escape lookup table.  Each
+//     warp counts and indexes its own window and emits its own chunks of
+//     tile i-3's records.
 // Record order, CSR and results are the same as the generic kernel's.
 #pragma once
 #include "common.cuh"

@@ -20,8 +20,10 @@
 //             rows), fp32 accumulate.  The work -- 256-row blocks times
 //             256-column chunks times 8 k-steps -- is split into equal
 //             contiguous k-step ranges, one per CTA (one resident CTA per
-//             SM); the 8 warps of a CTA take 32 rows each of the same range,
-//             so they read the same activation fragments (L1 hits).  The first
+//             SM); the warps of a CTA (16 with one 16-row tile each for up
+//             to 16 batch rows, else 8 with two) take different rows of the
+//             same range, so they read the same activation fragments (L1
+//             hits).  The first
 //             49,152 codeword words live in shared memory (a shared-memory
 //             gather costs a few wavefronts per warp, a global one up to one
 //             per lane); the rest are read through L1.  Indices and root-map
@@ -57,7 +59,7 @@ struct GvGeom {
     int32_t rows, cols, gpr, batch;
     int32_t nbt;       // batch tiles of 8
     int32_t nchunks;   // 256-column chunks (last one may be partial)
-    int32_t nrb;       // 32-row blocks
+    int32_t nrb;       // 256-row blocks
     int32_t nctas;     // main-kernel CTAs with work
     int32_t maxslots;  // partial slots per row block
     int32_t mstride;   // root-map bytes per row (32 * nchunks)
