@@ -2,8 +2,9 @@
 // records (+ dequantised output) for bf16 weights whose width is a multiple
 // of 256 and whose RHT block is 256..2048 ("E8-QAT", Figure 2 (a)-(c)).
 //
-// CTA = 8 compute warps + 1 service warp, persistent over row tiles of up
-// to 16K elements taken from an atomic ticket; one barrier per iteration.
+// CTA = 14 compute warps + 1 service warp (128 registers a thread), persistent
+// over row tiles of up to 28,672 elements (two 14336-wide rows, seven
+// 4096-wide rows) taken from an atomic ticket; one barrier per iteration.
 //   service warp, iteration i: claims tile i+1 and prefetches it with a
 //     1-D bulk copy (TMA engine) into the other shared-memory buffer; forms
 //     the chunk prefix of tile i-1's record counts, publishes them and
@@ -15,7 +16,8 @@
 //     tensor-core MMA against H_16 straight from the (sign-flipped) bf16
 //     input, bit 2 and bits 8..10 as fp32 butterflies, then an in-warp
 //     transpose through shared memory and bits 5..7.  Projection and core
-//     rank in registers; groups outside the core go to a per-warp queue,
+//     rank in registers (rank table T1 read through L1, T2 in shared
+//     memory); groups outside the core go to a per-warp queue,
 //     drained with all lanes busy through the escape lookup table.  Each
 //     warp counts and indexes its own window and emits its own chunks of
 //     tile i-3's records.
@@ -28,10 +30,12 @@
 
 namespace e8q {
 
-constexpr int kFastWarps = 8;
+constexpr int kFastWarps = 14;
 constexpr int kFastThreads = (kFastWarps + 1) * 32;  // compute warps, service warp
-constexpr int kFastTileElems = 16384;
+constexpr int kFastTileElems = kFastWarps * 2048;    // 28672: two 14336-wide rows, seven 4096-wide rows
 constexpr int kFastTileGroups = kFastTileElems / 8;
+constexpr int kFastChunks = kFastTileGroups / 32;    // 32-group chunks per tile
+constexpr int kFastCnt = kFastChunks + 1;            // per record kind: chunk counts (then prefixes), total
 constexpr int kFastMaxCtas = 160;
 constexpr int kWaitLimit = 1 << 24;
 
@@ -46,12 +50,10 @@ constexpr int kFastSlots = 4;
 
 // shared-memory layout (bytes)
 constexpr int kFsIn = 0;                                              // bf16 [2][16384]
-constexpr int kFsT1 = kFsIn + 2 * kFastTileElems * 2;                 // 65536
-constexpr int kFsT2 = kFsT1 + kEncT1Bytes;
+constexpr int kFsT2 = kFsIn + 2 * kFastTileElems * 2;                 // T1 (67 KB) is read through L1
 constexpr int kFsMap = kFsT2 + kEncT2Bytes;                           // u32 [4][2048]
-constexpr int kFsIdx = kFsMap + kFastSlots * kFastTileGroups * 4;     // u16 [2][2048]
-constexpr int kFsChunk = kFsIdx + 2 * kFastTileGroups * 2;            // u32 [4][2][65]
-constexpr int kFastSmemBytes = kFsChunk + kFastSlots * 2 * 65 * 4 + 8;
+constexpr int kFsChunk = kFsMap + kFastSlots * kFastTileGroups * 4;   // u32 [4][2][kFastCnt]
+constexpr int kFastSmemBytes = kFsChunk + kFastSlots * 2 * kFastCnt * 4 + 8;
 
 struct FastTile {
     int t;        // ticket (>= n_tiles: none)
@@ -384,10 +386,8 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                                                                   int16_t* __restrict__ ovf_scratch_all) {
     extern __shared__ __align__(16) unsigned char smem[];
     uint16_t* inbuf = reinterpret_cast<uint16_t*>(smem + kFsIn);
-    uint16_t* st1 = reinterpret_cast<uint16_t*>(smem + kFsT1);
     uint16_t* st2 = reinterpret_cast<uint16_t*>(smem + kFsT2);
     uint32_t* smap = reinterpret_cast<uint32_t*>(smem + kFsMap);
-    uint16_t* sidx = reinterpret_cast<uint16_t*>(smem + kFsIdx);
     uint32_t* schunk = reinterpret_cast<uint32_t*>(smem + kFsChunk);
 
     __shared__ __align__(8) uint64_t s_full[2];
@@ -401,13 +401,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
     int16_t* ovf_scratch = ovf_scratch_all + static_cast<size_t>(blockIdx.x) * kFastSlots * kFastTileGroups * 8;
     unsigned long long* status = p.ws + 2;
 
-    {  // constant tables
-        const uint4* a = reinterpret_cast<const uint4*>(g_t1);
-        uint4* b = reinterpret_cast<uint4*>(st1);
-        for (int i = tid; i < (2 * 2401 * 7 * 2) / 16; i += kFastThreads) b[i] = a[i];
-        for (int i = ((2 * 2401 * 7 * 2) / 16) * 8 + tid; i < 2 * 2401 * 7; i += kFastThreads) st1[i] = g_t1[i];
-        for (int i = tid; i < 2 * 2401; i += kFastThreads) st2[i] = g_t2[i];
-    }
+    for (int i = tid; i < 2 * 2401; i += kFastThreads) st2[i] = g_t2[i];  // rank table T2
     if (tid == 0) {
         mbar_init(&s_full[0], 1);
         mbar_init(&s_full[1], 1);
@@ -495,7 +489,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                 }
                 // projection + encoding of the warp's 8 x 32 groups
                 uint32_t* map = smap + sl * kFastTileGroups;
-                uint16_t* idxs = sidx + b * kFastTileGroups;
+                uint16_t* idxs = M.idx + static_cast<size_t>(cur.r0) * gpr;
                 int16_t* oscr = ovf_scratch + static_cast<size_t>(sl) * kFastTileGroups * 8;
                 if (w < nwin) {
                     const int a = lane >> 2, q = lane & 3;
@@ -534,7 +528,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     }
                     int rks[8];
 #pragma unroll
-                    for (int h = 0; h < 8; ++h) rks[h] = lane_ok ? core_rank_f(v[h], (oddm >> h) & 1u, st1, st2) : 0;
+                    for (int h = 0; h < 8; ++h) rks[h] = lane_ok ? core_rank_f(v[h], (oddm >> h) & 1u, g_t1, st2) : 0;
 #pragma unroll
                     for (int h = 0; h < 8; ++h) {
                         const int gt = 256 * w + 32 * a + 4 * h + q;
@@ -681,7 +675,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                 }
                 if (w < nwin) {
                     // the window's record counts per 32-group chunk, and its indices
-                    uint32_t* cnt = schunk + sl * 130;
+                    uint32_t* cnt = schunk + sl * 2 * kFastCnt;
                     __syncwarp();
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
@@ -694,7 +688,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         const unsigned be = __ballot_sync(0xFFFFFFFFu, kind == 1), bo = __ballot_sync(0xFFFFFFFFu, kind == 2);
                         if (lane == 0) {
                             cnt[c] = __popc(be);
-                            cnt[65 + c] = __popc(bo);
+                            cnt[kFastCnt + c] = __popc(bo);
                         }
                     }
                 }
@@ -706,7 +700,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                 const MatDesc& M = p.m[prev3.mat];
                 const int gpr = M.cols >> 3, G = prev3.nr * gpr, nch = (G + 31) >> 5;
                 const uint32_t* map = smap + sl3 * kFastTileGroups;
-                const uint32_t* cnt = schunk + sl3 * 130;
+                const uint32_t* cnt = schunk + sl3 * 2 * kFastCnt;
                 const int16_t* oscr = ovf_scratch + static_cast<size_t>(sl3) * kFastTileGroups * 8;
                 const long long ex_e = s_ex[sl3][0], ex_o = s_ex[sl3][1];
                 const uint32_t gid0 = M.group_base + static_cast<uint32_t>(prev3.r0) * gpr;
@@ -739,7 +733,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                                 *reinterpret_cast<uint2*>(p.esc + pos) = r;
                             }
                         } else if (kind == 2) {
-                            const long long pos = ex_o + cnt[65 + c] + __popc(bo & lanemask_lt());
+                            const long long pos = ex_o + cnt[kFastCnt + c] + __popc(bo & lanemask_lt());
                             if (pos < p.ovf_cap) {
                                 uint32_t* dst = reinterpret_cast<uint32_t*>(p.ovf + pos);
                                 dst[0] = gid0 + g;
@@ -751,10 +745,10 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                 for (int r = tid; r < prev3.nr; r += kFastWarps * 32) {
                     const int c = (r * gpr) >> 5;  // rows start on chunk boundaries (gpr % 32 == 0)
                     if (p.esc_rp) p.esc_rp[M.row_base + prev3.r0 + r] = ex_e + cnt[c];
-                    if (p.ovf_rp) p.ovf_rp[M.row_base + prev3.r0 + r] = ex_o + cnt[65 + c];
+                    if (p.ovf_rp) p.ovf_rp[M.row_base + prev3.r0 + r] = ex_o + cnt[kFastCnt + c];
                 }
                 if (prev3.t == p.n_tiles - 1 && tid == 0) {
-                    const long long te = ex_e + cnt[64], to = ex_o + cnt[65 + 64];
+                    const long long te = ex_e + cnt[kFastChunks], to = ex_o + cnt[kFastCnt + kFastChunks];
                     if (p.esc_rp) p.esc_rp[p.total_rows] = te;
                     if (p.ovf_rp) p.ovf_rp[p.total_rows] = to;
                     p.ctr->n_escape = te;
@@ -780,36 +774,36 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                 }
             }
             __syncwarp();
-            if (p1_ok) {  // tile i - 1: chunk prefix (group order), publish its counts, store its indices
+            if (p1_ok) {  // tile i - 1: chunk prefix (group order), publish its counts
                 const MatDesc& M = p.m[prev1.mat];
                 const int gpr = M.cols >> 3, nch = (prev1.nr * gpr + 31) >> 5;
-                uint32_t* cnt = schunk + sl1 * 130;
-                const unsigned ce0 = lane < nch ? cnt[lane] : 0u, ce1 = lane + 32 < nch ? cnt[lane + 32] : 0u;
-                const unsigned co0 = lane < nch ? cnt[65 + lane] : 0u, co1 = lane + 32 < nch ? cnt[65 + lane + 32] : 0u;
-                unsigned se0 = ce0, se1 = ce1, so0 = co0, so1 = co1;  // inclusive scans
+                uint32_t* cnt = schunk + sl1 * 2 * kFastCnt;
+                constexpr int kPer = (kFastChunks + 31) / 32;  // chunks per lane: lane + 32 k
+                unsigned ne = 0, no = 0;  // running totals of the earlier rounds
 #pragma unroll
-                for (int off = 1; off < 32; off <<= 1) {
-                    const unsigned a0 = __shfl_up_sync(0xFFFFFFFFu, se0, off), a1 = __shfl_up_sync(0xFFFFFFFFu, se1, off);
-                    const unsigned b0 = __shfl_up_sync(0xFFFFFFFFu, so0, off), b1 = __shfl_up_sync(0xFFFFFFFFu, so1, off);
-                    if (lane >= off) { se0 += a0; se1 += a1; so0 += b0; so1 += b1; }
+                for (int k = 0; k < kPer; ++k) {
+                    const int c = lane + 32 * k;
+                    const unsigned ce = c < nch ? cnt[c] : 0u, co = c < nch ? cnt[kFastCnt + c] : 0u;
+                    unsigned se = ce, so = co;  // inclusive scans
+#pragma unroll
+                    for (int off = 1; off < 32; off <<= 1) {
+                        const unsigned a0 = __shfl_up_sync(0xFFFFFFFFu, se, off), b0 = __shfl_up_sync(0xFFFFFFFFu, so, off);
+                        if (lane >= off) { se += a0; so += b0; }
+                    }
+                    if (c < kFastChunks) {
+                        cnt[c] = ne + se - ce;
+                        cnt[kFastCnt + c] = no + so - co;
+                    }
+                    ne += __shfl_sync(0xFFFFFFFFu, se, 31);
+                    no += __shfl_sync(0xFFFFFFFFu, so, 31);
                 }
-                const unsigned te0 = __shfl_sync(0xFFFFFFFFu, se0, 31), to0 = __shfl_sync(0xFFFFFFFFu, so0, 31);
-                const unsigned te1 = __shfl_sync(0xFFFFFFFFu, se1, 31), to1 = __shfl_sync(0xFFFFFFFFu, so1, 31);
-                cnt[lane] = se0 - ce0;
-                cnt[lane + 32] = te0 + se1 - ce1;
-                cnt[65 + lane] = so0 - co0;
-                cnt[65 + lane + 32] = to0 + so1 - co1;
                 if (lane == 0) {
-                    const unsigned ne = te0 + te1, no = to0 + to1;
-                    cnt[64] = ne;
-                    cnt[65 + 64] = no;
+                    cnt[kFastChunks] = ne;
+                    cnt[kFastCnt + kFastChunks] = no;
                     s_tot[sl1][0] = ne;
                     s_tot[sl1][1] = no;
                     const unsigned long long own = (static_cast<unsigned long long>(ne) << 31) | no;
                     st_volatile_u64(&status[prev1.t], (prev1.t == 0 ? (2ull << 62) : (1ull << 62)) | own);
-                    bulk_store(M.idx + static_cast<size_t>(prev1.r0) * gpr, sidx + ((i + 1) & 1) * kFastTileGroups,
-                               static_cast<unsigned>(prev1.nr) * gpr * 2u);
-                    bulk_commit();
                 }
             }
             __syncwarp();
@@ -873,12 +867,10 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                                 s_rowc[(i + 1) & 1], s_rowm[(i + 1) & 1], lane);
                 }
             }
-            if (lane == 0) bulk_wait_read_all();
             __syncwarp();
         }
         __syncthreads();
     }
-    if (service && lane == 0) bulk_wait_all();
 
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {

@@ -114,16 +114,18 @@ def test_encode_rejects_bad_args(lib):
 def test_workspace_bytes_counts_tiles(lib):
     from bit_e8_lattice_b200 import e8q
 
-    # 37 rows of 256 columns: 16 rows per 4K-element tile -> 3 tiles; plus
-    # 3 one-row tiles; the status words need 16 + 8 * 6 bytes, and the
-    # 16K-element path adds a per-CTA scratch of 3 x 2048 x 16 bytes
+    # 37 rows of 256 columns: one tile of the bf16 path (up to 64 rows of
+    # 28,672 elements); 3 rows of 14336: 2 rows per tile -> 2 tiles; the
+    # status words need 16 + 8 * 3 bytes, and the bf16 path adds a per-CTA
+    # scratch of 4 x 3584 x 16 bytes
     mats = (e8q.Matrix * 2)(_mat(rows=37, cols=256), _mat(rows=3, cols=14336))
     n = lib.e8q_encode_workspace_bytes(mats, 2)
-    assert n % 256 == 0 and n >= 16 + 8 * 6
-    assert n <= 256 + 6 * 4 * 2048 * 16
+    assert n % 256 == 0 and n >= 16 + 8 * 3
+    assert n <= 256 + 3 * 4 * 3584 * 16
     mats = (e8q.Matrix * 1)(_mat(rows=4096, cols=14336))
     n = lib.e8q_encode_workspace_bytes(mats, 1)
-    assert n >= 16 + 8 * 4096 and n <= (16 + 8 * 4096 + 255) // 256 * 256 + 160 * 4 * 2048 * 16
+    # status words for the general kernel's 4096 one-row tiles (either path may run)
+    assert n >= 16 + 8 * 4096 and n <= (16 + 8 * 4096 + 255) // 256 * 256 + 160 * 4 * 3584 * 16
 
 
 def test_decode_and_gemv_reject_bad_args(lib):
