@@ -358,6 +358,26 @@ def main():
                                          "frac_measured_hbm": gbs / peaks["hbm_gbs"],
                                          "frac_nominal_8TBs": gbs / NOMINAL_HBM_GBS, "bytes_per_launch": gb_bytes}
 
+    # decode of the encoded up matrix (not part of the QAT step, timed on its
+    # own): indices, records, scales and row pointers in, bf16 weights out
+    dq_out = torch.empty((D_MODEL, D_FF), dtype=torch.bfloat16, device=dev)
+    dec_bytes = 2 * up_groups + 8 * up_esc + 20 * up_ovf + 4 * D_MODEL + 16 * (D_MODEL + 1) + 16 * up_groups
+    for basis in ("rotated", "original"):
+        for _ in range(3):
+            e8q.e8q_decode(res.encoded[0], basis, dq_out)
+        torch.cuda.synchronize()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        n_dec = 20
+        e0.record()
+        for _ in range(n_dec):
+            e8q.e8q_decode(res.encoded[0], basis, dq_out)
+        e1.record()
+        torch.cuda.synchronize()
+        avg = e0.elapsed_time(e1) / n_dec
+        gbs = dec_bytes / (avg * 1e-3) / 1e9
+        kernels[f"decode_{basis}"] = {"launch_us": 1e3 * avg, "GB_s": gbs, "frac_measured_hbm": gbs / peaks["hbm_gbs"],
+                                      "frac_nominal_8TBs": gbs / NOMINAL_HBM_GBS, "bytes_per_launch": dec_bytes}
+
     # end to end through the public API: pinned host inputs in, results out
     e2e = None
     if args.e2e_steps > 0:

@@ -17,8 +17,8 @@
 //     input, bit 2 and bits 8..10 as fp32 butterflies, then an in-warp
 //     transpose through shared memory and bits 5..7.  Projection and core
 //     rank in registers (rank table T1 read through L1, T2 in shared
-//     memory); groups outside the core go to a per-warp queue,
-//     drained with all lanes busy through the escape lookup table.  Each
+//     memory); a group outside the core takes its encoding from the escape
+//     lookup table (the lane's 8 groups' gathers issued together).  Each
 //     warp counts and indexes its own window and emits its own chunks of
 //     tile i-3's records.
 // Record order, CSR and results are the same as the generic kernel's.
@@ -227,76 +227,6 @@ __device__ __forceinline__ void load_window_raw(unsigned (&raw)[8][4], const uin
     }
 }
 
-// Encoding of queued groups outside the core (entry: group | P0, P1 | P2,
-// ... P7 | flag), N per lane, by table: the extended rank of P (every E8
-// point with |P|^2 <= 88, two-table decomposition with digits
-// (P_i + 9) >> 1) indexes the encoding word -- rank(P - R) | root << 16 |
-// 1 << 24 for an escape, 2 << 24 for an overflow record; points beyond the
-// table are overflow records.  All entries are read, then all table words
-// gathered, then the results stored.
-template <int N>
-__device__ __forceinline__ void resolve_entries(const uint32_t* q, const int (&slot)[N], const bool (&ok)[N],
-                                                uint32_t* map, int16_t* ovf_scratch, unsigned long long& clamped) {
-    uint32_t e[N][5];
-#pragma unroll
-    for (int n = 0; n < N; ++n)
-#pragma unroll
-        for (int k = 0; k < 5; ++k) e[n][k] = ok[n] ? q[5 * slot[n] + k] : 0u;
-    uint32_t ia[N], ib[N];
-    bool inr[N];
-#pragma unroll
-    for (int n = 0; n < N; ++n) {
-        int P[8];
-        P[0] = static_cast<int16_t>(e[n][0] >> 16);
-        P[1] = static_cast<int16_t>(e[n][1] & 0xFFFFu);
-        P[2] = static_cast<int16_t>(e[n][1] >> 16);
-        P[3] = static_cast<int16_t>(e[n][2] & 0xFFFFu);
-        P[4] = static_cast<int16_t>(e[n][2] >> 16);
-        P[5] = static_cast<int16_t>(e[n][3] & 0xFFFFu);
-        P[6] = static_cast<int16_t>(e[n][3] >> 16);
-        P[7] = static_cast<int16_t>(e[n][4] & 0xFFFFu);
-        int n2 = 0, hk = 0, lk = 0;
-        bool in = ok[n];
-#pragma unroll
-        for (int i = 0; i < 8; ++i) {
-            n2 += P[i] * P[i];
-            in = in && static_cast<unsigned>(P[i] + 9) <= 18u;
-        }
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {
-            hk = hk * 10 + ((P[i] + 9) >> 1);
-            lk = lk * 10 + ((P[i + 4] + 9) >> 1);
-        }
-        in = in && n2 <= 88;
-        const int type = P[0] & 1;
-        inr[n] = in;
-        ia[n] = in ? __ldg(g_t1e + (type * 10000 + hk) * 12 + (n2 >> 3)) : 0u;
-        ib[n] = in ? __ldg(g_t2e + type * 10000 + lk) : 0u;
-    }
-    uint32_t out[N];
-#pragma unroll
-    for (int n = 0; n < N; ++n) {
-        const uint32_t r = ia[n] + ib[n];
-        const bool hit = inr[n] && ia[n] != 0xFFFFFFFFu && ib[n] != 0xFFFFFFFFu && r < static_cast<uint32_t>(kExtPoints);
-        out[n] = hit ? __ldg(g_res + r) : (2u << 24);
-    }
-#pragma unroll
-    for (int n = 0; n < N; ++n) {
-        if (!ok[n]) continue;
-        const int g = static_cast<int>(e[n][0] & 0xFFFFu);
-        map[map_slot(g)] = out[n];
-        if ((out[n] >> 24) == 2) {
-            uint4 o;
-            o.x = (e[n][0] >> 16) | (e[n][1] << 16);
-            o.y = (e[n][1] >> 16) | (e[n][2] << 16);
-            o.z = (e[n][2] >> 16) | (e[n][3] << 16);
-            o.w = (e[n][3] >> 16) | (e[n][4] << 16);
-            *reinterpret_cast<uint4*>(ovf_scratch + 8 * g) = o;
-            if (e[n][4] & 0x10000u) ++clamped;
-        }
-    }
-}
-
 template <int MAXM>
 __device__ __forceinline__ FastTile make_tile(const EncodeParams<MAXM>& p, int t) {
     FastTile ft;
@@ -499,10 +429,6 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     // advances at most once (at hcut) when the width is not a multiple of 2048
                     const int e0 = 8 * (256 * w + 32 * a + q);
                     const int r0l = e0 / C, hcut = (C - e0 % C + 31) >> 5;
-                    // escape queue in the window's shared-memory region (free until the
-                    // original-basis dequant): 5 words per entry, at most 159 live entries
-                    uint32_t* qbuf = reinterpret_cast<uint32_t*>(win);
-                    int qn = 0;
                     // the lane's 8 groups are independent: project all of them, then
                     // rank all of them, then queue, so that the chains overlap
                     unsigned oddm = 0u;
@@ -529,60 +455,69 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     int rks[8];
 #pragma unroll
                     for (int h = 0; h < 8; ++h) rks[h] = lane_ok ? core_rank_f(v[h], (oddm >> h) & 1u, g_t1, st2) : 0;
+                    // groups outside the core: extended rank straight from the coordinates
+                    // (digits (P + 9) >> 1 = P / 2 + 4 or + 4.5, keys base 10, exact in fp32),
+                    // the two table gathers of all 8 groups, then their encoding words
+                    uint32_t ia[8], ib[8];
+                    unsigned pendm = 0u;
 #pragma unroll
                     for (int h = 0; h < 8; ++h) {
+                        const float (&P)[8] = v[h];
+                        const bool pend = lane_ok && rks[h] < 0;
+                        pendm |= (pend ? 1u : 0u) << h;
+                        float2 n = __fmul2_rn(make_float2(P[0], P[4]), make_float2(P[0], P[4]));
+                        n = __ffma2_rn(make_float2(P[1], P[5]), make_float2(P[1], P[5]), n);
+                        n = __ffma2_rn(make_float2(P[2], P[6]), make_float2(P[2], P[6]), n);
+                        n = __ffma2_rn(make_float2(P[3], P[7]), make_float2(P[3], P[7]), n);
+                        const float n2 = n.x + n.y;
+                        const bool in = pend && n2 <= 88.f;  // then every |P_i| <= 9 as well
+                        float2 k = __fmul2_rn(make_float2(P[0], P[4]), make_float2(1000.f, 1000.f));
+                        k = __ffma2_rn(make_float2(P[1], P[5]), make_float2(100.f, 100.f), k);
+                        k = __ffma2_rn(make_float2(P[2], P[6]), make_float2(10.f, 10.f), k);
+                        k = __fadd2_rn(make_float2(P[3], P[7]), k);
+                        const float base = ((oddm >> h) & 1u) ? 14999.5f : 4444.f;  // type * 10000 + 1111 * (4.5 or 4)
+                        const int hk = __float_as_int(fmaf(k.x, 0.5f, base) + 8388608.f) - 0x4B000000;
+                        const int lk = __float_as_int(fmaf(k.y, 0.5f, base) + 8388608.f) - 0x4B000000;
+                        const int lv = __float_as_int(fmaf(n2, 0.125f, 8388608.f)) - 0x4B000000;
+                        ia[h] = in ? __ldg(g_t1e + hk * 12 + lv) : 0xFFFFFFFFu;
+                        ib[h] = in ? __ldg(g_t2e + lk) : 0xFFFFFFFFu;
+                    }
+                    uint32_t ew[8];
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) {
+                        const uint32_t r = ia[h] + ib[h];
+                        const bool hit = ia[h] != 0xFFFFFFFFu && ib[h] != 0xFFFFFFFFu && r < static_cast<uint32_t>(kExtPoints);
+                        ew[h] = hit ? __ldg(g_res + r) : (2u << 24);
+                    }
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) {
+                        if (!lane_ok) continue;
                         const int gt = 256 * w + 32 * a + 4 * h + q;
-                        const float (&Pf)[8] = v[h];
-                        const int rk = rks[h];
-                        const bool pend = lane_ok && rk < 0;
-                        if (lane_ok && !pend) map[map_slot(gt)] = static_cast<uint32_t>(rk);
-                        const unsigned bal = __ballot_sync(0xFFFFFFFFu, pend);
-                        if (pend) {
-                            uint32_t* e = qbuf + 5 * (qn + __popc(bal & lanemask_lt()));
+                        const bool pend = (pendm >> h) & 1u;
+                        const uint32_t word = pend ? ew[h] : static_cast<uint32_t>(rks[h]);
+                        map[map_slot(gt)] = word;
+                        if (pend && (word >> 24) == 2) {  // overflow record: keep the coordinates
                             int Pi[8];
                             bool clamp = false;
 #pragma unroll
                             for (int k = 0; k < 8; ++k) {
-                                Pi[k] = __float_as_int(Pf[k] + 12582912.f) - 0x4B400000;
+                                Pi[k] = __float_as_int(v[h][k] + 12582912.f) - 0x4B400000;
                                 if (p.clamp) {
                                     const int c16 = max(-32768, min(32767, Pi[k]));
                                     clamp |= c16 != Pi[k];
                                     Pi[k] = c16;
                                 }
                             }
-                            e[0] = static_cast<uint32_t>(gt) | (static_cast<uint32_t>(Pi[0]) << 16);
-                            e[1] = (static_cast<uint32_t>(Pi[1]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[2]) << 16);
-                            e[2] = (static_cast<uint32_t>(Pi[3]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[4]) << 16);
-                            e[3] = (static_cast<uint32_t>(Pi[5]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[6]) << 16);
-                            e[4] = (static_cast<uint32_t>(Pi[7]) & 0xFFFFu) | (clamp ? 0x10000u : 0u);
-                        }
-                        qn += __popc(bal);
-                        if (h == 3 || h == 7) {
-                            __syncwarp();
-                            int qh = 0;
-                            const int until = (h == 7) ? qn : (qn & ~31);
-                            for (; qh < until; qh += 64) {
-                                const int sl[2] = {qh + lane, qh + 32 + lane};
-                                const bool okk[2] = {qh + lane < until, qh + 32 + lane < until};
-                                resolve_entries<2>(qbuf, sl, okk, map, oscr, clamped);
-                            }
-                            qh = until;
-                            __syncwarp();
-                            if (h == 3 && qh > 0) {  // move the partial batch to the front
-                                const int left = qn - qh;
-                                uint32_t t[5];
-                                if (lane < left)
-#pragma unroll
-                                    for (int k = 0; k < 5; ++k) t[k] = qbuf[5 * (qh + lane) + k];
-                                __syncwarp();
-                                if (lane < left)
-#pragma unroll
-                                    for (int k = 0; k < 5; ++k) qbuf[5 * lane + k] = t[k];
-                                __syncwarp();
-                                qn = left;
-                            }
+                            uint4 o;
+                            o.x = (static_cast<uint32_t>(Pi[0]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[1]) << 16);
+                            o.y = (static_cast<uint32_t>(Pi[2]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[3]) << 16);
+                            o.z = (static_cast<uint32_t>(Pi[4]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[5]) << 16);
+                            o.w = (static_cast<uint32_t>(Pi[6]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[7]) << 16);
+                            *reinterpret_cast<uint4*>(oscr + 8 * gt) = o;
+                            if (clamp) ++clamped;
                         }
                     }
+                    __syncwarp();
 
                     // dequantised weights
                     if (p.dq_mode == E8Q_DEQUANT_ROTATED) {
