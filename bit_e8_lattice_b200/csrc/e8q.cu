@@ -10,6 +10,7 @@
 #include "../../include/e8q.h"
 #include "common.cuh"
 #include "decode.cuh"
+#include "decode_fast.cuh"
 #include "encode.cuh"
 #include "encode_fast.cuh"
 #include "gemv.cuh"
@@ -61,6 +62,9 @@ e8q_status ensure_device(int* dev_out) {
                                               kFastSmemBytes));
         if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileMaxElems * 4));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_decode_fast, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              static_cast<int>(kDfSmemBytes)));
         if (st == E8Q_OK) {
             // GEMV codeword words: nibble i = P_i + 8
             std::vector<uint32_t> words(65536);
@@ -360,6 +364,7 @@ e8q_status e8q_decode(const e8q_encoded* m, int32_t basis, void* out_bf16, e8q_s
     if (m->rows == 0) return E8Q_OK;
     if (!out_bf16 || !aligned(out_bf16, 16)) return E8Q_ERR_INVALID_ARG;
     if (basis == E8Q_DEQUANT_ORIGINAL && (!m->signs || !aligned(m->signs, 8))) return E8Q_ERR_INVALID_ARG;
+    if (m->esc_row_ptr && !aligned(m->esc, 8)) return E8Q_ERR_INVALID_ARG;
     int dev;
     st = ensure_device(&dev);
     if (st != E8Q_OK) return st;
@@ -379,6 +384,13 @@ e8q_status e8q_decode(const e8q_encoded* m, int32_t basis, void* out_bf16, e8q_s
     p.cols = static_cast<int32_t>(m->cols);
     p.logb = logb;
     p.basis = basis;
+    if (p.cols % 256 == 0 && logb >= 8) {  // register Hadamard path
+        p.rpt = decode_fast_rows_per_tile(p.cols);
+        p.n_tiles = (p.rows + p.rpt - 1) / p.rpt;
+        const int grid = p.n_tiles < 2 * g_sms[dev] ? p.n_tiles : 2 * g_sms[dev];
+        k_decode_fast<<<grid, kDfThreads, kDfSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+        return cuda_ok(cudaGetLastError());
+    }
     p.rpt = rows_per_tile(p.cols);
     p.n_tiles = (p.rows + p.rpt - 1) / p.rpt;
     const int grid = p.n_tiles < 2 * g_sms[dev] ? p.n_tiles : 2 * g_sms[dev];

@@ -227,6 +227,88 @@ __device__ __forceinline__ void load_window_raw(unsigned (&raw)[8][4], const uin
     }
 }
 
+// Original-basis dequant of one window, in place of its lattice points:
+// v holds doubled coordinates P in the transposed layout (lane (a, q), row
+// h = group 32 a + 4 h + q of the window); writes bf16 (s_r / sqrt(B)) *
+// d (.) H_B(p) for the window's chunks (dq_tile: the tile's first element;
+// rowm[r] = s_r / sqrt(B) per tile row).  H(p) is exact.
+__device__ __forceinline__ void window_dequant_original(float (&v)[8][8], float4* scratch, int lane, const HFrag& hf,
+                                                        int logb, uint16_t* dq_tile, const int8_t* signs, int C,
+                                                        int wbase, int nchunks, const float* rowm, bool win_rows,
+                                                        int row_w) {
+    // H(p) exactly: tensor-core stage on bf16 p = P/2 (split in two
+    // bf16 terms when some |P| >= 256), fp32 butterflies for the rest.
+    bool big = false;
+#pragma unroll
+    for (int h = 0; h < 8; ++h)
+#pragma unroll
+        for (int e = 0; e < 8; ++e) big |= fabsf(v[h][e]) > 255.f;
+    big = __any_sync(0xFFFFFFFFu, big);
+#pragma unroll
+    for (int h = 0; h < 8; ++h) {
+        float o[8];
+        unsigned r[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __nv_bfloat162 t = __floats2bfloat162_rn(0.5f * v[h][2 * j], 0.5f * v[h][2 * j + 1]);
+            r[j] = *reinterpret_cast<const unsigned*>(&t);
+        }
+        mma_h16(o, r[0], r[1], r[2], r[3], hf);
+        if (big) {  // p = t0 + t1 + t2, each term exact in bf16 (24 bits)
+            float rem[8];
+#pragma unroll
+            for (int j = 0; j < 4; ++j) {
+                const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&r[j]);
+                rem[2 * j] = 0.5f * v[h][2 * j] - __bfloat162float(hi.x);
+                rem[2 * j + 1] = 0.5f * v[h][2 * j + 1] - __bfloat162float(hi.y);
+            }
+#pragma unroll
+            for (int term = 0; term < 2; ++term) {
+#pragma unroll
+                for (int j = 0; j < 4; ++j) {
+                    const __nv_bfloat162 t = __floats2bfloat162_rn(rem[2 * j], rem[2 * j + 1]);
+                    r[j] = *reinterpret_cast<const unsigned*>(&t);
+                    rem[2 * j] -= __bfloat162float(t.x);
+                    rem[2 * j + 1] -= __bfloat162float(t.y);
+                }
+                float o2[8];
+                mma_h16(o2, r[0], r[1], r[2], r[3], hf);
+#pragma unroll
+                for (int e = 0; e < 8; ++e) o[e] += o2[e];
+            }
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[h][e] = o[e];
+    }
+    stage_e2(v);
+    stage_rows<1>(v);
+    stage_rows<2>(v);
+    stage_rows<4>(v);
+    warp_transpose(v, scratch, lane);
+    if (logb >= 9) stage_rows<1>(v);
+    if (logb >= 10) stage_rows<2>(v);
+    if (logb >= 11) stage_rows<4>(v);
+    uint16_t* dq = dq_tile;
+    int tc = (wbase + 8 * lane) % C, tr = (wbase + 8 * lane) / C;  // column, row of chunk 0
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        const int col = tc, rowk = tr;
+        tc += 256;
+        if (tc >= C) { tc -= C; ++tr; }
+        if (k >= nchunks) continue;
+        const int te = wbase + 256 * k + 8 * lane;  // tile element of the 8-run
+        const float m = rowm[win_rows ? row_w : rowk];
+        unsigned o[4];
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            const __nv_bfloat162 t = __floats2bfloat162_rn(v[k][2 * j] * m, v[k][2 * j + 1] * m);
+            o[j] = *reinterpret_cast<const unsigned*>(&t);
+        }
+        apply_signs(o, __ldg(reinterpret_cast<const uint2*>(signs + col)));
+        *reinterpret_cast<uint4*>(dq + te) = make_uint4(o[0], o[1], o[2], o[3]);
+    }
+}
+
 template <int MAXM>
 __device__ __forceinline__ FastTile make_tile(const EncodeParams<MAXM>& p, int t) {
     FastTile ft;
@@ -535,77 +617,9 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                             *reinterpret_cast<uint4*>(dq + 8 * gt) = o;
                         }
                     } else if (p.dq_mode == E8Q_DEQUANT_ORIGINAL) {
-                        // H(p) exactly: tensor-core stage on bf16 p = P/2 (split in two
-                        // bf16 terms when some |P| >= 256), fp32 butterflies for the rest.
-                        bool big = false;
-#pragma unroll
-                        for (int h = 0; h < 8; ++h)
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) big |= fabsf(v[h][e]) > 255.f;
-                        big = __any_sync(0xFFFFFFFFu, big);
-#pragma unroll
-                        for (int h = 0; h < 8; ++h) {
-                            float o[8];
-                            unsigned r[4];
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const __nv_bfloat162 t = __floats2bfloat162_rn(0.5f * v[h][2 * j], 0.5f * v[h][2 * j + 1]);
-                                r[j] = *reinterpret_cast<const unsigned*>(&t);
-                            }
-                            mma_h16(o, r[0], r[1], r[2], r[3], hf);
-                            if (big) {  // p = t0 + t1 + t2, each term exact in bf16 (24 bits)
-                                float rem[8];
-#pragma unroll
-                                for (int j = 0; j < 4; ++j) {
-                                    const __nv_bfloat162 hi = *reinterpret_cast<const __nv_bfloat162*>(&r[j]);
-                                    rem[2 * j] = 0.5f * v[h][2 * j] - __bfloat162float(hi.x);
-                                    rem[2 * j + 1] = 0.5f * v[h][2 * j + 1] - __bfloat162float(hi.y);
-                                }
-#pragma unroll
-                                for (int term = 0; term < 2; ++term) {
-#pragma unroll
-                                    for (int j = 0; j < 4; ++j) {
-                                        const __nv_bfloat162 t = __floats2bfloat162_rn(rem[2 * j], rem[2 * j + 1]);
-                                        r[j] = *reinterpret_cast<const unsigned*>(&t);
-                                        rem[2 * j] -= __bfloat162float(t.x);
-                                        rem[2 * j + 1] -= __bfloat162float(t.y);
-                                    }
-                                    float o2[8];
-                                    mma_h16(o2, r[0], r[1], r[2], r[3], hf);
-#pragma unroll
-                                    for (int e = 0; e < 8; ++e) o[e] += o2[e];
-                                }
-                            }
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) v[h][e] = o[e];
-                        }
-                        stage_e2(v);
-                        stage_rows<1>(v);
-                        stage_rows<2>(v);
-                        stage_rows<4>(v);
-                        warp_transpose(v, scratch, lane);
-                        if (logb >= 9) stage_rows<1>(v);
-                        if (logb >= 10) stage_rows<2>(v);
-                        if (logb >= 11) stage_rows<4>(v);
-                        uint16_t* dq = static_cast<uint16_t*>(M.dq) + static_cast<size_t>(cur.r0) * C;
-                        int tc = (wbase + 8 * lane) % C, tr = (wbase + 8 * lane) / C;  // column, row of chunk 0
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) {
-                            const int col = tc, rowk = tr;
-                            tc += 256;
-                            if (tc >= C) { tc -= C; ++tr; }
-                            if (k >= nchunks) continue;
-                            const int te = wbase + 256 * k + 8 * lane;  // tile element of the 8-run
-                            const float m = rowm_b[win_rows ? row_w : rowk];
-                            unsigned o[4];
-#pragma unroll
-                            for (int j = 0; j < 4; ++j) {
-                                const __nv_bfloat162 t = __floats2bfloat162_rn(v[k][2 * j] * m, v[k][2 * j + 1] * m);
-                                o[j] = *reinterpret_cast<const unsigned*>(&t);
-                            }
-                            apply_signs(o, __ldg(reinterpret_cast<const uint2*>(M.signs + col)));
-                            *reinterpret_cast<uint4*>(dq + te) = make_uint4(o[0], o[1], o[2], o[3]);
-                        }
+                        window_dequant_original(v, scratch, lane, hf, logb,
+                                                static_cast<uint16_t*>(M.dq) + static_cast<size_t>(cur.r0) * C, M.signs, C,
+                                                wbase, nchunks, rowm_b, win_rows, row_w);
                     }
                 }
                 if (w < nwin) {

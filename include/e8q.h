@@ -211,8 +211,11 @@ e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_
  *   basis E8Q_DEQUANT_ROTATED:  out = bf16(s_r * p), one rounding of the
  *                               exact product;
  *   basis E8Q_DEQUANT_ORIGINAL: out = bf16(d (.) H_B (s_r * p) / sqrt(B)).
- * out_bf16: [rows][cols] bf16, 16-byte aligned.  Requires that the encode
- * call dropped no records.
+ * out_bf16: [rows][cols] bf16, 16-byte aligned.  m->esc 8-byte aligned.
+ * Records must be listed per row through the row pointers (as the encode
+ * writes them); records outside their tile's rows are ignored.  Requires
+ * that the encode call dropped no records.  Asynchronous on `stream`;
+ * errors: INVALID_ARG, UNSUPPORTED, CUDA.
  */
 e8q_status e8q_decode(const e8q_encoded* m /* host */, int32_t basis, void* out_bf16, e8q_stream stream);
 

@@ -427,6 +427,28 @@ def test_mlp_full_size_sampled_rows(e8q, mlp_full):
     assert rp[0] == 0 and (np.diff(rp) >= 0).all() and rp[-1] == ctr["n_escape"]
 
 
+def test_decode_full_size(e8q, mlp_full):
+    """Decode of both full-size matrices: the original basis equals the
+    encode's own original-basis output bit for bit (same points, scales and
+    arithmetic); the rotated basis matches the oracle on sampled rows."""
+    res = mlp_full["res"]
+    rng = np.random.default_rng(321)
+    signs = [mlp_full["d_up"], mlp_full["d_dn"]]
+    for i in range(2):
+        m = res.encoded[i]
+        out = e8q.e8q_decode(m, "original")
+        torch.cuda.synchronize()
+        assert torch.equal(out.view(torch.int16), res.dequant[i].view(torch.int16)), f"matrix {i}: decode != encode dequant"
+        rot = e8q.e8q_decode(m, "rotated").cpu().view(torch.int16).numpy()
+        rows = np.sort(rng.choice(m.rows, 5, replace=False))
+        idx = host_idx(res.idx[i])
+        gpr = m.cols // 8
+        P_all, _, _, _, _ = gpu_points(idx.reshape(-1), res.escape_records(), res.overflow_records(), idx.size,
+                                       res.group_base[i])
+        P = P_all.reshape(m.rows, gpr, 8)[rows].reshape(-1, 8)
+        check_rotated_dequant(rot[rows], P, res.scale[i].cpu().numpy()[rows], signs[i], 2048, f"decode rotated [{i}]")
+
+
 @pytest.mark.parametrize("batch", [1, 4, 16, 64])
 def test_gemv_full_size(e8q, mlp_full, batch):
     res = mlp_full["res"]
