@@ -10,7 +10,7 @@
 //
 // Three launches:
 //  k_gv_prep  (a) per activation row and 2048-column segment: xr in fp32
-//             (natural order) and in fp16 scaled by a power of two chosen
+//             (group-major) and in fp16 scaled by a power of two chosen
 //             from the row's largest |x| so that no value can overflow fp16,
 //             stored in the order in which the MMA B fragments are read;
 //             (b) per weight row: a dense byte map group -> root + 1 (0: no
@@ -120,7 +120,7 @@ __host__ __device__ __forceinline__ int64_t gv_cta_of(int64_t u, int64_t T, int6
 struct GvPrepParams {
     const uint16_t* x;  // bf16 [batch][cols]
     const int8_t* signs;
-    float* x32;         // [cols][batch] (column-major: one group's batch rows contiguous)
+    float* x32;         // [groups][batch][8]: one group's 8 values of every batch row together
     uint4* x16;         // [nchunks][nbt][8 k-steps][32 lanes] x 8 halves
     float* xe;          // [batch]: 2^e, x16 = xr * 2^-e
     const e8q_escape* esc;
@@ -192,9 +192,11 @@ __global__ void __launch_bounds__(256) k_gv_prep(const __grid_constant__ GvPrepP
         __syncthreads();
         if (G.logb > 0) fwht_smem(buf, n, G.logb);
         const float inv = 1.0f / sqrtf(static_cast<float>(1 << G.logb));
-        for (int i = threadIdx.x; i < n; i += 256) p.x32[static_cast<size_t>(c0 + i) * G.batch + b] = buf[i] * inv;
         for (int t = threadIdx.x; t < n / 8; t += 256) {
             const int col = c0 + 8 * t;
+            float4* xg = reinterpret_cast<float4*>(p.x32 + (static_cast<size_t>(col >> 3) * G.batch + b) * 8);
+            xg[0] = make_float4(buf[8 * t] * inv, buf[8 * t + 1] * inv, buf[8 * t + 2] * inv, buf[8 * t + 3] * inv);
+            xg[1] = make_float4(buf[8 * t + 4] * inv, buf[8 * t + 5] * inv, buf[8 * t + 6] * inv, buf[8 * t + 7] * inv);
             const int c = col >> 8, gc = (col & 255) >> 3, q = gc >> 3, j = gc & 7;
             const int L = 4 * (b & 7) + q;
             float v[8];
@@ -616,17 +618,19 @@ __global__ void __launch_bounds__(256) k_gv_fin(const __grid_constant__ GvFinPar
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 if (gls[i] < 0) continue;
-                const float* xc = p.x32 + static_cast<size_t>(gls[i]) * 8 * G.batch;
+                const float4* xc = reinterpret_cast<const float4*>(p.x32 + static_cast<size_t>(gls[i]) * G.batch * 8);
 #pragma unroll
                 for (int k = 0; k < KB; ++k) {
                     const int b = bl + BL * k;
                     if (b < G.batch) {
+                        const float4 u = __ldg(xc + 2 * b), t = __ldg(xc + 2 * b + 1);
+                        const float xv[8] = {u.x, u.y, u.z, u.w, t.x, t.y, t.z, t.w};
                         float a = acc[k];
 #pragma unroll
                         for (int c = 0; c < 8; ++c) {
                             const int v = (c & 1) ? (cw[i][c >> 1] >> 16)
                                                   : static_cast<int>(static_cast<int16_t>(cw[i][c >> 1] & 0xFFFF));
-                            a = fmaf(static_cast<float>(v), __ldg(xc + static_cast<size_t>(c) * G.batch + b), a);
+                            a = fmaf(static_cast<float>(v), xv[c], a);
                         }
                         acc[k] = a;
                     }
