@@ -623,8 +623,15 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     }
                 }
                 if (w < nwin) {
-                    // the window's record counts per 32-group chunk, and its indices
+                    // the window's record counts per 32-group chunk and its indices;
+                    // its records are compacted, in group order, over its own 256 map
+                    // entries: local group << 24 | root << 16 | core index, the root
+                    // field 0xFF for an overflow record.  A record lands at or before
+                    // the slots of its own chunk, all read before the chunk's ballots.
                     uint32_t* cnt = schunk + sl * 2 * kFastCnt;
+                    uint32_t* wl = map + 256 * w;
+                    unsigned run = 0;
+                    const unsigned lt = lanemask_lt();
                     __syncwarp();
 #pragma unroll
                     for (int k = 0; k < 8; ++k) {
@@ -639,56 +646,50 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                             cnt[c] = __popc(be);
                             cnt[kFastCnt + c] = __popc(bo);
                         }
+                        if (kind != 0)
+                            wl[run + __popc((be | bo) & lt)] =
+                                (static_cast<uint32_t>(32 * k + lane) << 24) | (kind == 1 ? (m & 0xFFFFFFu) : 0xFF0000u);
+                        run += __popc(be | bo);
                     }
                 }
             }
             // emit the records of tile i - 3, placed by the service warp during
-            // the previous iteration: each warp its own window's 8 chunks, all
-            // loads before the ballots and stores
+            // the previous iteration: each warp copies its own window's compacted
+            // list, escape and overflow records each to their contiguous range
             if (p3_ok) {
                 const MatDesc& M = p.m[prev3.mat];
                 const int gpr = M.cols >> 3, G = prev3.nr * gpr, nch = (G + 31) >> 5;
-                const uint32_t* map = smap + sl3 * kFastTileGroups;
                 const uint32_t* cnt = schunk + sl3 * 2 * kFastCnt;
-                const int16_t* oscr = ovf_scratch + static_cast<size_t>(sl3) * kFastTileGroups * 8;
                 const long long ex_e = s_ex[sl3][0], ex_o = s_ex[sl3][1];
-                const uint32_t gid0 = M.group_base + static_cast<uint32_t>(prev3.r0) * gpr;
-                for (int c0 = 8 * warp; c0 < nch && c0 < 8 * warp + 8; c0 += 8) {
-                    uint32_t m[8];
-                    uint4 cw[8];
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int g = 32 * (c0 + k) + lane;
-                        m[k] = (c0 + k < nch && g < G) ? map[map_slot(g)] : 0u;
-                    }
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int g = 32 * (c0 + k) + lane;
-                        cw[k] = (m[k] >> 24) == 2 ? *reinterpret_cast<const uint4*>(oscr + 8 * g) : make_uint4(0, 0, 0, 0);
-                    }
-#pragma unroll
-                    for (int k = 0; k < 8; ++k) {
-                        const int c = c0 + k;
-                        if (c >= nch) break;
-                        const int g = 32 * c + lane;
-                        const uint32_t kind = m[k] >> 24;
-                        const unsigned be = __ballot_sync(0xFFFFFFFFu, kind == 1), bo = __ballot_sync(0xFFFFFFFFu, kind == 2);
-                        if (kind == 1) {
-                            const long long pos = ex_e + cnt[c] + __popc(be & lanemask_lt());
-                            if (pos < p.esc_cap) {
-                                uint2 r;
-                                r.x = gid0 + g;
-                                r.y = (m[k] & 0xFFFFu) | (((m[k] >> 16) & 0xFFu) << 16);
-                                *reinterpret_cast<uint2*>(p.esc + pos) = r;
-                            }
-                        } else if (kind == 2) {
-                            const long long pos = ex_o + cnt[kFastCnt + c] + __popc(bo & lanemask_lt());
+                if (8 * warp < nch) {
+                    const int c0 = 8 * warp;
+                    const uint32_t* wl = smap + sl3 * kFastTileGroups + 256 * warp;
+                    const int16_t* oscr = ovf_scratch + (static_cast<size_t>(sl3) * kFastTileGroups + 256 * warp) * 8;
+                    const uint32_t gw = M.group_base + static_cast<uint32_t>(prev3.r0) * gpr + 256u * warp;
+                    long long pe = ex_e + cnt[c0], po = ex_o + cnt[kFastCnt + c0];
+                    const int n = static_cast<int>((cnt[c0 + 8] - cnt[c0]) + (cnt[kFastCnt + c0 + 8] - cnt[kFastCnt + c0]));
+                    const unsigned lt = lanemask_lt();
+                    for (int j0 = 0; j0 < n; j0 += 32) {
+                        const int j = j0 + lane;
+                        const uint32_t e = j < n ? wl[j] : 0u;
+                        const bool ov = j < n && ((e >> 16) & 0xFFu) == 0xFFu;
+                        const bool es = j < n && !ov;
+                        const unsigned be = __ballot_sync(0xFFFFFFFFu, es), bo = __ballot_sync(0xFFFFFFFFu, ov);
+                        const uint32_t lg = e >> 24;
+                        if (es) {
+                            const long long pos = pe + __popc(be & lt);
+                            if (pos < p.esc_cap) *reinterpret_cast<uint2*>(p.esc + pos) = make_uint2(gw + lg, e & 0xFFFFFFu);
+                        } else if (ov) {
+                            const long long pos = po + __popc(bo & lt);
                             if (pos < p.ovf_cap) {
+                                const uint4 cw = *reinterpret_cast<const uint4*>(oscr + 8 * lg);
                                 uint32_t* dst = reinterpret_cast<uint32_t*>(p.ovf + pos);
-                                dst[0] = gid0 + g;
-                                dst[1] = cw[k].x; dst[2] = cw[k].y; dst[3] = cw[k].z; dst[4] = cw[k].w;
+                                dst[0] = gw + lg;
+                                dst[1] = cw.x; dst[2] = cw.y; dst[3] = cw.z; dst[4] = cw.w;
                             }
                         }
+                        pe += __popc(be);
+                        po += __popc(bo);
                     }
                 }
                 for (int r = tid; r < prev3.nr; r += kFastWarps * 32) {
