@@ -63,8 +63,11 @@ e8q_status ensure_device(int* dev_out) {
         if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileMaxElems * 4));
         if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_decode_fast, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              static_cast<int>(kDfSmemBytes)));
+            st = cuda_ok(cudaFuncSetAttribute(k_decode_fast<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              static_cast<int>(decode_fast_smem_bytes(false))));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_decode_fast<true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              static_cast<int>(decode_fast_smem_bytes(true))));
         if (st == E8Q_OK) {
             // GEMV codeword words: nibble i = P_i + 8
             std::vector<uint32_t> words(65536);
@@ -384,11 +387,21 @@ e8q_status e8q_decode(const e8q_encoded* m, int32_t basis, void* out_bf16, e8q_s
     p.cols = static_cast<int32_t>(m->cols);
     p.logb = logb;
     p.basis = basis;
-    if (p.cols % 256 == 0 && logb >= 8) {  // register Hadamard path
+    // fast path (original basis through the register Hadamard, B >= 256); its
+    // staging warp copies indices in 16-byte words and overflow group ids in
+    // 4-byte words
+    const bool orig = basis == E8Q_DEQUANT_ORIGINAL;
+    if (p.cols % 256 == 0 && (!orig || logb >= 8) && (reinterpret_cast<uintptr_t>(p.idx) & 15) == 0 &&
+        (reinterpret_cast<uintptr_t>(p.ovf) & 3) == 0) {
         p.rpt = decode_fast_rows_per_tile(p.cols);
         p.n_tiles = (p.rows + p.rpt - 1) / p.rpt;
-        const int grid = p.n_tiles < 2 * g_sms[dev] ? p.n_tiles : 2 * g_sms[dev];
-        k_decode_fast<<<grid, kDfThreads, kDfSmemBytes, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+        const int per_sm = orig ? kDfCtasOrig : kDfCtasRot;
+        const int grid = p.n_tiles < per_sm * g_sms[dev] ? p.n_tiles : per_sm * g_sms[dev];
+        if (orig)
+            k_decode_fast<true><<<grid, kDfThreads, decode_fast_smem_bytes(true), reinterpret_cast<cudaStream_t>(stream)>>>(p);
+        else
+            k_decode_fast<false>
+                <<<grid, kDfThreads, decode_fast_smem_bytes(false), reinterpret_cast<cudaStream_t>(stream)>>>(p);
         return cuda_ok(cudaGetLastError());
     }
     p.rpt = rows_per_tile(p.cols);

@@ -610,10 +610,10 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                             const int gt = 256 * w + 32 * a + 4 * h + q;
                             const float s = rows_b[win_rows ? row_w : r0l + (h >= hcut ? 1 : 0)];
                             uint4 o;
-                            o.x = pack_bf16x2(bf16_of_product(s, 0.5f * v[h][0]), bf16_of_product(s, 0.5f * v[h][1]));
-                            o.y = pack_bf16x2(bf16_of_product(s, 0.5f * v[h][2]), bf16_of_product(s, 0.5f * v[h][3]));
-                            o.z = pack_bf16x2(bf16_of_product(s, 0.5f * v[h][4]), bf16_of_product(s, 0.5f * v[h][5]));
-                            o.w = pack_bf16x2(bf16_of_product(s, 0.5f * v[h][6]), bf16_of_product(s, 0.5f * v[h][7]));
+                            o.x = bf16x2_of_half_products(s, v[h][0], v[h][1]);
+                            o.y = bf16x2_of_half_products(s, v[h][2], v[h][3]);
+                            o.z = bf16x2_of_half_products(s, v[h][4], v[h][5]);
+                            o.w = bf16x2_of_half_products(s, v[h][6], v[h][7]);
                             *reinterpret_cast<uint4*>(dq + 8 * gt) = o;
                         }
                     } else if (p.dq_mode == E8Q_DEQUANT_ORIGINAL) {

@@ -197,6 +197,44 @@ __device__ __forceinline__ unsigned pack_bf16x2(__nv_bfloat16 lo, __nv_bfloat16 
     return static_cast<unsigned>(__bfloat16_as_ushort(lo)) | (static_cast<unsigned>(__bfloat16_as_ushort(hi)) << 16);
 }
 
+// bf16 nearest of the exact products s * P0 / 2 and s * P1 / 2 (P small
+// integers, |P| < 2^16), packed lo | hi << 16: the same round-to-odd
+// argument as bf16_of_product on fp32 pairs.  s / 2 is exact for
+// |s| >= 1e-30; smaller scales take the double product.
+__device__ __forceinline__ unsigned bf16x2_of_half_products(float s, float P0, float P1) {
+    if (fabsf(s) < 1e-30f) {
+        const double sd = 0.5 * static_cast<double>(s);
+        return pack_bf16x2(__double2bfloat16(sd * static_cast<double>(P0)), __double2bfloat16(sd * static_cast<double>(P1)));
+    }
+    const float sh = 0.5f * s;
+    const float2 q = make_float2(P0, P1), ss = make_float2(sh, sh);
+    const float2 p = __fmul2_rz(ss, q);
+    const float2 r = __ffma2_rn(ss, q, make_float2(-p.x, -p.y));
+    const float lo = __uint_as_float(__float_as_uint(p.x) | (r.x != 0.f ? 1u : 0u));
+    const float hi = __uint_as_float(__float_as_uint(p.y) | (r.y != 0.f ? 1u : 0u));
+    const __nv_bfloat162 t = __floats2bfloat162_rn(lo, hi);
+    return *reinterpret_cast<const unsigned*>(&t);
+}
+
+// The 8 signed bytes of a packed point as exact floats: each byte, biased by
+// 128, is placed under the exponent of 2^23 and the bias removed again.
+__device__ __forceinline__ void bytes_to_floats(uint2 w, float (&f)[8]) {
+    const unsigned x = w.x ^ 0x80808080u, y = w.y ^ 0x80808080u;
+#pragma unroll
+    for (int j = 0; j < 4; j += 2) {
+        const float2 a = make_float2(__uint_as_float(__byte_perm(x, 0x4B000000u, 0x7440u + j)),
+                                     __uint_as_float(__byte_perm(x, 0x4B000000u, 0x7441u + j)));
+        const float2 b = make_float2(__uint_as_float(__byte_perm(y, 0x4B000000u, 0x7440u + j)),
+                                     __uint_as_float(__byte_perm(y, 0x4B000000u, 0x7441u + j)));
+        const float2 fa = __fadd2_rn(a, make_float2(-8388736.f, -8388736.f));
+        const float2 fb = __fadd2_rn(b, make_float2(-8388736.f, -8388736.f));
+        f[j] = fa.x;
+        f[j + 1] = fa.y;
+        f[4 + j] = fb.x;
+        f[4 + j + 1] = fb.y;
+    }
+}
+
 __device__ __forceinline__ int8_t coord_of(uint2 packed, int i) {
     const unsigned w = i < 4 ? packed.x : packed.y;
     return static_cast<int8_t>((w >> (8 * (i & 3))) & 0xFF);

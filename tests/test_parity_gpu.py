@@ -249,6 +249,31 @@ def test_bf16_nonfinite_inputs(e8q):
                            d, 2048, "nonfinite original")
 
 
+@pytest.mark.parametrize("kappa", [0.45, 1.0, 1.5, 200.0])
+def test_decode_record_heavy_tiles(e8q, kappa):
+    """Decode of 2048-wide rows (7 rows a tile, ragged last tile) at scales
+    whose tiles hold no records, or hundreds to thousands of them:
+    bit-identical to the encode's own dequant in both bases, and the rotated
+    one equal to the oracle's s * p."""
+    rng = np.random.default_rng(int(kappa * 100) + 9)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((50, 2048)) * 0.02)
+    d = synth.signs(31, 2048)
+    for mode in ("rotated", "original"):
+        enc, res = run_encode(e8q, [w], [d], 0, kappa=kappa, dequant=mode)
+        st = compare_all(e8q, res, [w], [d], [2048], kappa=kappa, label=f"kappa{kappa} {mode}")[0]
+        dq = res.dequant[0].cpu().view(torch.int16).numpy()
+        out = e8q.e8q_decode(res.encoded[0], mode).cpu().view(torch.int16).numpy()
+        np.testing.assert_array_equal(out, dq)
+        if mode == "rotated":
+            check_rotated_dequant(out, st["points"], res.scale[0].cpu().numpy(), d, 2048, f"kappa{kappa} decode")
+    ctr = res.read_counters()
+    per_tile = 7 * 2048 // 8
+    if kappa == 200.0:
+        assert ctr["n_overflow"] > 2 * per_tile  # every tile past the staging warp's first round
+    if kappa == 1.5:
+        assert ctr["n_escape"] > 8 * 512 and ctr["n_overflow"] > 8 * 64
+
+
 def test_large_points_small_scale(e8q):
     """kappa = 200: |x| in the hundreds, lattice points far outside the core
     (overflow records with large coordinates) and the original-basis dequant
