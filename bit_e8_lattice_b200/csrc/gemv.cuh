@@ -228,7 +228,7 @@ __global__ void __launch_bounds__(256) k_gv_prep(const __grid_constant__ GvPrepP
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
             const long long k = k0 + lane + 32 * i;
-            rec[i] = k < e1 ? __ldcs(reinterpret_cast<const uint2*>(p.esc + k)) : make_uint2(0xFFFFFFFFu, 0u);
+            rec[i] = k < e1 ? __ldcs(reinterpret_cast<const uint2*>(p.esc + k)) : make_uint2(0u, 0xFF0000u);  // root 255: none
         }
 #pragma unroll
         for (int i = 0; i < 8; ++i) {
