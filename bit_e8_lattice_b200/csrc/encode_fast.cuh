@@ -200,7 +200,7 @@ __device__ __forceinline__ float window_forward(float (&v)[8][8], const unsigned
 
 __device__ __forceinline__ void load_window_raw(unsigned (&raw)[8][4], const uint16_t* src_smem_or_global,
                                                 bool from_global, const int8_t* signs, int cols, int col0, int nchunks,
-                                                int lane, unsigned long long& nonfinite) {
+                                                int lane, unsigned& nonfinite) {
     int c = (col0 + 8 * lane) % cols;  // column of this lane's first element; chunks step 256
 #pragma unroll
     for (int k = 0; k < 8; ++k, c = (c + 256 >= cols) ? c + 256 - cols : c + 256) {
@@ -444,7 +444,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
     __syncthreads();
 
     const HFrag hf = make_hfrag(lane);
-    unsigned long long nonfinite = 0, clamped = 0;
+    unsigned nonfinite = 0, clamped = 0;  // per thread: at most 64 a tile
 
     // Iteration i: compute warps transform, project and count tile i and emit
     // the records of tile i - 3; the service warp claims and loads tile i + 1,
@@ -452,10 +452,11 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
     // tile i - 2 among all earlier tiles, and computes tile i + 1's row
     // scales.  One barrier per iteration.
     for (int i = 0;; ++i) {
-        const FastTile cur = s_info[i & 7];
-        const FastTile prev1 = s_info[(i + 7) & 7];
-        const FastTile prev2 = s_info[(i + 6) & 7];
-        const FastTile prev3 = s_info[(i + 5) & 7];
+        // tile descriptors stay in shared memory (the service warp writes only slot i + 1)
+        const FastTile& cur = s_info[i & 7];
+        const FastTile& prev1 = s_info[(i + 7) & 7];
+        const FastTile& prev2 = s_info[(i + 6) & 7];
+        const FastTile& prev3 = s_info[(i + 5) & 7];
         const bool cur_ok = cur.t < p.n_tiles, p1_ok = i >= 1 && prev1.t < p.n_tiles,
                    p2_ok = i >= 2 && prev2.t < p.n_tiles, p3_ok = i >= 3 && prev3.t < p.n_tiles;
         if (!cur_ok && !p1_ok && !p2_ok && !p3_ok) break;
@@ -578,26 +579,30 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         const bool pend = (pendm >> h) & 1u;
                         const uint32_t word = pend ? ew[h] : static_cast<uint32_t>(rks[h]);
                         map[map_slot(gt)] = word;
-                        if (pend && (word >> 24) == 2) {  // overflow record: keep the coordinates
-                            int Pi[8];
-                            bool clamp = false;
+                        // an overflow record keeps the coordinates as int16 (saturated when
+                        // the inputs were clamped); formed for every group, without a branch:
+                        // x + 1.5 * 2^23 holds the integer x in its low 16 bits (|x| < 2^22)
+                        const bool ovf = pend && (word >> 24) == 2;
+                        float c[8];
+                        bool clamp = false;
+#pragma unroll
+                        for (int k = 0; k < 8; ++k) c[k] = v[h][k];
+                        if (p.clamp) {
 #pragma unroll
                             for (int k = 0; k < 8; ++k) {
-                                Pi[k] = __float_as_int(v[h][k] + 12582912.f) - 0x4B400000;
-                                if (p.clamp) {
-                                    const int c16 = max(-32768, min(32767, Pi[k]));
-                                    clamp |= c16 != Pi[k];
-                                    Pi[k] = c16;
-                                }
+                                const float t = fminf(fmaxf(c[k], -32768.f), 32767.f);
+                                clamp |= t != c[k];
+                                c[k] = t;
                             }
-                            uint4 o;
-                            o.x = (static_cast<uint32_t>(Pi[0]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[1]) << 16);
-                            o.y = (static_cast<uint32_t>(Pi[2]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[3]) << 16);
-                            o.z = (static_cast<uint32_t>(Pi[4]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[5]) << 16);
-                            o.w = (static_cast<uint32_t>(Pi[6]) & 0xFFFFu) | (static_cast<uint32_t>(Pi[7]) << 16);
-                            *reinterpret_cast<uint4*>(oscr + 8 * gt) = o;
-                            if (clamp) ++clamped;
                         }
+                        unsigned o[4];
+#pragma unroll
+                        for (int j = 0; j < 4; ++j) {
+                            const float2 t = __fadd2_rn(make_float2(c[2 * j], c[2 * j + 1]), make_float2(12582912.f, 12582912.f));
+                            o[j] = prmt(__float_as_uint(t.x), __float_as_uint(t.y), 0x5410u);
+                        }
+                        if (ovf) *reinterpret_cast<uint4*>(oscr + 8 * gt) = make_uint4(o[0], o[1], o[2], o[3]);
+                        if (ovf && clamp) ++clamped;
                     }
                     __syncwarp();
 
@@ -822,14 +827,15 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
         __syncthreads();
     }
 
+    unsigned long long nf = nonfinite, cl = clamped;
 #pragma unroll
     for (int off = 16; off > 0; off >>= 1) {
-        nonfinite += __shfl_xor_sync(0xFFFFFFFFu, nonfinite, off);
-        clamped += __shfl_xor_sync(0xFFFFFFFFu, clamped, off);
+        nf += __shfl_xor_sync(0xFFFFFFFFu, nf, off);
+        cl += __shfl_xor_sync(0xFFFFFFFFu, cl, off);
     }
     if (lane == 0) {
-        if (nonfinite) atomicAdd(&p.ctr->n_nonfinite, nonfinite);
-        if (clamped) atomicAdd(&p.ctr->n_clamped, clamped);
+        if (nf) atomicAdd(&p.ctr->n_nonfinite, nf);
+        if (cl) atomicAdd(&p.ctr->n_clamped, cl);
     }
 }
 
