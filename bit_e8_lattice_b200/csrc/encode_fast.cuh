@@ -535,25 +535,22 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
 #pragma unroll
                         for (int e = 0; e < 8; ++e) v[h][e] = Pf[e];  // keep p for the dequant
                     }
-                    int rks[8];
-#pragma unroll
-                    for (int h = 0; h < 8; ++h) rks[h] = lane_ok ? core_rank_f(v[h], (oddm >> h) & 1u, g_t1, st2) : 0;
-                    // groups outside the core: extended rank straight from the coordinates
-                    // (digits (P + 9) >> 1 = P / 2 + 4 or + 4.5, keys base 10, exact in fp32),
-                    // the two table gathers of all 8 groups, then their encoding words
+                    // Groups that may lie outside the core: the core holds every point with
+                    // |p|^2 <= 10 and none with |p|^2 > 12, so only |P|^2 > 40 can escape.
+                    // Their extended rank comes straight from the coordinates (digits
+                    // (P + 9) >> 1 = P / 2 + 4 or + 4.5, keys base 10, exact in fp32); the two
+                    // table gathers of all 8 groups are issued before the core rank, so that
+                    // their latency overlaps it, and the encoding words after it.
                     uint32_t ia[8], ib[8];
-                    unsigned pendm = 0u;
 #pragma unroll
                     for (int h = 0; h < 8; ++h) {
                         const float (&P)[8] = v[h];
-                        const bool pend = lane_ok && rks[h] < 0;
-                        pendm |= (pend ? 1u : 0u) << h;
                         float2 n = __fmul2_rn(make_float2(P[0], P[4]), make_float2(P[0], P[4]));
                         n = __ffma2_rn(make_float2(P[1], P[5]), make_float2(P[1], P[5]), n);
                         n = __ffma2_rn(make_float2(P[2], P[6]), make_float2(P[2], P[6]), n);
                         n = __ffma2_rn(make_float2(P[3], P[7]), make_float2(P[3], P[7]), n);
                         const float n2 = n.x + n.y;
-                        const bool in = pend && n2 <= 88.f;  // then every |P_i| <= 9 as well
+                        const bool in = lane_ok && n2 > 40.f && n2 <= 88.f;  // then every |P_i| <= 9 as well
                         float2 k = __fmul2_rn(make_float2(P[0], P[4]), make_float2(1000.f, 1000.f));
                         k = __ffma2_rn(make_float2(P[1], P[5]), make_float2(100.f, 100.f), k);
                         k = __ffma2_rn(make_float2(P[2], P[6]), make_float2(10.f, 10.f), k);
@@ -565,11 +562,18 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         ia[h] = in ? __ldg(g_t1e + hk * 12 + lv) : 0xFFFFFFFFu;
                         ib[h] = in ? __ldg(g_t2e + lk) : 0xFFFFFFFFu;
                     }
+                    int rks[8];
+#pragma unroll
+                    for (int h = 0; h < 8; ++h) rks[h] = lane_ok ? core_rank_f(v[h], (oddm >> h) & 1u, g_t1, st2) : 0;
                     uint32_t ew[8];
+                    unsigned pendm = 0u;
 #pragma unroll
                     for (int h = 0; h < 8; ++h) {
+                        const bool pend = lane_ok && rks[h] < 0;
+                        pendm |= (pend ? 1u : 0u) << h;
                         const uint32_t r = ia[h] + ib[h];
-                        const bool hit = ia[h] != 0xFFFFFFFFu && ib[h] != 0xFFFFFFFFu && r < static_cast<uint32_t>(kExtPoints);
+                        const bool hit = pend && ia[h] != 0xFFFFFFFFu && ib[h] != 0xFFFFFFFFu &&
+                                         r < static_cast<uint32_t>(kExtPoints);
                         ew[h] = hit ? __ldg(g_res + r) : (2u << 24);
                     }
 #pragma unroll
