@@ -539,9 +539,10 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     // |p|^2 <= 10 and none with |p|^2 > 12, so only |P|^2 > 40 can escape.
                     // Their extended rank comes straight from the coordinates (digits
                     // (P + 9) >> 1 = P / 2 + 4 or + 4.5, keys base 10, exact in fp32); the two
-                    // table gathers of all 8 groups are issued before the core rank, so that
-                    // their latency overlaps it, and the encoding words after it.
+                    // table gathers of all 8 groups are issued together with the core ranks,
+                    // so that their latency overlaps them, and the encoding words after them.
                     uint32_t ia[8], ib[8];
+                    int rks[8];
 #pragma unroll
                     for (int h = 0; h < 8; ++h) {
                         const float (&P)[8] = v[h];
@@ -561,10 +562,8 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         const int lv = __float_as_int(fmaf(n2, 0.125f, 8388608.f)) - 0x4B000000;
                         ia[h] = in ? __ldg(g_t1e + hk * 12 + lv) : 0xFFFFFFFFu;
                         ib[h] = in ? __ldg(g_t2e + lk) : 0xFFFFFFFFu;
+                        rks[h] = lane_ok ? core_rank_nb(P, (oddm >> h) & 1u, n2, g_t1, st2) : 0;
                     }
-                    int rks[8];
-#pragma unroll
-                    for (int h = 0; h < 8; ++h) rks[h] = lane_ok ? core_rank_f(v[h], (oddm >> h) & 1u, g_t1, st2) : 0;
                     uint32_t ew[8];
                     unsigned pendm = 0u;
 #pragma unroll

@@ -321,6 +321,27 @@ __device__ __forceinline__ int core_rank_f(const float (&P)[8], bool odd, const 
     return (a != 0xFFFF && r < 65536) ? r : -1;
 }
 
+// core_rank_f without a branch, given n2 = |P|^2: both table reads happen
+// for every group (index 0 outside the key range), so that a warp's groups
+// stay converged.
+__device__ __forceinline__ int core_rank_nb(const float (&P)[8], bool odd, float n2, const uint16_t* __restrict__ t1,
+                                            const uint16_t* __restrict__ t2) {
+    const bool inr = n2 <= 48.f;  // then every |P_i| <= 6: digits in 0..6
+    float2 k = __fmul2_rn(make_float2(P[0], P[4]), make_float2(343.f, 343.f));
+    k = __ffma2_rn(make_float2(P[1], P[5]), make_float2(49.f, 49.f), k);
+    k = __ffma2_rn(make_float2(P[2], P[6]), make_float2(7.f, 7.f), k);
+    k = __fadd2_rn(make_float2(P[3], P[7]), k);
+    const float base = odd ? 3401.f : 1200.f;
+    const float hk = fmaf(k.x, 0.5f, base), lk = fmaf(k.y, 0.5f, base);
+    const float i1 = fmaf(hk, 7.f, n2 * 0.125f);
+    const int j1 = inr ? __float_as_int(i1 + 8388608.f) - 0x4B000000 : 0;
+    const int j2 = inr ? __float_as_int(lk + 8388608.f) - 0x4B000000 : 0;
+    const int a = t1[j1];
+    const int b = t2[j2];
+    const int r = a + b;
+    return (inr && a != 0xFFFF && r < 65536) ? r : -1;
+}
+
 // best_escape_root with bit masks instead of index loops (same choice).
 __device__ __forceinline__ void best_escape_root_lean(const int (&P)[8], int (&R)[8]) {
     int w[8];
