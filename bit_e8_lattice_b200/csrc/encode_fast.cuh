@@ -232,17 +232,22 @@ __device__ __forceinline__ void load_window_raw(unsigned (&raw)[8][4], const uin
 // h = group 32 a + 4 h + q of the window); writes bf16 (s_r / sqrt(B)) *
 // d (.) H_B(p) for the window's chunks (dq_tile: the tile's first element;
 // rowm[r] = s_r / sqrt(B) per tile row).  H(p) is exact.
+// big_hint: 1 if the lane may hold some |P| > 255 (a superset is fine: it
+// only selects the exact three-term path), 0 if it holds none, -1 to test
+// the values here.
 __device__ __forceinline__ void window_dequant_original(float (&v)[8][8], float4* scratch, int lane, const HFrag& hf,
                                                         int logb, uint16_t* dq_tile, const int8_t* signs, int C,
                                                         int wbase, int nchunks, const float* rowm, bool win_rows,
-                                                        int row_w) {
+                                                        int row_w, int big_hint = -1) {
     // H(p) exactly: tensor-core stage on bf16 p = P/2 (split in two
     // bf16 terms when some |P| >= 256), fp32 butterflies for the rest.
-    bool big = false;
+    bool big = big_hint > 0;
+    if (big_hint < 0) {
 #pragma unroll
-    for (int h = 0; h < 8; ++h)
+        for (int h = 0; h < 8; ++h)
 #pragma unroll
-        for (int e = 0; e < 8; ++e) big |= fabsf(v[h][e]) > 255.f;
+            for (int e = 0; e < 8; ++e) big |= fabsf(v[h][e]) > 255.f;
+    }
     big = __any_sync(0xFFFFFFFFu, big);
 #pragma unroll
     for (int h = 0; h < 8; ++h) {
@@ -543,6 +548,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     // so that their latency overlaps them, and the encoding words after them.
                     uint32_t ia[8], ib[8];
                     int rks[8];
+                    bool big = false;  // some |P_i| > 255 implies |P|^2 > 65025
 #pragma unroll
                     for (int h = 0; h < 8; ++h) {
                         const float (&P)[8] = v[h];
@@ -551,6 +557,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         n = __ffma2_rn(make_float2(P[2], P[6]), make_float2(P[2], P[6]), n);
                         n = __ffma2_rn(make_float2(P[3], P[7]), make_float2(P[3], P[7]), n);
                         const float n2 = n.x + n.y;
+                        big |= !(n2 <= 65025.f);
                         const bool in = lane_ok && n2 > 40.f && n2 <= 88.f;  // then every |P_i| <= 9 as well
                         float2 k = __fmul2_rn(make_float2(P[0], P[4]), make_float2(1000.f, 1000.f));
                         k = __ffma2_rn(make_float2(P[1], P[5]), make_float2(100.f, 100.f), k);
@@ -627,7 +634,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     } else if (p.dq_mode == E8Q_DEQUANT_ORIGINAL) {
                         window_dequant_original(v, scratch, lane, hf, logb,
                                                 static_cast<uint16_t*>(M.dq) + static_cast<size_t>(cur.r0) * C, M.signs, C,
-                                                wbase, nchunks, rowm_b, win_rows, row_w);
+                                                wbase, nchunks, rowm_b, win_rows, row_w, big ? 1 : 0);
                     }
                 }
                 if (w < nwin) {
