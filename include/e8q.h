@@ -178,6 +178,17 @@ e8q_status e8q_core_table(int8_t* out_coord2);
  * compare the table with other encoders. */
 e8q_status e8q_escape_lookup(const int8_t* coord2, int64_t n, uint32_t* out);
 
+/* Test and tuning hook: which main kernel e8q_dequant_gemv uses.  0 (the
+ * default): by batch; 1: the mma.sync kernel; 2: the tcgen05 kernel.  Both
+ * give the same sums up to fp32 summation order.  Process-wide; not to be
+ * changed while GEMV calls are being issued. */
+e8q_status e8q_set_gemv_path(int32_t mode);
+
+/* Device-side error flags of the current GPU (host call, synchronous):
+ * bit 0 = a bounded wait in the tcgen05 GEMV kernel gave up (its output is
+ * then undefined).  reset != 0 clears them after reading. */
+e8q_status e8q_device_error_flags(int32_t reset, uint64_t* flags);
+
 /* Workspace bytes e8q_project_encode needs for these matrices (>= 16). */
 size_t e8q_encode_workspace_bytes(const e8q_matrix* mats /* host [n_mats] */, int32_t n_mats);
 
