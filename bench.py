@@ -385,31 +385,61 @@ def main():
         Xh = {b: t_bf16(xs[b], True) for b in batches}
         Yh = {b: torch.empty((b, D_MODEL), dtype=torch.bfloat16).pin_memory() for b in batches}
         Ch = torch.empty(6, dtype=torch.int64).pin_memory()
-        Wd = [torch.empty_like(W[0]), torch.empty_like(W[1])]
-        Xd = {b: torch.empty_like(X[b]) for b in batches}
+        # two device buffer sets: a copy stream uploads step k + 1's inputs
+        # while step k computes, and brings step k's results back; events order
+        # the reuse of each set and of the result buffers
+        Wd = [[torch.empty_like(W[0]), torch.empty_like(W[1])] for _ in range(2)]
+        Xd = [{b: torch.empty_like(X[b]) for b in batches} for _ in range(2)]
         h2d = sum(w.numel() * 2 for w in Wh) + sum(x.numel() * 2 for x in Xh.values())
         d2h = sum(y.numel() * 2 for y in Yh.values()) + 48
+        cs, ps = stream, torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]    # a set's inputs are on the device
+        ev_used = [torch.cuda.Event() for _ in range(2)]  # the step computing from a set is done
+        ev_out = torch.cuda.Event()                       # the latest step's results are on the host
 
-        def e2e_step():
-            for i in range(2):
-                Wd[i].copy_(Wh[i], non_blocking=True)
-            for b in batches:
-                Xd[b].copy_(Xh[b], non_blocking=True)
-            r = enc(Wd)
-            for b in batches:
-                Yh[b].copy_(gemvs[b](Xd[b]), non_blocking=True)
-            Ch.copy_(r.counters, non_blocking=True)
+        def upload(k):
+            j = k % 2
+            with torch.cuda.stream(ps):
+                ps.wait_event(ev_used[j])
+                for i in range(2):
+                    Wd[j][i].copy_(Wh[i], non_blocking=True)
+                for b in batches:
+                    Xd[j][b].copy_(Xh[b], non_blocking=True)
+                ev_in[j].record(ps)
 
-        for _ in range(2):
-            e2e_step()
+        def compute(k):
+            j = k % 2
+            cs.wait_event(ev_in[j])
+            cs.wait_event(ev_out)
+            with torch.cuda.stream(cs):
+                r = enc(Wd[j])
+                ys = {b: gemvs[b](Xd[j][b]) for b in batches}
+            ev_used[j].record(cs)
+            with torch.cuda.stream(ps):
+                ps.wait_event(ev_used[j])
+                for b in batches:
+                    Yh[b].copy_(ys[b], non_blocking=True)
+                Ch.copy_(r.counters, non_blocking=True)
+                ev_out.record(ps)
+
+        def e2e_run(nsteps, start=None):
+            if start is not None:
+                ps.wait_event(start)
+            upload(0)
+            for k in range(nsteps):
+                if k + 1 < nsteps:
+                    upload(k + 1)
+                compute(k)
+            cs.wait_event(ev_out)
+
+        e2e_run(2)
         torch.cuda.synchronize()
         a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
-        a.record(stream)
-        for _ in range(args.e2e_steps):
-            e2e_step()
-        z.record(stream)
+        a.record(cs)
+        e2e_run(args.e2e_steps, start=a)
+        z.record(cs)
         torch.cuda.synchronize()
         ems = max_over_ranks(a.elapsed_time(z), dev)
         e2e = {"value": world * G * args.e2e_steps / (ems * 1e-3) / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
