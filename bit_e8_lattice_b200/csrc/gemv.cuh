@@ -650,20 +650,30 @@ __global__ void __launch_bounds__(256) k_gv_fin(const __grid_constant__ GvFinPar
 #pragma unroll
             for (int i = 0; i < 4; ++i) {
                 if (gls[i] < 0) continue;
+                // the record's coordinates as exact floats, once: an int16 x added to
+                // the bits of 1.5 * 2^23 is that float plus x
+                float pc[8];
+#pragma unroll
+                for (int c = 0; c < 4; ++c) {
+                    const int lo = static_cast<int>(static_cast<int16_t>(cw[i][c] & 0xFFFF)), hi = cw[i][c] >> 16;
+                    pc[2 * c] = __int_as_float(0x4B400000 + lo) - 12582912.f;
+                    pc[2 * c + 1] = __int_as_float(0x4B400000 + hi) - 12582912.f;
+                }
                 const float4* xc = reinterpret_cast<const float4*>(p.x32 + static_cast<size_t>(gls[i]) * G.batch * 8);
 #pragma unroll
                 for (int k = 0; k < KB; ++k) {
                     const int b = bl + BL * k;
                     if (b < G.batch) {
                         const float4 u = __ldg(xc + 2 * b), t = __ldg(xc + 2 * b + 1);
-                        const float xv[8] = {u.x, u.y, u.z, u.w, t.x, t.y, t.z, t.w};
                         float a = acc[k];
-#pragma unroll
-                        for (int c = 0; c < 8; ++c) {
-                            const int v = (c & 1) ? (cw[i][c >> 1] >> 16)
-                                                  : static_cast<int>(static_cast<int16_t>(cw[i][c >> 1] & 0xFFFF));
-                            a = fmaf(static_cast<float>(v), xv[c], a);
-                        }
+                        a = fmaf(pc[0], u.x, a);
+                        a = fmaf(pc[1], u.y, a);
+                        a = fmaf(pc[2], u.z, a);
+                        a = fmaf(pc[3], u.w, a);
+                        a = fmaf(pc[4], t.x, a);
+                        a = fmaf(pc[5], t.y, a);
+                        a = fmaf(pc[6], t.z, a);
+                        a = fmaf(pc[7], t.w, a);
                         acc[k] = a;
                     }
                 }
