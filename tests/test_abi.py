@@ -145,6 +145,23 @@ def test_decode_and_gemv_reject_bad_args(lib):
                                 ctypes.c_void_p(0x100000), need - 1, None) == 4
 
 
+def test_gemv_path_and_error_hooks(lib):
+    """The GEMV main-kernel selector accepts 0..2 only; the error-flag read
+    rejects a null output before touching a device; the GEMV workspace holds
+    the tcgen05 kernel's row-major fp16 activations and its split partial sums
+    (128-row tiles, 64-column K tiles, about 296 units)."""
+    from bit_e8_lattice_b200 import e8q
+
+    assert lib.e8q_set_gemv_path(3) == 1 and lib.e8q_set_gemv_path(-1) == 1
+    assert lib.e8q_set_gemv_path(2) == 0 and lib.e8q_set_gemv_path(0) == 0
+    assert lib.e8q_device_error_flags(0, None) == 1
+    m = e8q.EncodedC(0x100000, 0x100000, 0x100000, None, None, None, None, 0, 0, 4096, 14336, 0, 0, 0)
+    nrt, nkt = 4096 // 128, 14336 // 64
+    nsplit = min(nkt, (296 + nrt - 1) // nrt)
+    need = lib.e8q_gemv_workspace_bytes(ctypes.byref(m), 64)
+    assert need >= 64 * 14336 * 2 + nsplit * 4096 * 64 * 4
+
+
 def test_escape_table_matches_oracle(lib):
     """Every E8 point with |p|^2 <= 22 (1,113,841 points), plus a shell
     beyond: the kernels' lookup table gives the oracle's encoding (core
