@@ -16,7 +16,12 @@
 // Two compute layouts:
 // - rotated basis, bf16(s * p) with one rounding of the exact product: lane
 //   = group, 32 consecutive groups a step, so index reads, map reads and the
-//   16-byte stores are contiguous; few registers, four CTAs an SM;
+//   16-byte stores are contiguous; few registers, four CTAs an SM.  The
+//   staging warp also fills a 32-entry table per row of bf16(s * P / 2) for
+//   P = -16 .. 15 (64 bytes, one word per bank: lookups never conflict), so
+//   a coordinate costs one table read; overflow groups (whose coordinates may
+//   pass that range) are rewritten by the staging warp with the exact
+//   products one iteration later, after the barrier;
 // - original basis: each warp rebuilds one 2048-element window in the
 //   layout of the fast encode's dequant (lane (a, q), row h = group
 //   32 a + 4 h + q) and runs the same register Hadamard
@@ -104,7 +109,8 @@ __device__ __forceinline__ void df_map_overflow(uint16_t* map, uint32_t group, l
 
 // Staging warp: tile t (record ranges rg) into buffer half nb.
 __device__ __forceinline__ void df_stage(const DecodeParams& p, int t, const DfRange& rg, const DfShared& sh, int nb,
-                                         float* rows, float* rowm, long long* o0, float sqb, int lane) {
+                                         float* rows, float* rowm, long long* o0, float sqb, int lane,
+                                         uint16_t (*lut)[32]) {
     const int r0 = t * p.rpt, nr = min(p.rpt, p.rows - r0);
     const int gpr = p.cols >> 3, G = nr * gpr;
     const long long g0 = p.group_base + static_cast<long long>(r0) * gpr;
@@ -130,7 +136,37 @@ __device__ __forceinline__ void df_stage(const DecodeParams& p, int t, const DfR
     for (int j = lane; j < no; j += 32) df_map_overflow(smap, sh.og[j], j, g0, G);
     for (long long o = rg.o0 + no + lane; o < rg.o1; o += 32) df_map_overflow(smap, __ldg(&p.ovf[o].group), o - rg.o0, g0, G);
     for (int j = lane; j < nr; j += 32) rowm[j] = rows[j] / sqb;
+    if (lut) {  // rotated basis: each row's bf16(s * P / 2) for P = lane - 16
+        for (int r = 0; r < nr; ++r)
+            lut[r][lane] = __bfloat16_as_ushort(bf16_of_product(rows[r], 0.5f * static_cast<float>(lane - 16)));
+    }
     if (lane == 0) *o0 = rg.o0;
+}
+
+// Rotated basis, after tile t's compute warps have stored it: its overflow
+// groups (whose coordinates may pass the row tables' range) rewritten with
+// the exact products, from the records and the global scales.
+__device__ __forceinline__ void df_fix_overflow(const DecodeParams& p, int t, const DfRange& rg, int lane) {
+    if (t < 0 || t >= p.n_tiles) return;
+    const int r0 = t * p.rpt, nr = min(p.rpt, p.rows - r0);
+    const int gpr = p.cols >> 3, G = nr * gpr;
+    const long long g0 = p.group_base + static_cast<long long>(r0) * gpr;
+    for (long long o = rg.o0 + lane; o < rg.o1; o += 32) {
+        const e8q_overflow& rec = p.ovf[o];
+        const long long gl = static_cast<long long>(__ldg(&rec.group)) - g0;
+        if (gl < 0 || gl >= G) continue;
+        const int row = static_cast<int>(gl / gpr);
+        const float s = __ldg(p.scale + r0 + row);
+        float v[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[e] = static_cast<float>(rec.coord2[e]);
+        uint4 out;
+        out.x = bf16x2_of_half_products(s, v[0], v[1]);
+        out.y = bf16x2_of_half_products(s, v[2], v[3]);
+        out.z = bf16x2_of_half_products(s, v[4], v[5]);
+        out.w = bf16x2_of_half_products(s, v[6], v[7]);
+        *reinterpret_cast<uint4*>(p.out + static_cast<size_t>(r0) * p.cols + 8 * gl) = out;
+    }
 }
 
 // One group's doubled coordinates from its core index and map entry.
@@ -152,6 +188,7 @@ __global__ void __launch_bounds__(kDfThreads, kOriginal ? kDfCtasOrig : kDfCtasR
     extern __shared__ __align__(16) unsigned char smem[];
     __shared__ float s_rows[2][kMaxTileRows], s_rowm[2][kMaxTileRows];
     __shared__ long long s_o0[2];
+    __shared__ uint16_t s_lut[kOriginal ? 1 : 2][kOriginal ? 1 : kMaxTileRows][32];  // rotated: row tables
     const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
     const bool staging = warp == kDfWarps;
     const DfShared sh = df_shared(smem + (kOriginal ? kDfScratchBytes : 0));
@@ -159,7 +196,7 @@ __global__ void __launch_bounds__(kDfThreads, kOriginal ? kDfCtasOrig : kDfCtasR
     const float sqb = sqrtf(static_cast<float>(1 << p.logb));
     // both maps start empty; afterwards every entry set is cleared by the warp that reads it
     for (int i = tid; i < kDfTileGroups; i += kDfThreads) reinterpret_cast<uint32_t*>(sh.map)[i] = 0u;
-    DfRange next{0, 0, 0, 0};
+    DfRange next{0, 0, 0, 0}, staged1{0, 0, 0, 0}, staged2{0, 0, 0, 0};  // ranges staged 1 and 2 iterations ago
     if (staging) next = df_range(p, blockIdx.x);
     __syncthreads();
 
@@ -171,12 +208,18 @@ __global__ void __launch_bounds__(kDfThreads, kOriginal ? kDfCtasOrig : kDfCtasR
         if (t >= p.n_tiles) break;
         const int tn = t + static_cast<int>(gridDim.x);
         if (staging) {
+            // rotated basis: the tile computed in the previous iteration gets its overflow groups
+            if (!kOriginal) df_fix_overflow(p, t - static_cast<int>(gridDim.x), staged2, lane);
+            DfRange cur{0, 0, 0, 0};
             if (tn < p.n_tiles) {
                 const int nb = (k + 1) & 1;
-                const DfRange cur = next;
+                cur = next;
                 next = df_range(p, tn + static_cast<int>(gridDim.x));
-                df_stage(p, tn, cur, sh, nb, s_rows[nb], s_rowm[nb], &s_o0[nb], sqb, lane);
+                df_stage(p, tn, cur, sh, nb, s_rows[nb], s_rowm[nb], &s_o0[nb], sqb, lane,
+                         kOriginal ? nullptr : s_lut[kOriginal ? 0 : nb]);
             }
+            staged2 = staged1;
+            staged1 = cur;
         } else if (t >= 0) {
             const int b = k & 1;
             const int r0 = t * p.rpt;
@@ -201,14 +244,18 @@ __global__ void __launch_bounds__(kDfThreads, kOriginal ? kDfCtasOrig : kDfCtasR
                     const int g = gw + 32 * j + lane;
                     const unsigned m = tm[g];
                     if (m) tm[g] = 0;
-                    float v[8];
-                    df_point(cw[j], m, p.ovf, o0, v);
-                    const float s = s_rows[b][row];
+                    // core point + root bytewise (|P| <= 8); an overflow group stores the
+                    // core point of index 0 here and is rewritten after the barrier
+                    uint2 add = make_uint2(0, 0);
+                    if (m >= 1 && m <= 240) add = g_root8[m - 1];
+                    const unsigned w0 = __vadd4(cw[j].x, add.x), w1 = __vadd4(cw[j].y, add.y);
+                    const unsigned i0 = (w0 & 0x1F1F1F1Fu) ^ 0x10101010u, i1 = (w1 & 0x1F1F1F1Fu) ^ 0x10101010u;  // P + 16
+                    const uint16_t* lt = s_lut[kOriginal ? 0 : b][row];
                     uint4 o;
-                    o.x = bf16x2_of_half_products(s, v[0], v[1]);
-                    o.y = bf16x2_of_half_products(s, v[2], v[3]);
-                    o.z = bf16x2_of_half_products(s, v[4], v[5]);
-                    o.w = bf16x2_of_half_products(s, v[6], v[7]);
+                    o.x = static_cast<unsigned>(lt[i0 & 0xFFu]) | (static_cast<unsigned>(lt[(i0 >> 8) & 0xFFu]) << 16);
+                    o.y = static_cast<unsigned>(lt[(i0 >> 16) & 0xFFu]) | (static_cast<unsigned>(lt[i0 >> 24]) << 16);
+                    o.z = static_cast<unsigned>(lt[i1 & 0xFFu]) | (static_cast<unsigned>(lt[(i1 >> 8) & 0xFFu]) << 16);
+                    o.w = static_cast<unsigned>(lt[(i1 >> 16) & 0xFFu]) | (static_cast<unsigned>(lt[i1 >> 24]) << 16);
                     *reinterpret_cast<uint4*>(dq + 8 * g) = o;
                     rem += 32;
                     if (rem >= gpr) {
@@ -246,6 +293,13 @@ __global__ void __launch_bounds__(kDfThreads, kOriginal ? kDfCtasOrig : kDfCtasR
             }
         }
         __syncthreads();
+    }
+    // rotated basis: the CTA's last tile gets its overflow groups
+    if (!kOriginal && staging) {
+        const int nt = static_cast<int>(blockIdx.x) < p.n_tiles
+                           ? (p.n_tiles - 1 - static_cast<int>(blockIdx.x)) / static_cast<int>(gridDim.x)
+                           : -1;
+        df_fix_overflow(p, static_cast<int>(blockIdx.x) + nt * static_cast<int>(gridDim.x), staged2, lane);
     }
 }
 
