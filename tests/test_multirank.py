@@ -82,3 +82,79 @@ def test_shard_rows_partition():
             assert all(spans[i][1] == spans[i + 1][0] for i in range(world - 1))
             sizes = [b - a for a, b in spans]
             assert max(sizes) - min(sizes) <= 1
+
+
+def _library_form(out, rows, gpr):
+    """The oracle's encoding in the library's layout: int16 indices, fp32
+    scales, escape / overflow record bytes (group ids from the first row),
+    int64 row pointers."""
+    from bit_e8_lattice_b200.e8q import ESC_DTYPE, OVF_DTYPE
+
+    idx, kind, root, P = out["idx"], out["kind"], out["root"], out["P"]
+    ge, go = np.nonzero(kind == 1)[0], np.nonzero(kind == 2)[0]
+    esc = np.zeros(len(ge), ESC_DTYPE)
+    esc["group"], esc["core"], esc["root"] = ge, idx[ge], root[ge]
+    ovf = np.zeros(len(go), OVF_DTYPE)
+    ovf["group"], ovf["coord2"] = go, P[go]
+    erp = np.concatenate([[0], np.cumsum((kind == 1).reshape(rows, gpr).sum(1))]).astype(np.int64)
+    orp = np.concatenate([[0], np.cumsum((kind == 2).reshape(rows, gpr).sum(1))]).astype(np.int64)
+    return (idx.astype(np.uint16).view(np.int16).reshape(rows, gpr), out["scale"].astype(np.float32),
+            esc.tobytes(), len(ge), ovf.tobytes(), len(go), erp, orp)
+
+
+def _gather_worker(rank, world, port, q):
+    import sys
+
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    import oracle
+    from bit_e8_lattice_b200 import dist as e8dist
+    from bit_e8_lattice_b200 import synth
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        w, d = synth.small_f32()
+        a, b = e8dist.shard_rows(w.shape[0], world, rank)
+        out = oracle.project_encode(w[a:b].astype(np.float64), d, 256, want_x=False, want_margin=False)
+        idx, scale, esc, ne, ovf, no, erp, orp = _library_form(out, b - a, 256 // 8)
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x))
+        esc_t = torch.frombuffer(bytearray(esc + bytes(8)), dtype=torch.uint8)  # room past the records
+        ovf_t = torch.frombuffer(bytearray(ovf + bytes(20)), dtype=torch.uint8)
+        res = e8dist.gather_encoded(t(idx), t(scale), esc_t, ne, ovf_t, no, t(erp), t(orp), a)
+        q.put((rank, [r.numpy().copy() for r in res]))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gather_encoded_row_shards_equal_whole_matrix():
+    """Three gloo ranks with uneven row shards: after gather_encoded every
+    rank holds exactly the whole matrix's encoding (indices, scales, records
+    with group ids from the first row, row pointers)."""
+    import oracle
+    from bit_e8_lattice_b200 import synth
+
+    world = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gather_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    w, d = synth.small_f32()
+    full = oracle.project_encode(w.astype(np.float64), d, 256, want_x=False, want_margin=False)
+    idx, scale, esc, ne, ovf, no, erp, orp = _library_form(full, w.shape[0], 256 // 8)
+    assert ne > 0 and no >= 0
+    for rank, got in results:
+        np.testing.assert_array_equal(got[0], idx)
+        np.testing.assert_array_equal(got[1], scale)
+        assert got[2].tobytes() == esc and got[3].tobytes() == ovf
+        np.testing.assert_array_equal(got[4], erp)
+        np.testing.assert_array_equal(got[5], orp)

@@ -519,3 +519,34 @@ def test_moe_bank_full_size_sampled(e8q):
         out = oracle.project_encode(synth.bf16_bits_to_f64(W[i][rsel]), S[i], oracle.default_block(C))
         check_encode(out, host_idx(res.idx[i]), res.scale[i].cpu().numpy(), esc, ovf, res.group_base[i], rsel, C // 8,
                      label=f"moe[{i}]")
+
+
+def test_gather_encoded_nccl_one_rank(e8q):
+    """gather_encoded on CUDA tensors over NCCL (one rank: the gathered form
+    is the encode's own output, record bytes and row pointers included)."""
+    import socket
+    from datetime import timedelta
+
+    import torch.distributed as dist
+    from bit_e8_lattice_b200 import dist as e8dist
+
+    rng = np.random.default_rng(17)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((96, 2048)) * 0.02)
+    d = synth.signs(17, 2048)
+    enc, res = run_encode(e8q, [w], [d], 0)
+    ctr = res.read_counters()
+    s = socket.socket()
+    s.bind(("127.0.0.1", 0))
+    port = s.getsockname()[1]
+    s.close()
+    dist.init_process_group("nccl", init_method=f"tcp://127.0.0.1:{port}", rank=0, world_size=1,
+                            timeout=timedelta(seconds=60))
+    try:
+        out = e8dist.gather_encoded(res.idx[0], res.scale[0], res.esc, ctr["n_escape"], res.ovf, ctr["n_overflow"],
+                                    res.esc_row_ptr, res.ovf_row_ptr, 0)
+        torch.cuda.synchronize()
+    finally:
+        dist.destroy_process_group()
+    assert torch.equal(out[0], res.idx[0]) and torch.equal(out[1], res.scale[0])
+    assert torch.equal(out[2], res.esc[: 8 * ctr["n_escape"]]) and torch.equal(out[3], res.ovf[: 20 * ctr["n_overflow"]])
+    assert torch.equal(out[4], res.esc_row_ptr) and torch.equal(out[5], res.ovf_row_ptr)
