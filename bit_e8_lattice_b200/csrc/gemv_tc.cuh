@@ -43,8 +43,7 @@ constexpr int kTcRows = 128;   // M: weight rows per tile (tensor-memory lanes)
 constexpr int kTcKCols = 64;   // K columns per stage: 8 groups, 4 MMAs of K = 16
 constexpr int kTcStages = 4;
 constexpr int kTcProdWarps = 16;
-constexpr int kTcMmaWarp = kTcProdWarps;       // warp 16
-constexpr int kTcEpiWarp0 = kTcProdWarps + 1;  // warps 17..20
+constexpr int kTcMmaWarp = kTcProdWarps;                // warp 16; the epilogue warps are 17..20
 constexpr int kTcThreads = (kTcProdWarps + 1 + 4) * 32;
 constexpr int kTcWaitLimit = 1 << 22;
 // batch from which e8q_dequant_gemv picks this kernel by itself: none yet (it
