@@ -37,6 +37,14 @@ def max_over_ranks(value: float, device=None) -> float:
     return float(t.item())
 
 
+def shift_group_ids(words, offset: int):
+    """uint32 group ids held in an int32 tensor, plus offset, modulo 2^32 (as int32)."""
+    import torch
+
+    g = ((words.to(torch.int64) & 0xFFFFFFFF) + int(offset)) & 0xFFFFFFFF
+    return torch.where(g >= (1 << 31), g - (1 << 32), g).to(torch.int32)
+
+
 def gather_encoded(idx, scale, esc, n_esc: int, ovf, n_ovf: int, esc_row_ptr, ovf_row_ptr, row_start: int,
                    group=None):
     """All-gather a row-sharded encoding so that every rank holds the whole
@@ -98,10 +106,9 @@ def gather_encoded(idx, scale, esc, n_esc: int, ovf, n_ovf: int, esc_row_ptr, ov
         off = cnt[r][3] * gpr  # the shard's first group in the whole matrix
         e = esc_parts[r].clone()
         o = ovf_parts[r].clone()
-        for t in (e, o):  # group ids are uint32: shift them by the shard's first group
+        for t in (e, o):
             if t.shape[0]:
-                g = (t[:, 0].to(torch.int64) & 0xFFFFFFFF) + off
-                t[:, 0] = torch.where(g >= (1 << 31), g - (1 << 32), g).to(torch.int32)
+                t[:, 0] = shift_group_ids(t[:, 0], off)
         esc_out.append(e)
         ovf_out.append(o)
         erp_out.append(erp_parts[r][:-1] + e_base)

@@ -158,3 +158,16 @@ def test_gather_encoded_row_shards_equal_whole_matrix():
         assert got[2].tobytes() == esc and got[3].tobytes() == ovf
         np.testing.assert_array_equal(got[4], erp)
         np.testing.assert_array_equal(got[5], orp)
+
+
+def test_shift_group_ids_across_the_sign_bit():
+    """Group ids are uint32 carried in int32 words: shifting them by a shard's
+    first group crosses 2^31 without error and wraps at 2^32."""
+    import torch
+    from bit_e8_lattice_b200.dist import shift_group_ids
+
+    ids = np.array([0, 5, 2**31 - 3, 2**31 + 7, 2**32 - 1], dtype=np.uint64)
+    for off in (0, 1, 10, 2**31, 2**32 - 5):
+        words = torch.from_numpy(ids.astype(np.uint32).view(np.int32))
+        got = shift_group_ids(words, off).numpy().view(np.uint32).astype(np.uint64)
+        np.testing.assert_array_equal(got, (ids + np.uint64(off)) % np.uint64(2**32))
