@@ -85,9 +85,9 @@ e8q_status ensure_device(int* dev_out) {
         if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_gv_main<1, 2>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
         if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<2, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<1, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
         if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<2, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
+            st = cuda_ok(cudaFuncSetAttribute(k_gv_main<1, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
         // prep and finalize leave the SM configured for the main kernel's shared
         // memory, so that its CTAs can start while they are still running
         if (st == E8Q_OK)
@@ -536,11 +536,11 @@ e8q_status e8q_dequant_gemv(const e8q_encoded* m, const void* x_bf16, int32_t ba
     for (int v0 = 0; !tc && v0 < g.nbt; v0 += kGvPassTiles) {
         const int nt = g.nbt - v0 < kGvPassTiles ? g.nbt - v0 : kGvPassTiles;
         mp.v0 = v0;
-        // batch tiles <= 2: one 16-row tile per warp, 16 warps; else two tiles, 8 warps
+        // one 16-row tile per warp, 16 warps (two tiles on 8 warps measured slower at batch 64 and 256)
         if (nt == 1) st = launch_pdl(k_gv_main<1, 1>, grid, 512, kGvSmemBytes, s, mp);
         else if (nt == 2) st = launch_pdl(k_gv_main<1, 2>, grid, 512, kGvSmemBytes, s, mp);
-        else if (nt <= 4) st = launch_pdl(k_gv_main<2, 4>, grid, 256, kGvSmemBytes, s, mp);
-        else st = launch_pdl(k_gv_main<2, 8>, grid, 256, kGvSmemBytes, s, mp);
+        else if (nt <= 4) st = launch_pdl(k_gv_main<1, 4>, grid, 512, kGvSmemBytes, s, mp);
+        else st = launch_pdl(k_gv_main<1, 8>, grid, 512, kGvSmemBytes, s, mp);
         if (st != E8Q_OK) return st;
     }
 

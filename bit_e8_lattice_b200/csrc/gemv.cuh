@@ -20,10 +20,9 @@
 //             rows), fp32 accumulate.  The work -- 256-row blocks times
 //             256-column chunks times 8 k-steps -- is split into equal
 //             contiguous k-step ranges, one per CTA (one resident CTA per
-//             SM); the warps of a CTA (16 with one 16-row tile each for up
-//             to 16 batch rows, else 8 with two) take different rows of the
-//             same range, so they read the same activation fragments (L1
-//             hits).  The first
+//             SM); the 16 warps of a CTA, one 16-row tile each, take
+//             different rows of the same range, so they read the same
+//             activation fragments (L1 hits).  The first
 //             49,152 codeword words live in shared memory (a shared-memory
 //             gather costs a few wavefronts per warp, a global one up to one
 //             per lane); the rest are read through L1.  Indices and root-map
