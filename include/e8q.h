@@ -259,8 +259,11 @@ size_t e8q_gemv_workspace_bytes(const e8q_encoded* m /* host */, int32_t batch);
  * after a per-row power-of-two scaling chosen from the row's largest |x| (no
  * overflow is possible); fp32 accumulation; overflow records use the fp32
  * values; bf16 output (round to nearest even).  Expected relative error
- * about 1e-4 of the output norm.  Asynchronous on `stream`; errors:
- * INVALID_ARG, UNSUPPORTED (cols > 16384), WORKSPACE, CUDA.
+ * about 1e-4 of the output norm.  The product runs on mma.sync fragments
+ * (the default) or on tcgen05 with the accumulator in tensor memory
+ * (e8q_set_gemv_path); both give these sums up to fp32 summation order.
+ * Asynchronous on `stream`; errors: INVALID_ARG, UNSUPPORTED (cols > 16384),
+ * WORKSPACE, CUDA.
  */
 e8q_status e8q_dequant_gemv(const e8q_encoded* m /* host */, const void* x_bf16, int32_t batch, void* y_bf16,
                             void* ws, size_t ws_bytes, e8q_stream stream);
