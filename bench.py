@@ -223,6 +223,8 @@ def main():
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one captured graph")
+    ap.add_argument("--gemv-path", choices=["auto", "mma_sync", "tcgen05"], default="auto",
+                    help="GEMV main kernel (auto: the library's choice)")
     args = ap.parse_args()
     batches = [int(b) for b in args.batches.split(",") if b]
     if args.impl == "reference":
@@ -244,6 +246,7 @@ def main():
     from bit_e8_lattice_b200 import e8q
 
     e8q.init()
+    e8q.set_gemv_path(args.gemv_path)
     data = host_data(batches)
     (up, d_up), (down, d_dn), xs = data
 
@@ -461,7 +464,8 @@ def main():
             "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "groups_per_step_per_gpu": G, "kappa": 1.0, "rht_block": 2048,
-                       "gemv_batches": batches, "l2": "inputs larger than L2: 235 MB of latent weights read per step",
+                       "gemv_batches": batches, "gemv_main_kernel": args.gemv_path,
+                       "l2": "inputs larger than L2: 235 MB of latent weights read per step",
                        "escape_fraction": n_esc / G, "overflow_fraction": n_ovf / G,
                        "payload_bits_pages_formula": 2 + 20 * (n_esc + n_ovf) / G,
                        "parallelism": f"replicas x{world} (rows are independent; no collective)"},
