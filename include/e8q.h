@@ -68,7 +68,7 @@ typedef struct CUstream_st* e8q_stream;
 typedef enum {
     E8Q_OK = 0,
     E8Q_ERR_INVALID_ARG = 1, /* bad pointer, size, alignment or enum */
-    E8Q_ERR_UNSUPPORTED = 2, /* valid but outside this build's limits */
+    E8Q_ERR_UNSUPPORTED = 2, /* valid but outside the library's limits */
     E8Q_ERR_CUDA = 3,        /* a CUDA call or launch failed */
     E8Q_ERR_WORKSPACE = 4,   /* workspace missing or too small */
     E8Q_ERR_SCRATCH_LIMIT = 5 /* larger than e8q_project_encode_noalloc's built-in scratch */

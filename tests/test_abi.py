@@ -80,7 +80,7 @@ def _args(**kw):
 
 @pytest.mark.parametrize("kw,expect", [
     (dict(cols=12), 1),            # not a multiple of 8
-    (dict(cols=16392), 2),         # wider than this build handles
+    (dict(cols=16392), 2),         # wider than the library handles
     (dict(block=3), 1),            # not a power of two
     (dict(block=4096), 1),         # larger than 2048
     (dict(cols=96, block=64), 1),  # does not divide cols
