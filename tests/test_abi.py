@@ -183,3 +183,25 @@ def test_escape_table_matches_oracle(lib):
     bad = np.nonzero(words != expect)[0]
     assert len(bad) == 0, (len(bad), P[bad[:3]], words[bad[:3]], expect[bad[:3]])
     assert (kind[-len(far[::7]):] == 2).all()
+
+
+def test_bench_source_hash_ignores_comments_only(tmp_path, monkeypatch):
+    """bench.py matches a committed ncu summary to the kernels by a hash of
+    the kernel sources without comments and blank space: a comment edit keeps
+    the hash, a code edit changes it."""
+    import shutil
+    import sys
+
+    sys.path.insert(0, ROOT)
+    import bench
+
+    src = os.path.join(ROOT, "bit_e8_lattice_b200", "csrc")
+    dst = tmp_path / "bit_e8_lattice_b200" / "csrc"
+    shutil.copytree(src, dst)
+    monkeypatch.setattr(bench, "ROOT", str(tmp_path))
+    base = bench.source_sha()
+    f = dst / "ptx.cuh"
+    f.write_text(f.read_text() + "\n// a comment\n/* and\n another */\n\n")
+    assert bench.source_sha() == base
+    f.write_text(f.read_text() + "\nnamespace e8q { constexpr int kProbe = 1; }\n")
+    assert bench.source_sha() != base
