@@ -7,12 +7,16 @@ One step = one pass of the whole path over the dense-MLP workload
      sign flip, blockwise RHT (B = 2048), row scale, E8 projection, core
      index, ordered escape / overflow records with CSR, and the
      original-basis bf16 dequantised weights (identity-STE forward);
-  2. STE backward: the upstream gradient is passed to the latents as is
-     (an alias, no kernel);
+  2. STE backward: e8q_ste_backward hands the seeded N(0, 1e-3^2) bf16
+     gradient of both matrices to the latents as the same tensors (the
+     identity, aliased: nothing moves; the copying form is timed apart);
   3. decode: e8q_dequant_gemv of the encoded up matrix at batch 1, 4, 16
      and 64 (bf16 activations N(0, 1)).
 value = groups encoded per second over whole steps (Ggroups/s, all ranks).
-Inputs are larger than L2 (235 MB read per step), so no flush is needed.
+The step's inputs are larger than L2 (235 MB read per step), so the step
+needs no flush.  The per-kernel GEMV, decode and small-workload figures in
+"kernels" are medians of 20 calls, each after a 256 MB write that flushes
+L2.
 
 --impl reference runs the fp64 CPU oracle on a bounded sample of the same
 step on the host cores (rank 0 only).
@@ -21,9 +25,9 @@ from __future__ import annotations
 
 import argparse
 import hashlib
-import re
 import json
 import os
+import re
 import statistics
 import sys
 import threading
@@ -37,10 +41,14 @@ import numpy as np  # noqa: E402
 METRIC = "E8 project+encode Ggroups/s and dequant-GEMV GB/s, % of B200 HBM peak"
 UNIT = "Ggroups/s"
 WORKLOAD = ("mlp_14336 QAT step: project+encode+STE-dequant of up 4096x14336 and down 14336x4096 bf16 "
-            "(one launch), identity-STE backward, then 2-bit dequant-GEMV of up at batch 1,4,16,64")
+            "(one launch), identity-STE backward of the seeded gradient, then 2-bit dequant-GEMV of up at "
+            "batch 1,4,16,64")
 D_MODEL, D_FF = 4096, 14336
 NOMINAL_HBM_GBS = 8000.0
 CSRC = os.path.join("bit_e8_lattice_b200", "csrc")
+FLUSH_BYTES = 256 << 20
+KERNEL_REPS = 20
+SAMPLE_UP, SAMPLE_DN = 2, 7  # oracle sample rows per step (1 : 3.5, the workload's proportion)
 
 
 def source_sha() -> str:
@@ -83,6 +91,23 @@ def profile_traffic(kernel: str):
         return float(vals["traffic_bytes_per_launch"])
     except (KeyError, ValueError):
         return None
+
+
+def host_cpu():
+    """(threads usable by this process, CPU model name)."""
+    try:
+        n = len(os.sched_getaffinity(0))
+    except AttributeError:
+        n = os.cpu_count() or 1
+    model = "unknown"
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except OSError:
+        pass
+    return n, model
 
 
 class ClockSampler:
@@ -142,37 +167,118 @@ class ClockSampler:
 # --------------------------------------------------------------------------
 # CPU oracle sample (reference arm and cpu_baseline)
 # --------------------------------------------------------------------------
-def oracle_sample_step(data, batches, k):
-    """One bounded sample of the step on the host: rows of up and down
-    (in the workload's 1 : 3.5 proportion), projected, encoded and
-    dequantised to the original basis; the sampled up rows' GEMV outputs at
-    every batch.  Returns the number of groups processed."""
+def oracle_rows(up_rows, d_up, dn_rows, d_dn, xs):
+    """The step's arithmetic on sampled rows, on the host with the fp64
+    oracle: rows of up and down projected, encoded and dequantised to the
+    original basis; the sampled up rows' GEMV outputs at every batch.
+    Returns the number of groups processed.  (Top level, so that a spawned
+    worker process can run it.)"""
     import oracle
     from bit_e8_lattice_b200 import synth
 
-    (up, d_up), (down, d_dn), xs = data
-    n_up, n_dn = 2, 7
-    ru = [(k * n_up + i) % D_MODEL for i in range(n_up)]
-    rd = [(k * n_dn + i) % D_FF for i in range(n_dn)]
-    out_u = oracle.project_encode(synth.bf16_bits_to_f64(up[ru]), d_up, 2048, want_x=False, want_margin=False)
-    out_d = oracle.project_encode(synth.bf16_bits_to_f64(down[rd]), d_dn, 2048, want_x=False, want_margin=False)
+    out_u = oracle.project_encode(synth.bf16_bits_to_f64(up_rows), d_up, 2048, want_x=False, want_margin=False)
+    out_d = oracle.project_encode(synth.bf16_bits_to_f64(dn_rows), d_dn, 2048, want_x=False, want_margin=False)
     oracle.dequant(out_u["P"], out_u["scale"], d_up, 2048, "original")
     oracle.dequant(out_d["P"], out_d["scale"], d_dn, 2048, "original")
-    for b in batches:
-        oracle.gemv(out_u["P"], out_u["scale"], d_up, 2048, synth.bf16_bits_to_f64(xs[b]))
-    return n_up * (D_FF // 8) + n_dn * (D_MODEL // 8)
+    for x in xs:
+        oracle.gemv(out_u["P"], out_u["scale"], d_up, 2048, synth.bf16_bits_to_f64(x))
+    return up_rows.shape[0] * (up_rows.shape[1] // 8) + dn_rows.shape[0] * (dn_rows.shape[1] // 8)
 
 
-def cpu_oracle_rate(data, batches, seconds: float = 10.0):
-    t0 = time.perf_counter()
-    groups, k = 0, 0
-    while True:
-        groups += oracle_sample_step(data, batches, k)
-        k += 1
-        el = time.perf_counter() - t0
-        if el >= seconds:
-            break
-    return groups / el / 1e9, el, k
+def sample_task(data, k):
+    """Arguments of oracle_rows for the k-th bounded sample of the step."""
+    (up, d_up), (down, d_dn), xs = data
+    ru = [(k * SAMPLE_UP + i) % D_MODEL for i in range(SAMPLE_UP)]
+    rd = [(k * SAMPLE_DN + i) % D_FF for i in range(SAMPLE_DN)]
+    return (np.ascontiguousarray(up[ru]), d_up, np.ascontiguousarray(down[rd]), d_dn, [xs[b] for b in sorted(xs)])
+
+
+def _pool_worker(args):
+    return oracle_rows(*args)
+
+
+def cpu_oracle_rates(data, seconds: float):
+    """The oracle as it stands on bounded samples of the step: one thread,
+    then one spawned worker process per usable host thread over independent
+    samples (rows are independent).  Returns a cpu_baseline dict."""
+    import concurrent.futures as cf
+    import multiprocessing as mp
+
+    from threadpoolctl import threadpool_limits
+
+    n_threads, model = host_cpu()
+    with threadpool_limits(limits=1):  # the dense GEMV step's BLAS on one thread too
+        t0 = time.perf_counter()
+        groups, k = 0, 0
+        while time.perf_counter() - t0 < seconds:
+            groups += oracle_rows(*sample_task(data, k))
+            k += 1
+        el1 = time.perf_counter() - t0
+    rate1 = groups / el1 / 1e9
+    out = {"value": rate1, "unit": UNIT, "cores": 1, "kind": "oracle",
+           "sample": f"{k} samples of {SAMPLE_UP} up rows + {SAMPLE_DN} down rows "
+                     f"({SAMPLE_UP * D_FF // 8 + SAMPLE_DN * D_MODEL // 8} groups each) incl. original-basis dequant "
+                     f"and the sampled rows' GEMV at every batch, {el1:.1f} s, single thread",
+           "cpu_model": model, "host_threads": n_threads}
+    if n_threads > 1:
+        ctx = mp.get_context("spawn")
+        # one BLAS thread in each worker (set before the workers import numpy)
+        saved = {v: os.environ.get(v) for v in ("OMP_NUM_THREADS", "OPENBLAS_NUM_THREADS", "MKL_NUM_THREADS")}
+        os.environ.update({v: "1" for v in saved})
+        try:
+            ex = cf.ProcessPoolExecutor(max_workers=n_threads, mp_context=ctx)
+        finally:
+            for v, old in saved.items():
+                if old is None:
+                    os.environ.pop(v, None)
+                else:
+                    os.environ[v] = old
+        with ex:
+            list(ex.map(_pool_worker, [sample_task(data, j) for j in range(n_threads)]))  # start-up, imports
+            t0 = time.perf_counter()
+            gm, j = 0, 0
+            while time.perf_counter() - t0 < seconds:
+                tasks = [sample_task(data, k + j + i) for i in range(n_threads)]
+                gm += sum(ex.map(_pool_worker, tasks))
+                j += n_threads
+            elm = time.perf_counter() - t0
+        out["all_cores"] = {"value": gm / elm / 1e9, "unit": UNIT, "cores": n_threads,
+                            "sample": f"{j} samples over {n_threads} spawned processes, {elm:.1f} s"}
+    return out
+
+
+def oracle_parity_sample(res, data, rows_up, rows_dn):
+    """Near-tie count and agreement of the timed encode with the oracle on
+    sampled rows (part of the cpu_baseline leg: the only use of the oracle
+    on the measured path)."""
+    import oracle
+    from bit_e8_lattice_b200 import synth
+
+    (up, d_up), (down, d_dn), _ = data
+    esc, ovf = res.escape_records(), res.overflow_records()
+    erp, orp = res.esc_row_ptr.cpu().numpy(), res.ovf_row_ptr.cpu().numpy()
+    core, roots = oracle.core_points().astype(np.int32), oracle.roots().astype(np.int32)
+    tot = dict(groups=0, near_ties=0, mismatches_above_margin=0, rows=0)
+    for m, (bits, d, rows) in enumerate([(up, d_up, rows_up), (down, d_dn, rows_dn)]):
+        C = bits.shape[1]
+        gpr = C // 8
+        idx = res.idx[m].cpu().numpy().view(np.uint16)
+        out = oracle.project_encode(synth.bf16_bits_to_f64(bits[rows]), d, 2048, want_x=False)
+        for j, r in enumerate(rows):
+            grow = res.row_base[m] + r
+            P = core[idx[r].astype(np.int64)]
+            e = esc[erp[grow]:erp[grow + 1]]
+            o = ovf[orp[grow]:orp[grow + 1]]
+            g0 = res.group_base[m] + r * gpr
+            P[e["group"].astype(np.int64) - g0] += roots[e["root"].astype(np.int64)]
+            P[o["group"].astype(np.int64) - g0] = o["coord2"].astype(np.int32)
+            sl = slice(j * gpr, (j + 1) * gpr)
+            far = out["margin"][sl] > 1e-4
+            tot["groups"] += gpr
+            tot["near_ties"] += int((~far).sum())
+            tot["mismatches_above_margin"] += int(((P != out["P"][sl]).any(1) & far).sum())
+            tot["rows"] += 1
+    return tot
 
 
 def host_data(batches):
@@ -190,26 +296,86 @@ def run_reference(args, batches):
         return 0
     data = host_data(batches)
     for k in range(args.warmup):
-        oracle_sample_step(data, batches, k)
+        oracle_rows(*sample_task(data, k))
     times, groups = [], 0
     for k in range(args.steps):
         t0 = time.perf_counter()
-        groups += oracle_sample_step(data, batches, args.warmup + k)
+        groups += oracle_rows(*sample_task(data, args.warmup + k))
         times.append(time.perf_counter() - t0)
     total = sum(times)
     value = groups / total / 1e9
+    _, model = host_cpu()
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-        "config": {"workload": WORKLOAD, "sample": "2 rows of up + 7 rows of down per step, all four GEMV batches "
-                                                   "on the sampled up rows"},
-        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle",
-                         "sample": "2 up rows + 7 down rows per step (9,760 groups)"},
+        "config": {"workload": WORKLOAD, "sample": f"{SAMPLE_UP} rows of up + {SAMPLE_DN} rows of down per step, "
+                                                   "all four GEMV batches on the sampled up rows"},
+        "cpu_baseline": {"value": value, "unit": UNIT, "cores": 1, "kind": "oracle", "cpu_model": model,
+                         "sample": f"{SAMPLE_UP} up rows + {SAMPLE_DN} down rows per step "
+                                   f"({SAMPLE_UP * D_FF // 8 + SAMPLE_DN * D_MODEL // 8} groups)"},
         "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
     return 0
+
+
+# --------------------------------------------------------------------------
+# device timing helpers
+# --------------------------------------------------------------------------
+def time_flushed(fn, stream, flush, reps: int = KERNEL_REPS):
+    """Median and mean device time (ms) of fn() over `reps` calls, each
+    after a write of `flush` (larger than L2), captured as one CUDA graph
+    with a timing event on each side of every call (eager launches if the
+    capture is refused)."""
+    import torch
+
+    def record(ev):
+        for a, b in ev:
+            flush.zero_()
+            a.record()
+            fn()
+            b.record()
+
+    try:
+        ev = [(torch.cuda.Event(enable_timing=True, external=True), torch.cuda.Event(enable_timing=True, external=True))
+              for _ in range(reps)]
+        g = torch.cuda.CUDAGraph()
+        cap = torch.cuda.Stream()
+        cap.wait_stream(stream)
+        with torch.cuda.graph(g, stream=cap):
+            record(ev)
+        stream.wait_stream(cap)
+        g.replay()
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        del g
+    except Exception:
+        torch.cuda.synchronize()
+        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(reps)]
+        record(ev)
+        torch.cuda.synchronize()
+        record(ev)
+        torch.cuda.synchronize()
+    ms = [a.elapsed_time(b) for a, b in ev]
+    return statistics.median(ms), statistics.mean(ms)
+
+
+def kernel_entry(bytes_per_call, ms_median, ms_mean, peaks, groups=None, note=None):
+    gbs = bytes_per_call / (ms_median * 1e-3) / 1e9
+    e = {"launch_us": 1e3 * ms_median, "launch_us_mean": 1e3 * ms_mean, "GB_s": gbs,
+         "frac_measured_hbm": gbs / peaks["hbm_gbs"], "frac_nominal_8TBs": gbs / NOMINAL_HBM_GBS,
+         "bytes_per_launch": bytes_per_call, "timing": f"median of {KERNEL_REPS}, L2 flushed before each call"}
+    if groups is not None:
+        e["Ggroups_s"] = groups / (ms_median * 1e-3) / 1e9
+    if note:
+        e["note"] = note
+    return e
+
+
+def record_bytes(rp, lo, hi):
+    return int(rp[hi] - rp[lo])
 
 
 def main():
@@ -222,6 +388,8 @@ def main():
     ap.add_argument("--e2e-steps", type=int, default=10)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-workloads", action="store_true",
+                    help="skip the attention-projection and expert-bank encode timings")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one captured graph")
     ap.add_argument("--gemv-path", choices=["auto", "mma_sync", "tcgen05"], default="auto",
                     help="GEMV main kernel (auto: the library's choice)")
@@ -243,7 +411,7 @@ def main():
     torch.cuda.set_device(local)
     dev = torch.device("cuda", local)
 
-    from bit_e8_lattice_b200 import e8q
+    from bit_e8_lattice_b200 import e8q, synth
 
     e8q.init()
     e8q.set_gemv_path(args.gemv_path)
@@ -257,7 +425,8 @@ def main():
     W = [t_bf16(up), t_bf16(down)]
     S = [torch.from_numpy(d_up).to(dev), torch.from_numpy(d_dn).to(dev)]
     X = {b: t_bf16(xs[b]) for b in batches}
-    grad = torch.from_numpy(np.zeros(1, np.int16)).to(dev)  # identity STE: the gradient is aliased, never touched
+    # upstream gradient of the step (seeded N(0, 1e-3^2) bf16), resident
+    GRAD = [t_bf16(synth.mlp_grad((D_MODEL, D_FF), matrix=0)), t_bf16(synth.mlp_grad((D_FF, D_MODEL), matrix=1))]
     G = D_MODEL * (D_FF // 8) + D_FF * (D_MODEL // 8)
     enc = e8q.Encoder([(D_MODEL, D_FF), (D_FF, D_MODEL)], S, torch.bfloat16, 0, 1.0, "original",
                       esc_cap=G // 2, ovf_cap=G // 16)
@@ -265,8 +434,13 @@ def main():
     gemvs = {b: e8q.Gemv(res.encoded[0], b) for b in batches}
     stream = torch.cuda.current_stream()
 
+    def ste_backward():
+        # identity STE: the latents' gradient is the dequantised weights' gradient, aliased
+        return [e8q.e8q_ste_backward(g) for g in GRAD]
+
     def step():
         enc(W)
+        ste_backward()
         for b in batches:
             gemvs[b](X[b])
 
@@ -289,6 +463,7 @@ def main():
             ev[k][0].record()
             enc(W)
             ev[k][1].record()
+            ste_backward()
             for j, b in enumerate(batches):
                 gemvs[b](X[b])
                 ev[k][2 + j].record()
@@ -336,6 +511,8 @@ def main():
 
     enc_ms = [ev[k][0].elapsed_time(ev[k][1]) for k in range(K)]
     gem_ms = {b: [ev[k][1 + j].elapsed_time(ev[k][2 + j]) for k in range(K)] for j, b in enumerate(batches)}
+    if graph is not None:
+        del graph
     ctr = res.read_counters()
     n_esc, n_ovf = ctr["n_escape"], ctr["n_overflow"]
     rows = D_MODEL + D_FF
@@ -344,42 +521,86 @@ def main():
     peaks = measured_peaks()
     enc_gbs = enc_bytes / (enc_avg * 1e-3) / 1e9
 
-    # GEMV algorithmic bytes: indices, the up matrix's records, scales, x, y
+    # ---------------------------------------------------------- per kernel
+    flush = torch.empty(FLUSH_BYTES // 4, dtype=torch.float32, device=dev)
     up_groups = D_MODEL * (D_FF // 8)
     rp = res.esc_row_ptr.cpu().numpy()
     op = res.ovf_row_ptr.cpu().numpy()
-    up_esc, up_ovf = int(rp[D_MODEL] - rp[0]), int(op[D_MODEL] - op[0])
+    up_esc, up_ovf = record_bytes(rp, 0, D_MODEL), record_bytes(op, 0, D_MODEL)
     kernels = {"project_encode": {
-        "launch_us": 1e3 * enc_avg, "Ggroups_s": G / (enc_avg * 1e-3) / 1e9, "GB_s": enc_gbs,
+        "launch_us": 1e3 * enc_avg, "launch_us_median": 1e3 * statistics.median(enc_ms),
+        "Ggroups_s": G / (enc_avg * 1e-3) / 1e9, "GB_s": enc_gbs,
         "frac_measured_hbm": enc_gbs / peaks["hbm_gbs"], "frac_nominal_8TBs": enc_gbs / NOMINAL_HBM_GBS,
-        "bytes_per_launch": enc_bytes}}
+        "bytes_per_launch": enc_bytes, "timing": f"mean over the {K} timed steps (inputs larger than L2)"}}
     for b in batches:
         gb_bytes = 2 * up_groups + 8 * up_esc + 20 * up_ovf + 4 * D_MODEL + 16 * (D_MODEL + 1) + 2 * b * (D_FF + D_MODEL)
-        avg = statistics.mean(gem_ms[b])
-        gbs = gb_bytes / (avg * 1e-3) / 1e9
-        kernels[f"dequant_gemv_b{b}"] = {"launch_us": 1e3 * avg, "GB_s": gbs,
-                                         "frac_measured_hbm": gbs / peaks["hbm_gbs"],
-                                         "frac_nominal_8TBs": gbs / NOMINAL_HBM_GBS, "bytes_per_launch": gb_bytes}
+        med, mean = time_flushed(lambda b=b: gemvs[b](X[b]), stream, flush)
+        e = kernel_entry(gb_bytes, med, mean, peaks)
+        e["in_step_us_mean"] = 1e3 * statistics.mean(gem_ms[b])
+        kernels[f"dequant_gemv_b{b}"] = e
 
-    # decode of the encoded up matrix (not part of the QAT step, timed on its
-    # own): indices, records, scales and row pointers in, bf16 weights out
+    # decode of the encoded up matrix: indices, records, scales and row
+    # pointers in, bf16 weights out
     dq_out = torch.empty((D_MODEL, D_FF), dtype=torch.bfloat16, device=dev)
     dec_bytes = 2 * up_groups + 8 * up_esc + 20 * up_ovf + 4 * D_MODEL + 16 * (D_MODEL + 1) + 16 * up_groups
     for basis in ("rotated", "original"):
-        for _ in range(3):
-            e8q.e8q_decode(res.encoded[0], basis, dq_out)
+        med, mean = time_flushed(lambda basis=basis: e8q.e8q_decode(res.encoded[0], basis, dq_out), stream, flush)
+        kernels[f"decode_{basis}"] = kernel_entry(dec_bytes, med, mean, peaks, groups=up_groups)
+
+    # identity-STE backward in its copying form (grad_latent a separate buffer)
+    gl = [torch.empty_like(g) for g in GRAD]
+    med, mean = time_flushed(lambda: [e8q.e8q_ste_backward(g, o) for g, o in zip(GRAD, gl)], stream, flush)
+    ste_copy = kernel_entry(32 * G, med, mean, peaks, groups=G,
+                            note="both matrices' gradients copied: 16 B read + 16 B written per group")
+    kernels["ste_backward_copy"] = ste_copy
+    del gl
+
+    # the other seeded workloads: the 2048^2 attention projection (fits in
+    # L2: flushed before each call) and the 128-expert bank (one batched
+    # launch over 384 matrices, 1.2 GB of inputs)
+    workloads = {}
+    if not args.no_workloads:
+        aw, ad = synth.attn_2048()
+        aenc = e8q.Encoder([aw.shape], [torch.from_numpy(ad).to(dev)], torch.bfloat16, 0, 1.0, "none",
+                           esc_cap=aw.size // 8, ovf_cap=aw.size // 16)
+        AW = [t_bf16(aw)]
+        ares = aenc(AW)
         torch.cuda.synchronize()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        n_dec = 20
-        e0.record()
-        for _ in range(n_dec):
-            e8q.e8q_decode(res.encoded[0], basis, dq_out)
-        e1.record()
+        ac = ares.read_counters()
+        ag = aw.size // 8
+        med, mean = time_flushed(lambda: aenc(AW), stream, flush)
+        abytes = ag * 18 + aw.shape[0] * (4 + 16) + 8 * ac["n_escape"] + 20 * ac["n_overflow"]
+        kernels["attn_2048_project_encode"] = kernel_entry(abytes, med, mean, peaks, groups=ag)
+        adq = torch.empty(aw.shape, dtype=torch.bfloat16, device=dev)
+        med, mean = time_flushed(lambda: e8q.e8q_decode(ares.encoded[0], "original", adq), stream, flush)
+        dbytes = ag * 18 + aw.shape[0] * (4 + 16) + 8 * ac["n_escape"] + 20 * ac["n_overflow"]
+        kernels["attn_2048_decode_original"] = kernel_entry(dbytes, med, mean, peaks, groups=ag)
+        workloads["attn_2048"] = {"groups": ag, "escape_fraction": ac["n_escape"] / ag,
+                                  "overflow_fraction": ac["n_overflow"] / ag}
+        del aenc, ares, AW, adq
+
+        bank = synth.moe_bank()
+        shapes = [m.shape for m, _ in bank]
+        MW = [t_bf16(m) for m, _ in bank]
+        MS = [torch.from_numpy(d).to(dev) for _, d in bank]
+        mg = sum(r * (c // 8) for r, c in shapes)
+        menc = e8q.Encoder(shapes, MS, torch.bfloat16, 0, 1.0, "none", esc_cap=mg // 2, ovf_cap=mg // 16)
+        mres = menc(MW)
         torch.cuda.synchronize()
-        avg = e0.elapsed_time(e1) / n_dec
-        gbs = dec_bytes / (avg * 1e-3) / 1e9
-        kernels[f"decode_{basis}"] = {"launch_us": 1e3 * avg, "GB_s": gbs, "frac_measured_hbm": gbs / peaks["hbm_gbs"],
-                                      "frac_nominal_8TBs": gbs / NOMINAL_HBM_GBS, "bytes_per_launch": dec_bytes}
+        mc = mres.read_counters()
+        if mc["n_dropped"] or mc["err"]:
+            raise RuntimeError(f"expert-bank encode capacity or ordering problem: {mc}")
+        med, mean = time_flushed(lambda: menc(MW), stream, flush, reps=5)
+        mrows = sum(r for r, _ in shapes)
+        mbytes = mg * 18 + mrows * (4 + 16) + 8 * mc["n_escape"] + 20 * mc["n_overflow"]
+        e = kernel_entry(mbytes, med, mean, peaks, groups=mg, note="one launch over all 384 matrices")
+        e["timing"] = "median of 5, L2 flushed before each call (1.2 GB of inputs)"
+        kernels["moe_bank_project_encode"] = e
+        workloads["moe_bank"] = {"groups": mg, "matrices": len(shapes), "escape_fraction": mc["n_escape"] / mg,
+                                 "overflow_fraction": mc["n_overflow"] / mg}
+        del menc, mres, MW, MS, bank
+    del flush
+    torch.cuda.empty_cache()
 
     # end to end through the public API: pinned host inputs in, results out
     e2e = None
@@ -416,6 +637,7 @@ def main():
             cs.wait_event(ev_out)
             with torch.cuda.stream(cs):
                 r = enc(Wd[j])
+                ste_backward()
                 ys = {b: gemvs[b](Xd[j][b]) for b in batches}
             ev_used[j].record(cs)
             with torch.cuda.stream(ps):
@@ -448,12 +670,16 @@ def main():
         e2e = {"value": world * G * args.e2e_steps / (ems * 1e-3) / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
                "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
 
-    cpu = None
+    # cpu_baseline leg: the oracle timed on the host cores, and the near-tie
+    # count / agreement of the timed encode on sampled rows
+    cpu, psample = None, None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        rate, el, nsamp = cpu_oracle_rate(data, batches, args.cpu_seconds)
-        cpu = {"value": rate, "unit": UNIT, "cores": 1, "kind": "oracle",
-               "sample": f"{nsamp} samples of 2 up rows + 7 down rows (9,760 groups each) incl. dequant and GEMV "
-                         f"rows, {el:.1f} s"}
+        enc(W)
+        torch.cuda.synchronize()
+        rs = np.random.default_rng(7)
+        psample = oracle_parity_sample(res, data, np.sort(rs.choice(D_MODEL, 8, replace=False)),
+                                       np.sort(rs.choice(D_FF, 28, replace=False)))
+        cpu = cpu_oracle_rates(data, args.cpu_seconds)
 
     if world > 1:
         dist.barrier()
@@ -465,9 +691,15 @@ def main():
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "groups_per_step_per_gpu": G, "kappa": 1.0, "rht_block": 2048,
                        "gemv_batches": batches, "gemv_main_kernel": args.gemv_path,
-                       "l2": "inputs larger than L2: 235 MB of latent weights read per step",
+                       "l2": "step: inputs larger than L2 (235 MB of latent weights read per step); "
+                             "kernels: L2 flushed by a 256 MB write before each timed call",
                        "escape_fraction": n_esc / G, "overflow_fraction": n_ovf / G,
                        "payload_bits_pages_formula": 2 + 20 * (n_esc + n_ovf) / G,
+                       "near_tie_sample": psample,
+                       "ste_backward": {"form": "aliased (identity)", "bytes_per_group_aliased": 0,
+                                        "bytes_per_group_copied": 32,
+                                        "copy_us": ste_copy["launch_us"], "copy_GB_s": ste_copy["GB_s"]},
+                       "other_workloads": workloads,
                        "parallelism": f"replicas x{world} (rows are independent; no collective)"},
             "roofline": {"bound": "hbm", "kernel": "k_encode_fast", "achieved": enc_gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": enc_gbs / peaks["hbm_gbs"], "traffic": traffic,
@@ -475,7 +707,8 @@ def main():
             "kernels": kernels,
             "cpu_baseline": cpu,
             "e2e": e2e,
-            "gpu_launches": K * (1 + 2 * len(batches)),
+            # per step: the encode kernel, and prep + main + finalize for each GEMV call
+            "gpu_launches": K * (1 + 3 * len(batches)),
             "timing": mode,
             "clocks": clocks.summary(),
         }

@@ -15,6 +15,7 @@
 #include "encode_fast.cuh"
 #include "gemv.cuh"
 #include "gemv_tc.cuh"
+#include "ste.cuh"
 #include "tables.h"
 
 namespace e8q {
@@ -564,6 +565,36 @@ e8q_status e8q_dequant_gemv(const e8q_encoded* m, const void* x_bf16, int32_t ba
     if (kb == 2) return launch_pdl(k_gv_fin<2>, fgrid, 256, 0, s, fp);
     if (kb <= 4) return launch_pdl(k_gv_fin<4>, fgrid, 256, 0, s, fp);
     return launch_pdl(k_gv_fin<8>, fgrid, 256, 0, s, fp);
+}
+
+e8q_status e8q_ste_backward(const void* grad_dequant, void* grad_latent, int64_t n, e8q_stream stream) {
+    if (n < 0) return E8Q_ERR_INVALID_ARG;
+    if (n == 0) return E8Q_OK;
+    if (!grad_dequant || !grad_latent || !aligned(grad_dequant, 2) || !aligned(grad_latent, 2))
+        return E8Q_ERR_INVALID_ARG;
+    if (grad_dequant == grad_latent) return E8Q_OK;  // the identity, aliased: nothing to move
+    const uintptr_t a = reinterpret_cast<uintptr_t>(grad_dequant), b = reinterpret_cast<uintptr_t>(grad_latent);
+    const uintptr_t bytes = static_cast<uintptr_t>(n) * 2;
+    if (a < b + bytes && b < a + bytes) return E8Q_ERR_INVALID_ARG;  // partial overlap
+    int dev;
+    e8q_status st = ensure_device(&dev);
+    if (st != E8Q_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    const int grid = 4 * g_sms[dev];  // persistent grid: 4 CTAs of 512 threads an SM
+    if (aligned(grad_dequant, 16) && aligned(grad_latent, 16)) {
+        const long long n16 = n / 8;
+        if (n16 > 0)
+            k_ste_copy16<<<grid, kSteThreads, 0, s>>>(static_cast<const uint4*>(grad_dequant),
+                                                      static_cast<uint4*>(grad_latent), n16);
+        const long long tail = n - 8 * n16;
+        if (tail > 0)
+            k_ste_copy2<<<1, kSteThreads, 0, s>>>(static_cast<const uint16_t*>(grad_dequant) + 8 * n16,
+                                                  static_cast<uint16_t*>(grad_latent) + 8 * n16, tail);
+    } else {
+        k_ste_copy2<<<grid, kSteThreads, 0, s>>>(static_cast<const uint16_t*>(grad_dequant),
+                                                 static_cast<uint16_t*>(grad_latent), n);
+    }
+    return cuda_ok(cudaGetLastError());
 }
 
 }  // extern "C"

@@ -83,6 +83,8 @@ def lib():
         L.e8q_gemv_workspace_bytes.restype = sz
         L.e8q_dequant_gemv.argtypes = [ctypes.POINTER(EncodedC), vp, i32, vp, vp, sz, vp]
         L.e8q_dequant_gemv.restype = ctypes.c_int
+        L.e8q_ste_backward.argtypes = [vp, vp, i64, vp]
+        L.e8q_ste_backward.restype = ctypes.c_int
         L.e8q_set_gemv_path.argtypes = [i32]
         L.e8q_set_gemv_path.restype = ctypes.c_int
         L.e8q_device_error_flags.argtypes = [i32, ctypes.POINTER(ctypes.c_uint64)]
@@ -268,21 +270,35 @@ class Encoder:
             if tuple(w.shape) != self.shapes[i] or w.dtype != self.in_dtype:
                 raise E8qError(f"weight {i}: expected {self.shapes[i]} {self.in_dtype}, got {tuple(w.shape)} {w.dtype}")
             self._mats[i].w = w.data_ptr()
-        if self.scale_in:
-            if scales is None:
-                raise E8qError("scale_in encoder needs scales")
-            for i, s in enumerate(scales):
-                self.scale[i].copy_(s)
+        self._load_scales(scales)
         rc = lib().e8q_project_encode(self._mats, len(self.shapes), ctypes.byref(self._args),
                                       ctypes.c_void_p(self.workspace.data_ptr()), self.workspace.numel(),
                                       _stream_handle(stream))
         _check(rc, "e8q_project_encode")
         return self.result()
 
-    def run_noalloc(self, weights: Sequence[torch.Tensor], stream=None) -> EncodeResult:
+    def _load_scales(self, scales):
+        """Given scales go to the scale buffers the kernels read; an encoder
+        built with scale_in must be given them on every call."""
+        if not self.scale_in:
+            if scales is not None:
+                raise E8qError("scales given to an encoder built without scale_in")
+            return
+        if scales is None:
+            raise E8qError("scale_in encoder needs scales")
+        if len(scales) != len(self.shapes):
+            raise E8qError("number of scale vectors does not match the encoder")
+        for i, s in enumerate(scales):
+            if s.numel() != self.shapes[i][0]:
+                raise E8qError(f"scales {i}: expected {self.shapes[i][0]} values, got {s.numel()}")
+            self.scale[i].copy_(s.reshape(-1))
+
+    def run_noalloc(self, weights: Sequence[torch.Tensor], scales: Optional[Sequence[torch.Tensor]] = None,
+                    stream=None) -> EncodeResult:
         """Same encode through e8q_project_encode_noalloc: the library's
         built-in scratch instead of this encoder's workspace (for callers
-        that cannot allocate; calls on one device must not overlap)."""
+        that cannot allocate; calls on one device must not overlap).  An
+        encoder built with scale_in takes its scales here as in __call__."""
         if len(weights) != len(self.shapes):
             raise E8qError("number of weights does not match the encoder")
         for i, w in enumerate(weights):
@@ -290,6 +306,7 @@ class Encoder:
             if tuple(w.shape) != self.shapes[i] or w.dtype != self.in_dtype:
                 raise E8qError(f"weight {i}: expected {self.shapes[i]} {self.in_dtype}, got {tuple(w.shape)} {w.dtype}")
             self._mats[i].w = w.data_ptr()
+        self._load_scales(scales)
         rc = lib().e8q_project_encode_noalloc(self._mats, len(self.shapes), ctypes.byref(self._args),
                                               _stream_handle(stream))
         _check(rc, "e8q_project_encode_noalloc")
@@ -324,6 +341,24 @@ def e8q_decode(m: Encoded, basis: str = "rotated", out: Optional[torch.Tensor] =
     _require_cuda(out, "out")
     mc = m.c()
     _check(lib().e8q_decode(ctypes.byref(mc), DEQUANT[basis], _ptr(out), _stream_handle(stream)), "e8q_decode")
+    return out
+
+
+def e8q_ste_backward(grad_dequant: torch.Tensor, grad_latent: Optional[torch.Tensor] = None,
+                     stream=None) -> torch.Tensor:
+    """Identity-STE backward: the latents' gradient is the dequantised
+    weights' gradient.  With grad_latent None (or the same tensor) the result
+    is grad_dequant itself and nothing runs; otherwise the library copies it
+    into grad_latent (bf16, same number of elements)."""
+    _require_cuda(grad_dequant, "grad_dequant")
+    if grad_dequant.dtype != torch.bfloat16:
+        raise E8qError("grad_dequant must be bf16")
+    out = grad_dequant if grad_latent is None else grad_latent
+    _require_cuda(out, "grad_latent")
+    if out.dtype != torch.bfloat16 or out.numel() != grad_dequant.numel():
+        raise E8qError("grad_latent must be bf16 with as many elements as grad_dequant")
+    _check(lib().e8q_ste_backward(_ptr(grad_dequant), _ptr(out), grad_dequant.numel(), _stream_handle(stream)),
+           "e8q_ste_backward")
     return out
 
 

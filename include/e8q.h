@@ -269,6 +269,24 @@ e8q_status e8q_dequant_gemv(const e8q_encoded* m /* host */, const void* x_bf16,
                             void* ws, size_t ws_bytes, e8q_stream stream);
 
 /*
+ * Identity-STE backward (E8-QAT, Figure 2 (b): the projection is trained
+ * with an identity straight-through estimator): the gradient of the loss
+ * with respect to the latent weights equals its gradient with respect to the
+ * dequantised weights, element for element, in bf16.
+ *
+ * grad_dequant  [n] bf16 (device): the upstream gradient dL/dW~.
+ * grad_latent   [n] bf16 (device), out: dL/dW.  It may be grad_dequant
+ *               itself: the identity then needs no work, and the call
+ *               returns at once without launching anything (the usual use,
+ *               0 bytes moved).  Otherwise the two buffers must not overlap
+ *               and the call copies the n values (2n bytes read, 2n written).
+ * Both pointers 2-byte aligned; 16-byte alignment of both takes the vector
+ * copy.  Asynchronous on `stream`; errors: INVALID_ARG (n < 0, NULL or
+ * misaligned pointers with n > 0, partially overlapping buffers), CUDA.
+ */
+e8q_status e8q_ste_backward(const void* grad_dequant, void* grad_latent, int64_t n, e8q_stream stream);
+
+/*
  * Project + encode without allocating anything: the same computation and
  * outputs as e8q_project_encode, for callers that cannot allocate device
  * memory at all -- code running where cudaMalloc is unavailable or
@@ -279,17 +297,24 @@ e8q_status e8q_dequant_gemv(const e8q_encoded* m /* host */, const void* x_bf16,
  * The ordering scratch lives in a 2 MiB array compiled into the library
  * (a file-scope __device__ array: every GPU that loads the library holds
  * it until the process exits), so there is no ws argument.  A call needs
- * 16 + 8 * tiles bytes of it, tiles = sum over matrices of
- * ceil(rows / max(1, min(64, 4096 / cols))); a call that needs more returns
- * E8Q_ERR_SCRATCH_LIMIT (about 1 G weights of any shape fit).  The kernel
- * is the general one (any supported shape and dtype); it clears the part of
- * the scratch it uses on `stream` before running.
+ * 16 + 8 * tiles bytes of it, so it fits while tiles <= (2 MiB - 16) / 8 =
+ * 262,142, with tiles = sum over matrices of ceil(rows / rpt) and
+ * rpt = max(1, min(64, floor(4096 / cols))) rows a tile.  The weight count
+ * that fits therefore depends on the width: about 134 M weights at cols = 8,
+ * 268 M at 16, 537 M at 32, 1.07 G at every power-of-two width from 64 to
+ * 4096, and 262,142 rows (4.3 G weights at 16384) for widths above 4096.
+ * A call that needs more returns E8Q_ERR_SCRATCH_LIMIT.  The kernel is the
+ * general one (any supported shape and dtype); it clears the part of the
+ * scratch it uses on `stream` before running.
  *
  * The first call on each device looks up the device address of the scratch
  * array (and uploads the constant tables); make it before any stream
- * capture.  All calls share the one array: calls that overlap on the GPU
- * (other streams, other host threads) race and must be serialised by the
- * caller.  Other arguments, outputs and errors as for e8q_project_encode.
+ * capture.  That address, like the uploaded tables, belongs to the device's
+ * primary context: after cudaDeviceReset the library's per-device state is
+ * stale and must not be used (reload the library in a new process).  All
+ * calls share the one array: calls that overlap on the GPU (other streams,
+ * other host threads) race and must be serialised by the caller.  Other
+ * arguments, outputs and errors as for e8q_project_encode.
  */
 e8q_status e8q_project_encode_noalloc(const e8q_matrix* mats, int32_t n_mats, const e8q_encode_args* args,
                                       e8q_stream stream);

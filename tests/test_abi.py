@@ -145,6 +145,19 @@ def test_decode_and_gemv_reject_bad_args(lib):
                                 ctypes.c_void_p(0x100000), need - 1, None) == 4
 
 
+def test_ste_backward_argument_checks(lib):
+    """The identity-STE backward rejects bad arguments, returns at once for
+    an aliased or empty call (nothing to launch, so no device is needed),
+    and refuses partially overlapping buffers."""
+    vp = ctypes.c_void_p
+    assert lib.e8q_ste_backward(vp(0x100000), vp(0x200000), -1, None) == 1
+    assert lib.e8q_ste_backward(None, vp(0x200000), 8, None) == 1
+    assert lib.e8q_ste_backward(vp(0x100001), vp(0x200000), 8, None) == 1  # odd address
+    assert lib.e8q_ste_backward(vp(0x100000), vp(0x100000), 1 << 20, None) == 0  # aliased: the identity
+    assert lib.e8q_ste_backward(None, None, 0, None) == 0
+    assert lib.e8q_ste_backward(vp(0x100000), vp(0x100010), 64, None) == 1  # overlap by 112 bytes
+
+
 def test_gemv_path_and_error_hooks(lib):
     """The GEMV main-kernel selector accepts 0..2 only; the error-flag read
     rejects a null output before touching a device; the GEMV workspace holds

@@ -521,6 +521,32 @@ def test_moe_bank_full_size_sampled(e8q):
                      label=f"moe[{i}]")
 
 
+def test_ste_backward_identity_on_mlp_gradient(e8q):
+    """Identity STE (Figure 2 (b)): the dense-MLP step's seeded N(0, 1e-3^2)
+    bf16 gradients of both matrices reach the latents bit for bit, copied
+    (vector path, and an unaligned element path with a ragged tail) or
+    aliased (the same tensor, nothing launched)."""
+    for i, shape in enumerate([(4096, 14336), (14336, 4096)]):
+        g_bits = synth.mlp_grad(shape, matrix=i)
+        g = dev_bf16(g_bits)
+        out = torch.full_like(g, float("nan"))
+        r = e8q.e8q_ste_backward(g, out)
+        torch.cuda.synchronize()
+        assert r is out
+        assert np.array_equal(out.cpu().view(torch.int16).numpy().view(np.uint16), g_bits)
+        assert e8q.e8q_ste_backward(g) is g
+    g = dev_bf16(synth.mlp_grad((3, 1001), matrix=2))
+    buf = torch.full((3 * 1001 + 1,), float("nan"), dtype=torch.bfloat16, device="cuda")
+    e8q.e8q_ste_backward(g.reshape(-1), buf[1:])  # 2-byte aligned destination
+    flat = g.reshape(-1)[5:]
+    dst = torch.empty(flat.numel(), dtype=torch.bfloat16, device="cuda")
+    e8q.e8q_ste_backward(flat, dst)  # 2-byte aligned source, 3,998 values
+    torch.cuda.synchronize()
+    assert torch.equal(buf[1:].view(torch.int16), g.reshape(-1).view(torch.int16))
+    assert torch.equal(dst.view(torch.int16), flat.view(torch.int16))
+    assert torch.isnan(buf[:1].float()).all()
+
+
 def test_gather_encoded_nccl_one_rank(e8q):
     """gather_encoded on CUDA tensors over NCCL (one rank: the gathered form
     is the encode's own output, record bytes and row pointers included)."""

@@ -26,7 +26,7 @@ def _dev_bf16(bits):
 def _snapshot(res):
     return dict(idx=[t.cpu().numpy().view(np.uint16).copy() for t in res.idx],
                 scale=[t.cpu().numpy().copy() for t in res.scale],
-                dq=[t.cpu().view(torch.int16).numpy().copy() for t in res.dequant],
+                dq=[t.cpu().view(torch.int16).numpy().copy() for t in res.dequant if t is not None],
                 esc=res.escape_records().copy(), ovf=res.overflow_records().copy(),
                 erp=res.esc_row_ptr.cpu().numpy().copy(), orp=res.ovf_row_ptr.cpu().numpy().copy(),
                 ctr=res.read_counters())
@@ -38,7 +38,8 @@ def _scrub(res):
     for t in res.scale:
         t.fill_(float("nan"))
     for t in res.dequant:
-        t.fill_(float("nan"))
+        if t is not None:
+            t.fill_(float("nan"))
     res.esc.fill_(0xFF)
     res.ovf.fill_(0xFF)
     res.esc_row_ptr.fill_(-1)
@@ -106,6 +107,93 @@ def test_noalloc_matches_workspace_entry_point_bf16():
         np.testing.assert_array_equal(k[far], k_ref[far])
         np.testing.assert_array_equal(r[far], r_ref[far])
         check_original_dequant(got["dq"][0], P, got["scale"][0], d, 2048, "noalloc original")
+
+
+def _run_pair(e8q, shapes, mats, signs, dtype, dequant, scales=None, block=0):
+    """The workspace entry point once, then the no-allocation one twice on
+    scrubbed outputs; returns the three snapshots."""
+    W = [torch.from_numpy(m).cuda() if dtype == torch.float32 else _dev_bf16(m) for m in mats]
+    S = [torch.from_numpy(d).cuda() for d in signs]
+    sc = None if scales is None else [torch.from_numpy(s).cuda() for s in scales]
+    enc = e8q.Encoder(shapes, S, dtype, block, 1.0, dequant, scales is not None, esc_cap=4096, ovf_cap=4096)
+    ref = _snapshot(enc(W, sc))
+    got = []
+    for _ in range(2):
+        _scrub(enc.result())
+        got.append(_snapshot(enc.run_noalloc(W, sc)))
+    return ref, got
+
+
+def _assert_same(ref, got):
+    for k in ("idx", "scale", "dq"):
+        for a, b in zip(ref[k], got[k]):
+            np.testing.assert_array_equal(a, b, err_msg=k)
+    for k in ("esc", "ovf"):
+        assert ref[k].tobytes() == got[k].tobytes(), k
+    np.testing.assert_array_equal(ref["erp"], got["erp"])
+    np.testing.assert_array_equal(ref["orp"], got["orp"])
+    assert ref["ctr"] == got["ctr"]
+
+
+@pytest.mark.gpu
+def test_noalloc_empty_call_writes_csr_terminators():
+    """A call whose only matrix has no rows launches no kernel: the entry
+    point still clears the counters and writes the CSR terminators."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_e8_lattice_b200 import e8q
+
+    e8q.init()
+    d = synth.signs(32, 256)
+    ref, got = _run_pair(e8q, [(0, 256)], [np.zeros((0, 256), np.float32)], [d], torch.float32, "none")
+    for g in got:
+        _assert_same(ref, g)
+        np.testing.assert_array_equal(g["erp"], [0])
+        np.testing.assert_array_equal(g["orp"], [0])
+        assert all(v == 0 for v in g["ctr"].values()), g["ctr"]
+
+
+@pytest.mark.gpu
+def test_noalloc_given_scales_no_dequant():
+    """scale_in = 1 (fixed reconstruction scales, including a zero and a
+    non-finite one) with no dequant output: the scales the caller passes are
+    the ones used, and both entry points agree bit for bit."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_e8_lattice_b200 import e8q
+
+    e8q.init()
+    rng = np.random.default_rng(33)
+    m = (rng.standard_normal((24, 512)) * 0.02).astype(np.float32)
+    s = (np.sqrt((m.astype(np.float64) ** 2).mean(1)) * rng.uniform(0.5, 1.5, 24)).astype(np.float32)
+    s[3], s[7] = 0.0, np.inf
+    d = synth.signs(33, 512)
+    ref, got = _run_pair(e8q, [m.shape], [m], [d], torch.float32, "none", scales=[s])
+    np.testing.assert_array_equal(ref["scale"][0], s)
+    assert (ref["idx"][0][3] == 0).all() and (ref["idx"][0][7] == 0).all()
+    for g in got:
+        _assert_same(ref, g)
+
+
+@pytest.mark.gpu
+def test_noalloc_rotated_dequant_bf16_narrow():
+    """bf16 rows 96 wide (both entry points take the general kernel) with the
+    rotated-basis dequant: outputs agree bit for bit, and the dequant is the
+    exact bf16 product of the encoded points."""
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from bit_e8_lattice_b200 import e8q
+
+    e8q.init()
+    rng = np.random.default_rng(34)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((50, 96)) * 0.02)
+    d = synth.signs(34, 96)
+    ref, got = _run_pair(e8q, [w.shape], [w], [d], torch.bfloat16, "rotated")
+    for g in got:
+        _assert_same(ref, g)
+    P, _, _, _, _ = gpu_points(got[1]["idx"][0].reshape(-1), got[1]["esc"], got[1]["ovf"], 50 * 12)
+    want, _ = oracle.dequant(P, got[1]["scale"][0].astype(np.float64), d, 32, "rotated")
+    np.testing.assert_array_equal(got[1]["dq"][0].view(np.uint16).reshape(want.shape), want)
 
 
 def test_noalloc_rejects_problems_beyond_its_scratch():
