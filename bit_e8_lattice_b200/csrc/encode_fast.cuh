@@ -227,6 +227,26 @@ __device__ __forceinline__ void load_window_raw(unsigned (&raw)[8][4], const uin
     }
 }
 
+// Copy of a window from global memory to shared memory with every
+// non-finite value replaced by 0 (and counted).
+__device__ __forceinline__ void sanitize_window(uint16_t* dst, const uint16_t* src, int nchunks, int lane,
+                                                unsigned& nonfinite) {
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+        if (k >= nchunks) break;
+        const uint4 q = __ldg(reinterpret_cast<const uint4*>(src + 256 * k + 8 * lane));
+        unsigned w[4] = {q.x, q.y, q.z, q.w};
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+            unsigned keep = 0xFFFFFFFFu;
+            if ((w[j] & 0x7F80u) == 0x7F80u) { keep &= 0xFFFF0000u; ++nonfinite; }
+            if ((w[j] & 0x7F800000u) == 0x7F800000u) { keep &= 0x0000FFFFu; ++nonfinite; }
+            w[j] &= keep;
+        }
+        *reinterpret_cast<uint4*>(dst + 256 * k + 8 * lane) = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+}
+
 // Original-basis dequant of one window, in place of its lattice points:
 // v holds doubled coordinates P in the transposed layout (lane (a, q), row
 // h = group 32 a + 4 h + q of the window); writes bf16 (s_r / sqrt(B)) *
@@ -310,7 +330,7 @@ __device__ __forceinline__ void window_dequant_original(float (&v)[8][8], float4
             o[j] = *reinterpret_cast<const unsigned*>(&t);
         }
         apply_signs(o, __ldg(reinterpret_cast<const uint2*>(signs + col)));
-        *reinterpret_cast<uint4*>(dq + te) = make_uint4(o[0], o[1], o[2], o[3]);
+        __stcs(reinterpret_cast<uint4*>(dq + te), make_uint4(o[0], o[1], o[2], o[3]));  // written once: streaming
     }
 }
 
@@ -431,8 +451,8 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
             const MatDesc& M = p.m[ft.mat];
             const unsigned bytes = static_cast<unsigned>(ft.nr) * M.cols * 2u;
             mbar_arrive_expect_tx(&s_full[0], bytes);
-            bulk_load(inbuf, static_cast<const uint16_t*>(M.w) + static_cast<size_t>(ft.r0) * M.cols, bytes,
-                      &s_full[0]);
+            bulk_load_hint(inbuf, static_cast<const uint16_t*>(M.w) + static_cast<size_t>(ft.r0) * M.cols, bytes,
+                           &s_full[0], l2_policy_evict_first());
         }
     }
     __syncthreads();
@@ -494,15 +514,20 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                             }
                         }
                     }
-                    unsigned raw[8][4];
-                    load_window_raw(raw, win, false, M.signs, C, wbase, nchunks, lane, nonfinite);
-                    __syncwarp();
-                    const float ss = window_forward(v, raw, logb, nchunks, scratch, lane, hf);
-                    if (__any_sync(0xFFFFFFFFu, !isfinite(ss))) {  // non-finite input: redo from global, sanitised
-                        const uint16_t* g = static_cast<const uint16_t*>(M.w) + static_cast<size_t>(cur.r0) * C + wbase;
-                        load_window_raw(raw, g, true, M.signs, C, wbase, nchunks, lane, nonfinite);
+                    // a window with a non-finite input runs again from a copy of its
+                    // input in which those values read as 0 (one copy of the transform)
+#pragma unroll 1
+                    for (int pass = 0; pass < 2; ++pass) {
+                        if (pass == 1) {
+                            sanitize_window(win, static_cast<const uint16_t*>(M.w) + static_cast<size_t>(cur.r0) * C + wbase,
+                                            nchunks, lane, nonfinite);
+                            __syncwarp();
+                        }
+                        unsigned raw[8][4];
+                        load_window_raw(raw, win, false, M.signs, C, wbase, nchunks, lane, nonfinite);
                         __syncwarp();
-                        window_forward(v, raw, logb, nchunks, scratch, lane, hf);
+                        const float ss = window_forward(v, raw, logb, nchunks, scratch, lane, hf);
+                        if (!__any_sync(0xFFFFFFFFu, !isfinite(ss))) break;
                     }
                 }
                 // projection + encoding of the warp's 8 x 32 groups
@@ -546,6 +571,8 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     // (P + 9) >> 1 = P / 2 + 4 or + 4.5, keys base 10, exact in fp32); the two
                     // table gathers of all 8 groups are issued together with the core ranks,
                     // so that their latency overlaps them, and the encoding words after them.
+                    // These tables are read through L2 only (__ldcg): their scattered
+                    // lines would otherwise push the rank table T1 out of L1.
                     uint32_t ia[8], ib[8];
                     int rks[8];
                     bool big = false;  // some |P_i| > 255 implies |P|^2 > 65025
@@ -567,8 +594,8 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         const int hk = __float_as_int(fmaf(k.x, 0.5f, base) + 8388608.f) - 0x4B000000;
                         const int lk = __float_as_int(fmaf(k.y, 0.5f, base) + 8388608.f) - 0x4B000000;
                         const int lv = __float_as_int(fmaf(n2, 0.125f, 8388608.f)) - 0x4B000000;
-                        ia[h] = in ? __ldg(g_t1e + hk * 12 + lv) : 0xFFFFFFFFu;
-                        ib[h] = in ? __ldg(g_t2e + lk) : 0xFFFFFFFFu;
+                        ia[h] = in ? __ldcg(g_t1e + hk * 12 + lv) : 0xFFFFFFFFu;
+                        ib[h] = in ? __ldcg(g_t2e + lk) : 0xFFFFFFFFu;
                         rks[h] = lane_ok ? core_rank_nb(P, (oddm >> h) & 1u, n2, g_t1, st2) : 0;
                     }
                     uint32_t ew[8];
@@ -580,7 +607,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         const uint32_t r = ia[h] + ib[h];
                         const bool hit = pend && ia[h] != 0xFFFFFFFFu && ib[h] != 0xFFFFFFFFu &&
                                          r < static_cast<uint32_t>(kExtPoints);
-                        ew[h] = hit ? __ldg(g_res + r) : (2u << 24);
+                        ew[h] = hit ? __ldcg(g_res + r) : (2u << 24);
                     }
 #pragma unroll
                     for (int h = 0; h < 8; ++h) {
@@ -629,7 +656,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                             o.y = bf16x2_of_half_products(s, v[h][2], v[h][3]);
                             o.z = bf16x2_of_half_products(s, v[h][4], v[h][5]);
                             o.w = bf16x2_of_half_products(s, v[h][6], v[h][7]);
-                            *reinterpret_cast<uint4*>(dq + 8 * gt) = o;
+                            __stcs(reinterpret_cast<uint4*>(dq + 8 * gt), o);
                         }
                     } else if (p.dq_mode == E8Q_DEQUANT_ORIGINAL) {
                         window_dequant_original(v, scratch, lane, hf, logb,
@@ -655,7 +682,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         const int g = 32 * c + lane;
                         const uint32_t m = g < G ? map[map_slot(g)] : 0u;
                         const uint32_t kind = m >> 24;
-                        if (g < G) idxs[g] = static_cast<uint16_t>(kind == 2 ? 0u : (m & 0xFFFFu));
+                        if (g < G) __stcs(idxs + g, static_cast<unsigned short>(kind == 2 ? 0u : (m & 0xFFFFu)));
                         const unsigned be = __ballot_sync(0xFFFFFFFFu, kind == 1), bo = __ballot_sync(0xFFFFFFFFu, kind == 2);
                         if (lane == 0) {
                             cnt[c] = __popc(be);
@@ -682,7 +709,10 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     const int16_t* oscr = ovf_scratch + (static_cast<size_t>(sl3) * kFastTileGroups + 256 * warp) * 8;
                     const uint32_t gw = M.group_base + static_cast<uint32_t>(prev3.r0) * gpr + 256u * warp;
                     long long pe = ex_e + cnt[c0], po = ex_o + cnt[kFastCnt + c0];
-                    const int n = static_cast<int>((cnt[c0 + 8] - cnt[c0]) + (cnt[kFastCnt + c0 + 8] - cnt[kFastCnt + c0]));
+                    // (at most the window's 256 groups: the bound keeps every list read
+                    // inside the window's part of the map)
+                    const int n = min(256, static_cast<int>((cnt[c0 + 8] - cnt[c0]) +
+                                                            (cnt[kFastCnt + c0 + 8] - cnt[kFastCnt + c0])));
                     const unsigned lt = lanemask_lt();
                     for (int j0 = 0; j0 < n; j0 += 32) {
                         const int j = j0 + lane;
@@ -693,7 +723,7 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                         const uint32_t lg = e >> 24;
                         if (es) {
                             const long long pos = pe + __popc(be & lt);
-                            if (pos < p.esc_cap) *reinterpret_cast<uint2*>(p.esc + pos) = make_uint2(gw + lg, e & 0xFFFFFFu);
+                            if (pos < p.esc_cap) __stcs(reinterpret_cast<uint2*>(p.esc + pos), make_uint2(gw + lg, e & 0xFFFFFFu));
                         } else if (ov) {
                             const long long pos = po + __popc(bo & lt);
                             if (pos < p.ovf_cap) {
@@ -734,8 +764,11 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     const unsigned bytes = static_cast<unsigned>(nt.nr) * M.cols * 2u;
                     uint64_t* bar = &s_full[(i + 1) & 1];
                     mbar_arrive_expect_tx(bar, bytes);
-                    bulk_load(inbuf + ((i + 1) & 1) * kFastTileElems,
-                              static_cast<const uint16_t*>(M.w) + static_cast<size_t>(nt.r0) * M.cols, bytes, bar);
+                    // the latent weights are read once: their L2 lines go first, so that
+                    // the lookup tables stay in L2
+                    bulk_load_hint(inbuf + ((i + 1) & 1) * kFastTileElems,
+                                   static_cast<const uint16_t*>(M.w) + static_cast<size_t>(nt.r0) * M.cols, bytes, bar,
+                                   l2_policy_evict_first());
                 }
             }
             __syncwarp();
