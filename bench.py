@@ -378,6 +378,141 @@ def record_bytes(rp, lo, hi):
     return int(rp[hi] - rp[lo])
 
 
+def run_sharded(args, batches, rank, world, dev):
+    """Row-sharded blocks of one model (weak scaling): rank r holds rows
+    [4096 r, 4096 (r + 1)) of an up matrix and [14336 r, 14336 (r + 1)) of a
+    down matrix (the dense-MLP recipe, seeded per rank).  One step: the
+    rank's project+encode launch, the identity-STE backward, the exchange of
+    every rank's encoded block (gather_encoded: every rank then holds the
+    whole model in the 2-bit form), the dequant-GEMV of the rank's up rows
+    at each batch and the all-gather of the products (gemv_rows_allgather).
+    Timed on the device with events, eager launches (the exchange reads its
+    sizes on the host), max over ranks."""
+    import torch
+    import torch.distributed as dist
+
+    from bit_e8_lattice_b200 import dist as e8dist
+    from bit_e8_lattice_b200 import e8q, synth
+    from bit_e8_lattice_b200.dist import max_over_ranks
+
+    (up, d_up), (down, d_dn) = synth.mlp_14336(seed=4 + 1000 * rank)
+    t = lambda bits: torch.from_numpy(bits.view(np.int16)).view(torch.bfloat16).to(dev)
+    W = [t(up), t(down)]
+    S = [torch.from_numpy(d_up).to(dev), torch.from_numpy(d_dn).to(dev)]
+    X = {b: t(synth.gemv_x(b, D_FF)) for b in batches}
+    GRAD = [t(synth.mlp_grad((D_MODEL, D_FF), seed=40 + rank, matrix=0)),
+            t(synth.mlp_grad((D_FF, D_MODEL), seed=40 + rank, matrix=1))]
+    G = D_MODEL * (D_FF // 8) + D_FF * (D_MODEL // 8)
+    enc = e8q.Encoder([(D_MODEL, D_FF), (D_FF, D_MODEL)], S, torch.bfloat16, 0, 1.0, "original",
+                      esc_cap=G // 2, ovf_cap=G // 16)
+    res = enc(W)
+    gemvs = {b: e8q.Gemv(res.encoded[0], b) for b in batches}
+
+    def exchange(m):
+        erp = res.esc_row_ptr[res.row_base[m]: res.row_base[m] + res.encoded[m].rows + 1]
+        orp = res.ovf_row_ptr[res.row_base[m]: res.row_base[m] + res.encoded[m].rows + 1]
+        e0, e1, o0, o1 = torch.stack([erp[0], erp[-1], orp[0], orp[-1]]).cpu().tolist()  # one host read
+        esc = res.esc[8 * e0: 8 * e1]
+        ovf = res.ovf[20 * o0: 20 * o1]
+        rows = res.encoded[m].rows
+        # group ids of the second matrix start after the first one's groups: rebase to the matrix
+        base = res.group_base[m]
+        if base and e1 > e0:
+            esc = esc.view(torch.int32).view(-1, 2).clone()
+            esc[:, 0] = e8dist.shift_group_ids(esc[:, 0], -base)
+            esc = esc.view(torch.uint8).reshape(-1)
+        if base and o1 > o0:
+            ovf = ovf.view(torch.int32).view(-1, 5).clone()
+            ovf[:, 0] = e8dist.shift_group_ids(ovf[:, 0], -base)
+            ovf = ovf.view(torch.uint8).reshape(-1)
+        part = (res.idx[m], res.scale[m], esc, e1 - e0, ovf, o1 - o0, erp - e0, orp - o0, rank * rows)
+        if world == 1:
+            return e8dist.combine_shards([part], res.encoded[m].cols // 8)
+        return e8dist.gather_encoded(*part)
+
+    def step(Win, Xin):
+        enc(Win)
+        for g in GRAD:
+            e8q.e8q_ste_backward(g)
+        whole = [exchange(0), exchange(1)]
+        ys = {}
+        for b in batches:
+            y = gemvs[b](Xin[b])
+            ys[b] = e8dist.gemv_rows_allgather(y) if world > 1 else y
+        return whole, ys
+
+    for _ in range(max(args.warmup, 3)):
+        step(W, X)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    a, z = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    with ClockSampler(int(os.environ.get("LOCAL_RANK", "0"))) as clocks:
+        a.record()
+        for _ in range(args.steps):
+            whole, ys = step(W, X)
+        z.record()
+        torch.cuda.synchronize()
+    ms = max_over_ranks(a.elapsed_time(z), dev)
+    wire = sum(int(x.numel() * x.element_size()) for x in whole[0] + whole[1])
+
+    # end to end: this step's inputs from pinned host memory, every product back
+    e2e = None
+    if args.e2e_steps > 0:
+        Wh = [W[0].cpu().pin_memory(), W[1].cpu().pin_memory()]
+        Xh = {b: X[b].cpu().pin_memory() for b in batches}
+        Wd = [torch.empty_like(W[0]), torch.empty_like(W[1])]
+        Xd = {b: torch.empty_like(X[b]) for b in batches}
+        Yh = {b: torch.empty((b, world * D_MODEL), dtype=torch.bfloat16).pin_memory() for b in batches}
+        h2d = sum(w.numel() * 2 for w in Wh) + sum(x.numel() * 2 for x in Xh.values())
+        d2h = sum(y.numel() * 2 for y in Yh.values())
+
+        def e2e_step():
+            for i in range(2):
+                Wd[i].copy_(Wh[i], non_blocking=True)
+            for b in batches:
+                Xd[b].copy_(Xh[b], non_blocking=True)
+            _, ys2 = step(Wd, Xd)
+            for b in batches:
+                Yh[b].copy_(ys2[b], non_blocking=True)
+
+        e2e_step()
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        a2, z2 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a2.record()
+        for _ in range(args.e2e_steps):
+            e2e_step()
+        z2.record()
+        torch.cuda.synchronize()
+        ems = max_over_ranks(a2.elapsed_time(z2), dev)
+        e2e = {"value": world * G * args.e2e_steps / (ems * 1e-3) / 1e9, "unit": UNIT, "h2d_bytes_per_step": h2d,
+               "d2h_bytes_per_step": d2h, "steps": args.e2e_steps}
+    if world > 1:
+        dist.barrier()
+    if rank == 0:
+        value = world * G * args.steps / (ms * 1e-3) / 1e9
+        line = {
+            "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+            "config": {"workload": WORKLOAD + "; row-sharded blocks, one per GPU, with their exchange",
+                       "groups_per_step_per_gpu": G, "gemv_batches": batches,
+                       "parallelism": f"row-sharded x{world}: gather_encoded (2-bit form of every block to every "
+                                      f"rank) + all-gather of each GEMV product",
+                       "exchanged_bytes_per_rank_per_step": wire,
+                       "l2": "inputs larger than L2 (235 MB of latent weights read per step per GPU)"},
+            "timing": "eager launches, device events, max over ranks",
+            "gpu_launches": args.steps * (1 + 3 * len(batches)),
+            "cpu_baseline": None, "e2e": e2e, "clocks": clocks.summary(),
+        }
+        print(json.dumps(line), flush=True)
+    if world > 1:
+        dist.destroy_process_group()
+    return 0
+
+
 def main():
     ap = argparse.ArgumentParser(description=__doc__)
     ap.add_argument("--gpus", type=int, default=1)
@@ -393,6 +528,9 @@ def main():
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one captured graph")
     ap.add_argument("--gemv-path", choices=["auto", "mma_sync", "tcgen05"], default="auto",
                     help="GEMV main kernel (auto: the library's choice)")
+    ap.add_argument("--mode", choices=["auto", "replicas", "sharded"], default="auto",
+                    help="several GPUs: independent replicas, or row-sharded blocks of one model with their "
+                         "exchange (gather_encoded + all-gather of y); auto: sharded when N > 1")
     args = ap.parse_args()
     batches = [int(b) for b in args.batches.split(",") if b]
     if args.impl == "reference":
@@ -415,6 +553,9 @@ def main():
 
     e8q.init()
     e8q.set_gemv_path(args.gemv_path)
+    mode = args.mode if args.mode != "auto" else ("sharded" if world > 1 else "replicas")
+    if mode == "sharded":
+        return run_sharded(args, batches, rank, world, dev)
     data = host_data(batches)
     (up, d_up), (down, d_dn), xs = data
 

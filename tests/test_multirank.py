@@ -171,3 +171,83 @@ def test_shift_group_ids_across_the_sign_bit():
         words = torch.from_numpy(ids.astype(np.uint32).view(np.int32))
         got = shift_group_ids(words, off).numpy().view(np.uint32).astype(np.uint64)
         np.testing.assert_array_equal(got, (ids + np.uint64(off)) % np.uint64(2**32))
+
+
+def _gemv_split_worker(rank, world, port, q):
+    import sys
+
+    sys.path.insert(0, ROOT)
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port), RANK=str(rank), WORLD_SIZE=str(world))
+    import torch
+    import torch.distributed as dist
+    from datetime import timedelta
+
+    import oracle
+    from bit_e8_lattice_b200 import dist as e8dist
+    from bit_e8_lattice_b200 import synth
+
+    dist.init_process_group("gloo", rank=rank, world_size=world, timeout=timedelta(seconds=60))
+    try:
+        w, d = synth.small_f32(rows=200)
+        x = synth.bf16_bits_to_f64(synth.gemv_x(3, 256))
+        a, b = e8dist.shard_rows(w.shape[0], world, rank)
+        out = oracle.project_encode(w[a:b].astype(np.float64), d, 256, want_x=False, want_margin=False)
+        y_local = oracle.gemv(out["P"], out["scale"], d, 256, x)  # this rank's rows of W x
+        y = e8dist.gemv_rows_allgather(torch.from_numpy(y_local))
+        q.put((rank, y.numpy().copy()))
+    finally:
+        dist.destroy_process_group()
+
+
+def test_gemv_row_split_allgather_equals_whole_matrix():
+    """Two gloo ranks, uneven row shards of a 200-row matrix: each multiplies
+    its own rows (oracle GEMV on its shard's encoding), gemv_rows_allgather
+    gives every rank the whole y, equal to the oracle's whole-matrix product."""
+    import oracle
+    from bit_e8_lattice_b200 import synth
+
+    world = 3
+    ctx = mp.get_context("spawn")
+    q = ctx.Queue()
+    port = _free_port()
+    procs = [ctx.Process(target=_gemv_split_worker, args=(r, world, port, q)) for r in range(world)]
+    for p in procs:
+        p.start()
+    results = [q.get(timeout=180) for _ in range(world)]
+    for p in procs:
+        p.join(timeout=60)
+        assert p.exitcode == 0
+    w, d = synth.small_f32(rows=200)
+    x = synth.bf16_bits_to_f64(synth.gemv_x(3, 256))
+    full = oracle.project_encode(w.astype(np.float64), d, 256, want_x=False, want_margin=False)
+    y_ref = oracle.gemv(full["P"], full["scale"], d, 256, x)
+    for rank, y in results:
+        assert y.shape == y_ref.shape
+        np.testing.assert_allclose(y, y_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_combine_shards_without_a_process_group():
+    """combine_shards alone (the step after the exchange) joins three uneven
+    shards, given out of order, into the whole matrix's encoding."""
+    import torch
+
+    import oracle
+    from bit_e8_lattice_b200 import dist as e8dist
+    from bit_e8_lattice_b200 import synth
+
+    w, d = synth.small_f32()
+    parts = []
+    for a, b in [(100, 256), (0, 37), (37, 100)]:
+        out = oracle.project_encode(w[a:b].astype(np.float64), d, 256, want_x=False, want_margin=False)
+        idx, scale, esc, ne, ovf, no, erp, orp = _library_form(out, b - a, 32)
+        t = lambda x: torch.from_numpy(np.ascontiguousarray(x))
+        parts.append((t(idx), t(scale), torch.frombuffer(bytearray(esc + bytes(8)), dtype=torch.uint8), ne,
+                      torch.frombuffer(bytearray(ovf + bytes(20)), dtype=torch.uint8), no, t(erp), t(orp), a))
+    got = [r.numpy() for r in e8dist.combine_shards(parts, 32)]
+    full = oracle.project_encode(w.astype(np.float64), d, 256, want_x=False, want_margin=False)
+    idx, scale, esc, ne, ovf, no, erp, orp = _library_form(full, w.shape[0], 32)
+    np.testing.assert_array_equal(got[0], idx)
+    np.testing.assert_array_equal(got[1], scale)
+    assert got[2].tobytes() == esc and got[3].tobytes() == ovf
+    np.testing.assert_array_equal(got[4], erp)
+    np.testing.assert_array_equal(got[5], orp)

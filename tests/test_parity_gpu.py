@@ -547,9 +547,57 @@ def test_ste_backward_identity_on_mlp_gradient(e8q):
     assert torch.isnan(buf[:1].float()).all()
 
 
+def _encoded_view(e8q, idx, scale, signs, esc, ovf, erp, orp, cols):
+    """An e8q.Encoded over combined (whole-matrix) buffers."""
+    return e8q.Encoded(idx, scale, signs, esc, erp, ovf, orp, idx.shape[0], cols, 0, 0,
+                       max(1, esc.numel() // 8), max(1, ovf.numel() // 20))
+
+
+def test_row_shards_encoded_on_gpu_equal_oracle_whole_matrix(e8q):
+    """Row-sharded encoding (the multi-GPU path's local step) with the CUDA
+    kernels: three uneven row shards of one matrix, each its own encode call
+    (group ids from the shard's first row), joined by combine_shards, equal
+    the oracle's encoding of the whole matrix (above the tie margin); the
+    row-split GEMV (each shard's rows, concatenated) matches the oracle's
+    whole-matrix product."""
+    from bit_e8_lattice_b200 import dist as e8dist
+
+    rng = np.random.default_rng(18)
+    R, C = 300, 2048
+    w = synth.f64_to_bf16_bits(rng.standard_normal((R, C)) * 0.02)
+    d = synth.signs(18, C)
+    x_bits = synth.gemv_x(4, C)
+    x = dev_bf16(x_bits)
+    parts, ys = [], []
+    for a, b in [(0, 77), (77, 150), (150, 300)]:
+        _, res = run_encode(e8q, [w[a:b]], [d], 0)
+        ctr = res.read_counters()
+        parts.append((res.idx[0], res.scale[0], res.esc.clone(), ctr["n_escape"], res.ovf.clone(), ctr["n_overflow"],
+                      res.esc_row_ptr.clone(), res.ovf_row_ptr.clone(), a))
+        ys.append(e8q.Gemv(res.encoded[0], 4)(x).clone())
+    idx, scale, esc, ovf, erp, orp = e8dist.combine_shards(parts, C // 8)
+    torch.cuda.synchronize()
+    out = oracle.project_encode(synth.bf16_bits_to_f64(w), d, 2048)
+    esc_np = np.frombuffer(esc.cpu().numpy().tobytes(), e8q.ESC_DTYPE)
+    ovf_np = np.frombuffer(ovf.cpu().numpy().tobytes(), e8q.OVF_DTYPE)
+    st = check_encode(out, host_idx(idx), scale.cpu().numpy(), esc_np, ovf_np, 0, None, C // 8, "row shards")
+    assert st["rho"] > 0.1
+    np.testing.assert_array_equal(erp.cpu().numpy()[-1], len(esc_np))
+    # the whole-matrix GEMV from the joined form equals the shards' rows
+    m = _encoded_view(e8q, idx, scale, dev(d), esc, ovf, erp, orp, C)
+    y_whole = e8q.Gemv(m, 4)(x)
+    y_split = torch.cat(ys, dim=1)
+    P = st["points"]
+    y_ref = oracle.gemv(P, scale.cpu().numpy().astype(np.float64), d, 2048, synth.bf16_bits_to_f64(x_bits))
+    check_gemv(y_split.cpu().view(torch.int16).numpy(), y_ref, "row-split GEMV")
+    check_gemv(y_whole.cpu().view(torch.int16).numpy(), y_ref, "joined-form GEMV")
+
+
 def test_gather_encoded_nccl_one_rank(e8q):
-    """gather_encoded on CUDA tensors over NCCL (one rank: the gathered form
-    is the encode's own output, record bytes and row pointers included)."""
+    """gather_encoded on CUDA tensors over NCCL (one rank, its two
+    collectives included): the gathered encoding of a matrix equals the
+    oracle's encoding of it above the tie margin, and its record bytes and
+    row pointers equal the encode call's own."""
     import socket
     from datetime import timedelta
 
@@ -570,9 +618,17 @@ def test_gather_encoded_nccl_one_rank(e8q):
     try:
         out = e8dist.gather_encoded(res.idx[0], res.scale[0], res.esc, ctr["n_escape"], res.ovf, ctr["n_overflow"],
                                     res.esc_row_ptr, res.ovf_row_ptr, 0)
+        y = e8dist.gemv_rows_allgather(e8q.Gemv(res.encoded[0], 4)(dev_bf16(synth.gemv_x(4, 2048))))
         torch.cuda.synchronize()
     finally:
         dist.destroy_process_group()
     assert torch.equal(out[0], res.idx[0]) and torch.equal(out[1], res.scale[0])
     assert torch.equal(out[2], res.esc[: 8 * ctr["n_escape"]]) and torch.equal(out[3], res.ovf[: 20 * ctr["n_overflow"]])
     assert torch.equal(out[4], res.esc_row_ptr) and torch.equal(out[5], res.ovf_row_ptr)
+    ref = oracle.project_encode(synth.bf16_bits_to_f64(w), d, 2048)
+    esc_np = np.frombuffer(out[2].cpu().numpy().tobytes(), e8q.ESC_DTYPE)
+    ovf_np = np.frombuffer(out[3].cpu().numpy().tobytes(), e8q.OVF_DTYPE)
+    st = check_encode(ref, host_idx(out[0]), out[1].cpu().numpy(), esc_np, ovf_np, 0, None, 256, "gathered")
+    y_ref = oracle.gemv(st["points"], out[1].cpu().numpy().astype(np.float64), d, 2048,
+                        synth.bf16_bits_to_f64(synth.gemv_x(4, 2048)))
+    check_gemv(y.cpu().view(torch.int16).numpy(), y_ref, "gathered GEMV")
