@@ -71,6 +71,10 @@ def lib():
         L.eo_project_encode_rows.argtypes = [vp, i64, i64, vp, i64, f64, vp, vp, vp, vp, vp, vp, vp]
         L.eo_project_encode_rows.restype = i64
         L.eo_project_encode_vectors.argtypes = [vp, i64, vp, vp, vp, vp, vp]
+        L.eo_nearest_core.argtypes = [vp, vp]
+        L.eo_nearest_core.restype = i32
+        L.eo_project_core_rows.argtypes = [vp, i64, i64, vp, i64, f64, vp, vp, vp, vp]
+        L.eo_project_core_rows.restype = i64
         L.eo_dequant_rows.argtypes = [vp, vp, i64, i64, vp, i64, ctypes.c_int, vp, vp]
         L.eo_rht_vectors.argtypes = [vp, i64, i64, vp, i64, vp]
         rc = L.eo_init()
@@ -129,6 +133,38 @@ def project_encode_vectors(x: np.ndarray):
     root = np.zeros(n, np.int32)
     lib().eo_project_encode_vectors(_p(x), n, _p(P), _p(m), _p(idx), _p(kind), _p(root))
     return dict(P=P, margin=m, idx=idx, kind=kind, root=root)
+
+
+def nearest_core_vectors(x: np.ndarray):
+    """Core-clipped projection (Figure 2 (a): PTQ from the fixed core): the
+    nearest of the 65,536 core codewords to each 8-vector, searched
+    exhaustively; ties to the smaller index.  Returns idx, P, margin."""
+    x = np.ascontiguousarray(np.asarray(x, np.float64).reshape(-1, 8))
+    n = x.shape[0]
+    idx = np.zeros(n, np.int32)
+    m = np.zeros(n, np.float64)
+    L = lib()
+    for k in range(n):
+        mk = ctypes.c_double()
+        idx[k] = L.eo_nearest_core(_p(x[k]), ctypes.byref(mk))
+        m[k] = mk.value
+    return dict(idx=idx, P=core_points()[idx].astype(np.int32), margin=m)
+
+
+def project_core(w: np.ndarray, signs: np.ndarray, block: int, kappa: float = 1.0, want_margin: bool = True):
+    """The row pipeline of project_encode with the core-clipped projection:
+    every group's nearest core point (no escape or overflow records)."""
+    w = np.ascontiguousarray(np.asarray(w, np.float64))
+    R, C = w.shape
+    d = np.ascontiguousarray(np.asarray(signs, np.int8).reshape(C))
+    G = R * (C // 8)
+    scale = np.zeros(R, np.float64)
+    P = np.zeros((G, 8), np.int32)
+    m = np.zeros(G, np.float64) if want_margin else None
+    idx = np.zeros(G, np.int32)
+    nf = lib().eo_project_core_rows(_p(w), R, C, _p(d), int(block), float(kappa), _p(scale), _p(P),
+                                    _p(m) if m is not None else None, _p(idx))
+    return dict(scale=scale, P=P, margin=m, idx=idx, nonfinite=int(nf))
 
 
 def encode_points(P: np.ndarray):

@@ -351,6 +351,78 @@ int64_t eo_project_encode_rows(const double* w, int64_t R, int64_t C, const int8
     return nonfinite;
 }
 
+/* ---------------------------------------------------------------------
+ * Core-clipped projection [E8QAT-F2 (a): post-training quantisation starts
+ * the latent weights from a fixed E8 core; (b) contrasts it with the
+ * unclipped projection used during QAT]: the core point nearest to x,
+ * found by searching all 65,536 core codewords in fp64.  Equal distances
+ * go to the smaller core index.  margin = second-smallest minus smallest
+ * squared distance (x units) over the core.
+ * ------------------------------------------------------------------- */
+int32_t eo_nearest_core(const double* x, double* margin)
+{
+    if (eo_init() != 0) return -1;
+    double best = INFINITY, second = INFINITY;
+    int32_t bi = 0;
+    for (int32_t k = 0; k < EO_CORE; k++) {
+        const int8_t* P = g_pts[k].c;
+        double dd = 0.0;
+        for (int i = 0; i < 8; i++) {
+            double t = x[i] - 0.5 * (double)P[i];
+            dd += t * t;
+        }
+        if (dd < best) {
+            second = best;
+            best = dd;
+            bi = k;
+        } else if (dd < second) {
+            second = dd;
+        }
+    }
+    if (margin) *margin = second - best;
+    return bi;
+}
+
+/* Row pipeline with the core-clipped projection: the transform and scale of
+ * eo_project_encode_rows, then the nearest core point of every group
+ * (idx[G]; P[G][8] its doubled coordinates; margin[G] nullable). */
+int64_t eo_project_core_rows(const double* w, int64_t R, int64_t C, const int8_t* d, int64_t B, double kappa,
+                             double* scale, int32_t* P, double* margin, int32_t* idx)
+{
+    int64_t nonfinite = 0;
+    double* v = (double*)malloc(sizeof(double) * (size_t)(C > 0 ? C : 1));
+    int64_t gpr = C / 8;
+    for (int64_t r = 0; r < R; r++) {
+        for (int64_t c = 0; c < C; c++) {
+            double t = w[r * C + c];
+            if (!isfinite(t)) {
+                t = 0.0;
+                nonfinite++;
+            }
+            v[c] = (double)d[c] * t;
+        }
+        if (B > 1) {
+            double inv = 1.0 / sqrt((double)B);
+            for (int64_t b0 = 0; b0 < C; b0 += B) {
+                eo_fwht(v + b0, B);
+                for (int64_t j = 0; j < B; j++) v[b0 + j] *= inv;
+            }
+        }
+        double ss = 0.0;
+        for (int64_t c = 0; c < C; c++) ss += v[c] * v[c];
+        double s = (C > 0) ? sqrt(ss / (double)C) / kappa : 0.0;
+        scale[r] = s;
+        for (int64_t c = 0; c < C; c++) v[c] = (s > 0.0) ? v[c] / s : 0.0;
+        for (int64_t g = 0; g < gpr; g++) {
+            int64_t G = r * gpr + g;
+            idx[G] = eo_nearest_core(v + 8 * g, margin ? margin + G : NULL);
+            for (int i = 0; i < 8; i++) P[8 * G + i] = g_pts[idx[G]].c[i];
+        }
+    }
+    free(v);
+    return nonfinite;
+}
+
 /* Project and encode free 8-vectors (no transform, no scale). */
 void eo_project_encode_vectors(const double* x, int64_t n, int32_t* P, double* margin, int32_t* idx, int32_t* kind,
                                int32_t* root)

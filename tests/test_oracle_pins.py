@@ -423,3 +423,79 @@ def test_escape_fraction_counts_groups(orc):
     rho = kv["escaped_groups"] / (kv["quantized_params"] / kv["group_size"])
     assert round(rho, 9) == kv["rho_step375"]
     assert kv["core_codewords"] == len(orc.core_points())
+
+
+# ----------------------------------------------------------------------
+# Core-clipped projection (E8-QAT Figure 2 (a): PTQ from the fixed core)
+# ----------------------------------------------------------------------
+def _independent_core():
+    """The 65,536 first points in (norm, lex) order, enumerated by numpy
+    (not the oracle's table), as undoubled coordinates."""
+    P, _ = np_e8_points(48)
+    return P[:65536].astype(np.float64) / 2.0
+
+
+def test_nearest_core_matches_kdtree_search(orc):
+    """A KD-tree nearest-neighbour query over an independently enumerated core
+    gives the oracle's nearest core point on every vector clear of a tie;
+    vectors span the core's inside, its boundary and far outside it."""
+    from scipy.spatial import cKDTree
+
+    core = _independent_core()
+    tree = cKDTree(core)
+    rng = np.random.default_rng(77)
+    x = np.concatenate([rng.standard_normal((600, 8)) * s for s in (0.7, 1.2, 1.8, 3.0)])
+    out = orc.nearest_core_vectors(x)
+    dist, k = tree.query(x)
+    clear = out["margin"] > 1e-9
+    assert clear.mean() > 0.99
+    np.testing.assert_array_equal(out["idx"][clear], k[clear])
+    np.testing.assert_allclose(((x - out["P"] / 2.0) ** 2).sum(1), dist ** 2, rtol=1e-12, atol=1e-12)
+
+
+def test_nearest_core_fixes_core_points_and_agrees_inside(orc):
+    """Every core point maps to itself (rho = 0 at PTQ init, Table 9, step
+    100); a vector whose nearest E8 point is in the core gets that point."""
+    core = orc.core_points().astype(np.float64) / 2.0
+    sel = np.arange(0, 65536, 97)
+    out = orc.nearest_core_vectors(core[sel] + 1e-3)
+    np.testing.assert_array_equal(out["idx"], sel)
+    rng = np.random.default_rng(78)
+    x = rng.standard_normal((800, 8)) * 1.1
+    free = orc.project_encode_vectors(x)
+    inside = (free["kind"] == 0) & (free["margin"] > 1e-9)
+    assert inside.mean() > 0.5
+    out = orc.nearest_core_vectors(x[inside])
+    np.testing.assert_array_equal(out["idx"], free["idx"][inside])
+
+
+def test_nearest_core_of_far_vectors_lies_on_the_boundary(orc):
+    """Far outside the core the nearest core point has |p|^2 >= 10 (the core
+    holds the whole ball |p|^2 <= 10 and part of the next shell) and points
+    the way of x."""
+    rng = np.random.default_rng(79)
+    x = rng.standard_normal((300, 8))
+    x = x / np.linalg.norm(x, axis=1, keepdims=True) * 6.0
+    out = orc.nearest_core_vectors(x)
+    p = out["P"] / 2.0
+    assert ((p ** 2).sum(1) >= 10 - 1e-9).all()
+    cos = (p * x).sum(1) / (np.linalg.norm(p, axis=1) * 6.0)
+    assert (cos > 0.8).all()
+
+
+def test_project_core_rows_scale_and_no_records(orc):
+    """The row pipeline with the core-clipped projection: the same scales as
+    the unclipped pipeline, every group a core point, each as close as any
+    core point can be (checked against the KD-tree on the oracle's x)."""
+    from scipy.spatial import cKDTree
+
+    w, d = synth.small_f32(rows=24)
+    full = orc.project_encode(w.astype(np.float64), d, 256)
+    core = orc.project_core(w.astype(np.float64), d, 256)
+    np.testing.assert_array_equal(core["scale"], full["scale"])
+    tree = cKDTree(_independent_core())
+    dist, k = tree.query(full["x"].reshape(-1, 8))
+    clear = core["margin"] > 1e-9
+    np.testing.assert_array_equal(core["idx"][clear], k[clear])
+    kept = full["kind"] == 0
+    np.testing.assert_array_equal(core["idx"][kept & clear], full["idx"][kept & clear])
