@@ -33,9 +33,125 @@ struct EncodeParams {
     int32_t n_mats;
     int32_t n_tiles;
     int32_t total_rows;
-    int32_t clamp;  // fast kernel: inputs may reach |2x| >= 2^14 (given scales or large kappa)
+    int32_t clamp;      // fast kernel: inputs may reach |2x| >= 2^14 (given scales or large kappa)
+    int32_t core_only;  // the core-clipped projection (E8Q_ENCODE_CORE_ONLY)
     MatDesc m[MAXM];
 };
+
+// Nearest core point of X = 2x whose nearest E8 point P lies outside the
+// core ("E8-QAT", Figure 2 (a): post-training quantisation starts from the
+// fixed core).  Equal distances go to the smaller core index.  On return P
+// holds the core point; the result is its core index.
+//
+// A first bound comes from two points near x: the escape base P - r (the
+// escape rule's root), when in the core, and the nearest E8 point of x
+// pulled in to |x|^2 = 6, which is always in the core.  Then every E8 point
+// c within that distance of x and with |c|^2 <= 12 (a superset of the core)
+// is visited by a depth-first enumeration of each coset (D8 and D8 + 1/2:
+// integer vectors z, or z + 1/2, with an even coordinate sum), the radius
+// shrinking as closer core points are found; each point visited is checked
+// against the core by its rank.
+__device__ __noinline__ int nearest_core_point(const float (&X)[8], int (&P)[8], const uint16_t* __restrict__ st1,
+                                               const uint16_t* __restrict__ st2) {
+    float best = INFINITY;  // squared distance, x units
+    int brank = 0x7FFFFFFF;
+    int bP[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i) bP[i] = 0;
+    auto consider = [&](const int (&C)[8]) {
+        float d = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) {
+            const float t = 0.5f * (X[i] - static_cast<float>(C[i]));
+            d = fmaf(t, t, d);
+        }
+        if (d <= best) {
+            const int r = core_rank(C, st1, st2);
+            if (r >= 0 && (d < best || r < brank)) {
+                best = d;
+                brank = r;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) bP[i] = C[i];
+            }
+        }
+    };
+    {
+        int R[8], Q[8];
+        best_escape_root(P, R);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) Q[i] = P[i] - R[i];
+        consider(Q);
+        // x pulled in to |x'|^2 = 6: its nearest E8 point p' has |p'| <= sqrt(6) + 1
+        // (the covering radius is 1), so |p'|^2 <= 10 and p' is in the core
+        float n2 = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) n2 = fmaf(X[i], X[i], n2);
+        const float k = fminf(4.8989795f * rsqrtf(fmaxf(n2, 1e-30f)), 1.f);  // |2x'| = 2 sqrt(6)
+        float Xs[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) Xs[i] = X[i] * k;
+        int Ps[8];
+        e8_nearest_doubled(Xs, Ps);
+        consider(Ps);
+    }
+    // every E8 point c within the current distance of x with |c|^2 <= 12 (all
+    // core points have), coset by coset, depth first over the coordinates
+    constexpr float kCoreN2 = 12.f + 1e-3f;
+    for (int coset = 0; coset < 2; ++coset) {
+        const float off = coset ? 0.5f : 0.f;
+        float cy[8];
+#pragma unroll
+        for (int i = 0; i < 8; ++i) cy[i] = 0.5f * X[i] - off;
+        int z[8], hi[8];
+        float part[9], pn[9];  // partial squared distance to x, partial squared norm of c
+        part[0] = 0.f;
+        pn[0] = 0.f;
+        int lvl = 0;
+        auto bounds = [&](int l) {
+            const float sq = sqrtf(fmaxf(best - part[l], 0.f));
+            const float sn = sqrtf(fmaxf(kCoreN2 - pn[l], 0.f));
+            z[l] = max(static_cast<int>(ceilf(cy[l] - sq)), static_cast<int>(ceilf(-sn - off)));
+            hi[l] = min(static_cast<int>(floorf(cy[l] + sq)), static_cast<int>(floorf(sn - off)));
+        };
+        bounds(0);
+        int guard = 0;
+        while (lvl >= 0 && ++guard < (1 << 22)) {  // bounded: the lens holds at most the 117,361 points of |c|^2 <= 12
+            if (z[lvl] > hi[lvl]) {
+                --lvl;
+                if (lvl >= 0) ++z[lvl];
+                continue;
+            }
+            const float t = cy[lvl] - static_cast<float>(z[lvl]);
+            const float pt = fmaf(t, t, part[lvl]);
+            const float c = static_cast<float>(z[lvl]) + off;
+            const float pc = fmaf(c, c, pn[lvl]);
+            if (pt > best || pc > kCoreN2) {
+                ++z[lvl];
+                continue;
+            }
+            if (lvl == 7) {
+                int sum = 0;
+#pragma unroll
+                for (int i = 0; i < 8; ++i) sum += z[i];
+                if ((sum & 1) == 0) {
+                    int C[8];
+#pragma unroll
+                    for (int i = 0; i < 8; ++i) C[i] = 2 * z[i] + coset;
+                    consider(C);
+                }
+                ++z[lvl];
+                continue;
+            }
+            part[lvl + 1] = pt;
+            pn[lvl + 1] = pc;
+            ++lvl;
+            bounds(lvl);
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) P[i] = bP[i];
+    return brank == 0x7FFFFFFF ? 0 : brank;
+}
 
 // shared-memory layout of the encode kernel (bytes)
 constexpr int kEncTileBytes = kTileMaxElems * 4;                      // 65536
@@ -253,6 +369,8 @@ __global__ void __launch_bounds__(kEncThreads, 1) k_encode(const __grid_constant
                 const int rk = core_rank(P, st1, st2);
                 if (rk >= 0) {
                     idxv = rk;
+                } else if (p.core_only) {
+                    idxv = nearest_core_point(X, P, st1, st2);
                 } else {
                     int R[8], Q[8];
                     best_escape_root(P, R);

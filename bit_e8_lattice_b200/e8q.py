@@ -40,7 +40,10 @@ class EncodeArgs(ctypes.Structure):
     _fields_ = [("kappa", ctypes.c_float), ("dequant", ctypes.c_int32), ("scale_in", ctypes.c_int32),
                 ("esc", ctypes.c_void_p), ("esc_cap", ctypes.c_int64), ("ovf", ctypes.c_void_p),
                 ("ovf_cap", ctypes.c_int64), ("esc_row_ptr", ctypes.c_void_p), ("ovf_row_ptr", ctypes.c_void_p),
-                ("counters", ctypes.c_void_p)]
+                ("counters", ctypes.c_void_p), ("flags", ctypes.c_int32), ("reserved", ctypes.c_int32)]
+
+
+ENCODE_CORE_ONLY = 1
 
 
 class EncodedC(ctypes.Structure):
@@ -212,7 +215,7 @@ class Encoder:
 
     def __init__(self, shapes: Sequence[tuple], signs: Sequence[torch.Tensor], in_dtype=torch.bfloat16,
                  rht_block=0, kappa: float = 1.0, dequant: str = "none", scale_in: bool = False,
-                 esc_cap: Optional[int] = None, ovf_cap: Optional[int] = None, device=None):
+                 esc_cap: Optional[int] = None, ovf_cap: Optional[int] = None, device=None, core_only: bool = False):
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.shapes = [(int(r), int(c)) for r, c in shapes]
         blocks = rht_block if isinstance(rht_block, (list, tuple)) else [rht_block] * len(self.shapes)
@@ -257,9 +260,11 @@ class Encoder:
             m.dequant = self.dequant[i].data_ptr() if self.dequant[i] is not None else None
         ws_bytes = lib().e8q_encode_workspace_bytes(self._mats, len(self.shapes))
         self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+        self.core_only = bool(core_only)
         self._args = EncodeArgs(self.kappa, self.dq, 1 if self.scale_in else 0, self.esc.data_ptr(), self.esc_cap,
                                 self.ovf.data_ptr(), self.ovf_cap, self.esc_row_ptr.data_ptr(),
-                                self.ovf_row_ptr.data_ptr(), self.counters.data_ptr())
+                                self.ovf_row_ptr.data_ptr(), self.counters.data_ptr(),
+                                ENCODE_CORE_ONLY if self.core_only else 0, 0)
 
     def __call__(self, weights: Sequence[torch.Tensor], scales: Optional[Sequence[torch.Tensor]] = None,
                  stream=None) -> EncodeResult:

@@ -135,7 +135,20 @@ typedef struct e8q_encode_args {
     int64_t* esc_row_ptr;      /* out: [total_rows + 1] CSR offsets into esc, or NULL */
     int64_t* ovf_row_ptr;      /* out: [total_rows + 1] CSR offsets into ovf, or NULL */
     e8q_counters* counters;    /* out: required */
+    int32_t flags;             /* E8Q_ENCODE_* bits; 0 = the projection of QAT */
+    int32_t reserved;          /* 0 */
 } e8q_encode_args;
+
+/* e8q_encode_args.flags */
+enum {
+    /* Core-clipped projection (E8-QAT Figure 2 (a): post-training quantisation
+     * initialises the latent weights from the fixed E8 core): every group
+     * takes the core point nearest to x (equal distances: the smaller core
+     * index) instead of the nearest E8 point, so the call writes indices only
+     * and no escape or overflow record (rho = 0).  The dequant outputs are
+     * those of the chosen core points. */
+    E8Q_ENCODE_CORE_ONLY = 1
+};
 
 /* One encoded matrix, as read by decode and GEMV. */
 typedef struct e8q_encoded {
@@ -209,8 +222,11 @@ size_t e8q_encode_workspace_bytes(const e8q_matrix* mats /* host [n_mats] */, in
  *   shortfall; row_ptr offsets are the true ones (they may pass the cap).
  * ws, ws_bytes: at least e8q_encode_workspace_bytes(); the call clears it.
  * Errors: E8Q_ERR_INVALID_ARG for NULL required pointers, bad shapes,
- *   block, dtype, kappa or misaligned buffers; E8Q_ERR_UNSUPPORTED for
- *   cols > 16384 or too many groups; E8Q_ERR_WORKSPACE; E8Q_ERR_CUDA.
+ *   block, dtype, kappa, flags or misaligned buffers; E8Q_ERR_UNSUPPORTED
+ *   for cols > 16384 or too many groups; E8Q_ERR_WORKSPACE; E8Q_ERR_CUDA.
+ * flags: E8Q_ENCODE_CORE_ONLY selects the core-clipped projection (then
+ *   esc / ovf may be NULL with zero capacity; the counters and row pointers
+ *   report no records).
  */
 e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_encode_args* args, void* ws,
                               size_t ws_bytes, e8q_stream stream);

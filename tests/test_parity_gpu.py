@@ -521,6 +521,74 @@ def test_moe_bank_full_size_sampled(e8q):
                      label=f"moe[{i}]")
 
 
+# ----------------------------------------------------------------------
+# core-clipped projection (Figure 2 (a): PTQ from the fixed core)
+# ----------------------------------------------------------------------
+def run_core(e8q, mats, signs, blocks=0, kappa=1.0, dequant="none", dtype=torch.bfloat16, scales=None):
+    ws = [dev_bf16(m) if dtype == torch.bfloat16 else dev(m.astype(np.float32)) for m in mats]
+    ss = [dev(s) for s in signs]
+    sc = [dev(s.astype(np.float32)) for s in scales] if scales is not None else None
+    enc = e8q.Encoder([w.shape for w in ws], ss, dtype, blocks, kappa, dequant, scales is not None, 64, 64,
+                      core_only=True)
+    res = enc(ws, sc)
+    torch.cuda.synchronize()
+    ctr = res.read_counters()
+    assert ctr["err"] == 0 and ctr["n_escape"] == 0 and ctr["n_overflow"] == 0 and ctr["n_dropped"] == 0, ctr
+    assert (res.esc_row_ptr.cpu().numpy() == 0).all() and (res.ovf_row_ptr.cpu().numpy() == 0).all()
+    return res
+
+
+def check_core(out, idx_gpu, label):
+    idx = np.asarray(idx_gpu).astype(np.int64).reshape(-1) & 0xFFFF
+    far = out["margin"] > MARGIN
+    bad = far & (idx != out["idx"])
+    assert not bad.any(), f"{label}: {bad.sum()} core indices differ above the margin, e.g. {np.nonzero(bad)[0][:5]}"
+    return int((~far).sum())
+
+
+@pytest.mark.parametrize("kappa", [1.0, 0.5, 3.0])
+def test_core_only_f32_matches_oracle(e8q, kappa):
+    """f32 256x256 (general kernel), kappa 1 (a quarter of the groups outside
+    the core), 0.5 (far outside: the exhaustive fallback) and 3 (almost all
+    inside): the nearest core point of every group clear of a tie, and the
+    scales of the unclipped projection."""
+    w, d = synth.small_f32()
+    res = run_core(e8q, [w], [d], 0, kappa, "rotated", torch.float32)
+    out = oracle.project_core(w.astype(np.float64), d, 256, kappa)
+    check_core(out, host_idx(res.idx[0]), f"core kappa {kappa}")
+    np.testing.assert_allclose(res.scale[0].cpu().numpy(), out["scale"], rtol=1e-5)
+    core = oracle.core_points().astype(np.int32)
+    P = core[host_idx(res.idx[0]).astype(np.int64).reshape(-1)]
+    check_rotated_dequant(res.dequant[0].cpu().view(torch.int16).numpy(), P, res.scale[0].cpu().numpy(), d, 256,
+                          "core rotated")
+
+
+def test_core_only_bf16_rows_and_original_basis(e8q):
+    """bf16 2048-wide rows (the general kernel takes the core-only calls) with
+    the original-basis dequant of the chosen core points."""
+    w, d = synth.attn_2048()
+    w = w[:96]
+    res = run_core(e8q, [w], [d], 0, 1.0, "original")
+    out = oracle.project_core(synth.bf16_bits_to_f64(w), d, 2048)
+    ties = check_core(out, host_idx(res.idx[0]), "core bf16")
+    assert ties < 50
+    core = oracle.core_points().astype(np.int32)
+    P = core[host_idx(res.idx[0]).astype(np.int64).reshape(-1)]
+    check_original_dequant(res.dequant[0].cpu().view(torch.int16).numpy(), P, res.scale[0].cpu().numpy(), d, 2048,
+                           "core original")
+
+
+def test_core_only_fixes_every_core_point(e8q):
+    """All 65,536 core points fed exactly (no transform, scale 1) with a
+    small perturbation map to themselves: rho = 0 at PTQ init."""
+    core = oracle.core_points().astype(np.float64) / 2.0
+    rng = np.random.default_rng(19)
+    x = (core + rng.uniform(-0.05, 0.05, core.shape)).astype(np.float32).reshape(-1, 64)
+    ones = np.ones(64, np.int8)
+    res = run_core(e8q, [x], [ones], 1, 1.0, "none", torch.float32, scales=[np.ones(x.shape[0])])
+    np.testing.assert_array_equal(host_idx(res.idx[0]).astype(np.int64).reshape(-1), np.arange(65536))
+
+
 def test_ste_backward_identity_on_mlp_gradient(e8q):
     """Identity STE (Figure 2 (b)): the dense-MLP step's seeded N(0, 1e-3^2)
     bf16 gradients of both matrices reach the latents bit for bit, copied
