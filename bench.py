@@ -47,6 +47,7 @@ D_MODEL, D_FF = 4096, 14336
 NOMINAL_HBM_GBS = 8000.0
 CSRC = os.path.join("bit_e8_lattice_b200", "csrc")
 FLUSH_BYTES = 256 << 20
+PAGES_DRIFT = 0.125  # drift of core-initialised latents, in units of the weights' std
 KERNEL_REPS = 20
 SAMPLE_UP, SAMPLE_DN = 2, 7  # oracle sample rows per step (1 : 3.5, the workload's proportion)
 
@@ -740,6 +741,39 @@ def main():
         workloads["moe_bank"] = {"groups": mg, "matrices": len(shapes), "escape_fraction": mc["n_escape"] / mg,
                                  "overflow_fraction": mc["n_overflow"] / mg}
         del menc, mres, MW, MS, bank
+
+        # PTQ initialisation from the fixed core (E8-QAT Figure 2 (a)): the
+        # core-clipped projection of the dense-MLP pair with its original-basis
+        # dequant, then the regime the pages train in: those latents plus a
+        # small drift (std PAGES_DRIFT x the weights' 0.015), encoded as in the step
+        penc = e8q.Encoder([(D_MODEL, D_FF), (D_FF, D_MODEL)], S, torch.bfloat16, 0, 1.0, "original",
+                           esc_cap=64, ovf_cap=64, core_only=True)
+        pres = penc(W)
+        torch.cuda.synchronize()
+        pc = pres.read_counters()
+        med, mean = time_flushed(lambda: penc(W), stream, flush, reps=3)
+        pbytes = G * (16 + 2 + 16) + rows * (4 + 16)
+        e = kernel_entry(pbytes, med, mean, peaks, groups=G,
+                         note="nearest of the 65,536 core points by ball enumeration (general kernel)")
+        e["timing"] = "median of 3, L2 flushed before each call"
+        kernels["ptq_core_projection"] = e
+        sigma = PAGES_DRIFT * 0.015
+        WP = [(pres.dequant[i].float() + sigma * torch.from_numpy(synth.latent_drift(tuple(pres.dequant[i].shape),
+                                                                                     matrix=i)).to(dev)).bfloat16()
+              for i in range(2)]
+        del penc, pres
+        qenc = e8q.Encoder([(D_MODEL, D_FF), (D_FF, D_MODEL)], S, torch.bfloat16, 0, 1.0, "original",
+                           esc_cap=G // 2, ovf_cap=G // 16)
+        qres = qenc(WP)
+        torch.cuda.synchronize()
+        qc = qres.read_counters()
+        med, mean = time_flushed(lambda: qenc(WP), stream, flush)
+        qbytes = G * (16 + 2 + 16) + rows * (4 + 16) + 8 * qc["n_escape"] + 20 * qc["n_overflow"]
+        kernels["pages_regime_project_encode"] = kernel_entry(qbytes, med, mean, peaks, groups=G)
+        workloads["pages_regime"] = {
+            "groups": G, "drift_std_over_weight_std": PAGES_DRIFT, "core_points_clipped": pc["n_escape"] == 0,
+            "escape_fraction": qc["n_escape"] / G, "overflow_fraction": qc["n_overflow"] / G}
+        del qenc, qres, WP
     del flush
     torch.cuda.empty_cache()
 

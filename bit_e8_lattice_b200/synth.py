@@ -18,6 +18,9 @@ row-major.  Workloads (named by what they are):
                      from U(0.5, 2), seed 3.
 * ``mlp_14336``      up 4096x14336 and down 14336x4096 bf16, N(0, 0.015^2),
                      seed 4; upstream gradient N(0, 1e-3^2) bf16, seed 40.
+* ``latent_drift``   float32 N(0, 1) [rows][cols], seed [41, matrix]: the
+                     drift of latents initialised from the E8 core (the
+                     caller scales it, e.g. by 0.15 x the weights' 0.015).
 * ``gemv_x``         activations [batch][cols] bf16, N(0, 1), seed 5.
 """
 from __future__ import annotations
@@ -101,6 +104,13 @@ def mlp_14336(seed: int = 4, d_model: int = 4096, d_ff: int = 14336):
 def mlp_grad(shape, seed: int = 40, matrix: int = 0) -> np.ndarray:
     rng = np.random.default_rng([seed, matrix])
     return f64_to_bf16_bits(rng.standard_normal(shape) * 1e-3)
+
+
+def latent_drift(shape, seed: int = 41, matrix: int = 0) -> np.ndarray:
+    """Unit-variance drift directions for the latents of a core-initialised
+    model: float32 N(0, 1), scaled by the caller."""
+    rng = np.random.default_rng([seed, matrix])
+    return rng.standard_normal(shape, dtype=np.float32)
 
 
 def gemv_x(batch: int, cols: int, seed: int = 5) -> np.ndarray:

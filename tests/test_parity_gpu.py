@@ -434,6 +434,41 @@ def test_gemv_large_activations(e8q, gemv_path):
     assert rel < 1e-2, rel
 
 
+def test_gemv_repeatable(e8q, gemv_path):
+    """The partial sums are added in a fixed order: two calls on the same
+    inputs give the same bits."""
+    rng = np.random.default_rng(21)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((700, 4096)) * 0.02)
+    d = synth.signs(21, 4096)
+    enc, res = run_encode(e8q, [w], [d], 0)
+    xb = synth.gemv_x(5, 4096)
+    g = e8q.Gemv(res.encoded[0], 5)
+    y1 = g(dev_bf16(xb)).clone()
+    y2 = g(dev_bf16(xb)).clone()
+    torch.cuda.synchronize()
+    assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
+
+
+def test_gemv_far_overflow_points(e8q, gemv_path):
+    """A scale far below the rows' rms (s = rms / kappa, kappa 50) makes
+    every group an overflow record, most with doubled coordinates beyond
+    +-127; the GEMV applies those records from their 16-bit coordinates."""
+    rng = np.random.default_rng(31)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((160, 1024)) * 0.02)
+    d = synth.signs(31, 1024)
+    B = oracle.default_block(1024)
+    enc, res = run_encode(e8q, [w], [d], 0, kappa=50.0, esc_cap=160 * 128, ovf_cap=160 * 128)
+    st = compare_all(e8q, res, [w], [d], [B], kappa=50.0, label="gemv_farP")[0]
+    P = st["points"]
+    assert (np.abs(P) > 127).any(axis=1).sum() > 10000
+    for batch in (3, 70):
+        xb = synth.gemv_x(batch, 1024)
+        y = e8q.Gemv(res.encoded[0], batch)(dev_bf16(xb))
+        torch.cuda.synchronize()
+        y_ref = oracle.gemv(P, res.scale[0].cpu().numpy().astype(np.float64), d, B, synth.bf16_bits_to_f64(xb))
+        check_gemv(y.cpu().view(torch.int16).numpy(), y_ref, f"gemv far points b={batch}")
+
+
 # ----------------------------------------------------------------------
 # full-size workloads, in the launch configuration bench.py times
 # ----------------------------------------------------------------------
