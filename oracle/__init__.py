@@ -292,6 +292,90 @@ def fwht(u: np.ndarray) -> np.ndarray:
 
 
 # --------------------------------------------------------------------------
+# Shape-gain variant (SQuAT page, "shape and scale split" section): every
+# weight vector splits into a unit direction, quantised against a spherical
+# E8 codebook, and a scalar gain through a low-bit scalar quantiser.  The
+# page fixes neither the codebook shell nor the gain grid; the readings
+# taken here: the direction codebook is the 2160-point shell |p|^2 = 4
+# (the core's indices 241 .. 2400, direction index = core index - 241,
+# 12 bits); the gain g = |x| of the row-normalised group goes through a
+# 16-level uniform quantiser on [0, 6): level k = min(15, floor(g / D)),
+# D = 6 / 16, value (k + 1/2) D; code = k << 12 | direction (16 bits a
+# group, 2 bits a weight).  The reconstruction is (k + 1/2) D * c / |c|.
+# --------------------------------------------------------------------------
+SG_SHELL_FIRST = 241      # core index of the first |p|^2 = 4 point
+SG_SHELL_SIZE = 2160
+SG_LEVELS = 16
+SG_GAIN_MAX = 6.0
+SG_STEP = SG_GAIN_MAX / SG_LEVELS
+
+
+def sg_shell() -> np.ndarray:
+    """The 2160 directions: doubled points of the |p|^2 = 4 shell in core
+    (lex) order."""
+    return core_points()[SG_SHELL_FIRST:SG_SHELL_FIRST + SG_SHELL_SIZE].astype(np.int64)
+
+
+def sg_encode_vectors(x: np.ndarray):
+    """Direction = the shell point of largest inner product with x (all
+    shell points have one norm, so this is the nearest direction; equal
+    products go to the smaller index), found by scoring all 2160; gain
+    level from |x|.  Returns code, direction, level, margin (the gap between
+    the best and second-best cosine)."""
+    x = np.asarray(x, np.float64).reshape(-1, 8)
+    S = sg_shell().astype(np.float64)
+    score = x @ S.T                              # <x, P>, |P| = 4
+    d = np.argmax(score, axis=1)
+    top = np.take_along_axis(score, d[:, None], 1)[:, 0]
+    score[np.arange(len(d)), d] = -np.inf
+    second = score.max(axis=1)
+    n = np.sqrt((x * x).sum(axis=1))
+    margin = np.where(n > 0, (top - second) / (4.0 * np.where(n > 0, n, 1.0)), 0.0)
+    k = np.minimum(SG_LEVELS - 1, np.floor(n / SG_STEP)).astype(np.int64)
+    return (k << 12) | d, d, k, margin
+
+
+def sg_points(code: np.ndarray) -> np.ndarray:
+    """x-hat of each code: (k + 1/2) D * P / 4 (float64 [G][8])."""
+    code = np.asarray(code, np.int64).reshape(-1)
+    S = sg_shell().astype(np.float64)
+    k = code >> 12
+    return ((k + 0.5) * SG_STEP)[:, None] * S[code & 0xFFF] / 4.0
+
+
+def _bf16_rne(v: np.ndarray) -> np.ndarray:
+    """Round float64 to bf16 bits once, half to even (finite values)."""
+    f = np.asarray(v, np.float64)
+    m, e = np.frexp(f)                       # f = m 2^e, |m| in [0.5, 1)
+    q = np.ldexp(np.rint(np.ldexp(m, 8)), e - 8)   # 8 significant bits, ties to even
+    u = q.astype(np.float32).view(np.uint32)     # exact: q has 8 bits
+    return (u >> np.uint32(16)).astype(np.uint16)
+
+
+def sg_dequant(xhat: np.ndarray, scale: np.ndarray, signs: np.ndarray, block: int, basis: str):
+    """bf16 bits of s * x-hat (basis 'rotated') or of d * H_B(s * x-hat) / sqrt(B)
+    (basis 'original', the STE forward in the weights' own basis)."""
+    scale = np.asarray(scale, np.float64)
+    R = scale.shape[0]
+    xh = np.asarray(xhat, np.float64).reshape(R, -1)
+    v = scale[:, None] * xh
+    if basis == "original":
+        C = xh.shape[1]
+        v = rht_vectors(v, np.ones(C, np.int8), block) * np.asarray(signs, np.float64).reshape(1, C)
+    return _bf16_rne(v), v
+
+
+def sg_project_encode(w: np.ndarray, signs: np.ndarray, block: int, kappa: float = 1.0):
+    """The shape-gain pipeline on one matrix: sign flip, blockwise RHT, row
+    scale (as for the lattice projection), then the shape-gain code of every
+    8-group."""
+    out = project_encode(w, signs, block, kappa, want_x=True, want_margin=False)
+    code, d, k, margin = sg_encode_vectors(out["x"])
+    return dict(scale=out["scale"], x=out["x"], code=code, dir=d, level=k, margin=margin,
+                xhat=sg_points(code))
+
+
+# --------------------------------------------------------------------------
 # Payload accounting (Table 10; Figure 6 (c))
 # --------------------------------------------------------------------------
 def payload_bits_pages(rho: float) -> float:

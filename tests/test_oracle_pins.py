@@ -499,3 +499,113 @@ def test_project_core_rows_scale_and_no_records(orc):
     np.testing.assert_array_equal(core["idx"][clear], k[clear])
     kept = full["kind"] == 0
     np.testing.assert_array_equal(core["idx"][kept & clear], full["idx"][kept & clear])
+
+
+# ----------------------------------------------------------------------
+# shape-gain variant (SQuAT page, "shape and scale split")
+# ----------------------------------------------------------------------
+def structured_direction(x):
+    """Best |p|^2 = 4 shell point for one vector by the shell's three
+    families (doubled coordinates): +-4 e_i; +-2 on four coordinates; odd
+    coordinates with one +-3 and a coordinate sum divisible by 4.  Written
+    from the shell's structure, independent of the oracle's scoring."""
+    ax = np.abs(x)
+    sg = np.where(x < 0, -1, 1)
+    best = []
+    i = int(np.argmax(ax))
+    P = np.zeros(8, np.int64)
+    P[i] = 4 * sg[i]
+    best.append(P)
+    top = np.argsort(-ax, kind="stable")[:4]
+    P = np.zeros(8, np.int64)
+    P[top] = 2 * sg[top]
+    best.append(P)
+    for j in range(8):  # position of the +-3
+        for flip in range(-1, 8):  # no flip, or the coordinate whose sign is reversed
+            P = sg.astype(np.int64).copy()
+            P[j] *= 3
+            if flip >= 0:
+                P[flip] = -P[flip]
+            if P.sum() % 4 == 0:
+                best.append(P)
+    scores = [float(x @ P) for P in best]
+    return best[int(np.argmax(scores))], max(scores)
+
+
+def test_sg_shell_is_the_norm4_shell(orc):
+    S = orc.sg_shell()
+    P, n2 = np_e8_points(16)
+    ref = P[n2 == 16]
+    assert S.shape == (2160, 8) and (S == ref).all()
+    assert orc.rank(S[0]) == orc.SG_SHELL_FIRST and orc.rank(S[-1]) == orc.SG_SHELL_FIRST + 2159
+    # the shell's families: 16 of type +-4 e_i, 1120 of type (+-2)^4, 1024 odd
+    a = np.abs(S)
+    assert ((a == 4).sum(1) == 1).sum() == 16
+    assert ((a == 2).sum(1) == 4).sum() == 1120
+    assert ((a % 2 == 1).all(1)).sum() == 1024
+
+
+def test_sg_direction_matches_structured_search(orc):
+    rng = np.random.default_rng(77)
+    x = rng.standard_normal((3000, 8)) * rng.uniform(0.2, 4.0, (3000, 1))
+    code, d, k, margin = orc.sg_encode_vectors(x)
+    S = orc.sg_shell()
+    checked = 0
+    for i in range(len(x)):
+        P, sc = structured_direction(x[i])
+        assert abs(sc - float(x[i] @ S[d[i]])) <= 1e-9 * (1 + abs(sc))
+        if margin[i] > 1e-9:
+            assert (P == S[d[i]]).all()
+            checked += 1
+    assert checked > 2900
+
+
+def test_sg_direction_fixed_points_symmetry_and_scale(orc):
+    S = orc.sg_shell()
+    code, d, k, m = orc.sg_encode_vectors(S / 2.0)
+    assert (d == np.arange(2160)).all() and (k == 5).all()  # |p| = 2 -> floor(2 / 0.375) = 5
+    rng = np.random.default_rng(5)
+    x = rng.standard_normal((500, 8))
+    _, d1, _, m1 = orc.sg_encode_vectors(x)
+    _, d2, _, _ = orc.sg_encode_vectors(3.7 * x)
+    _, d3, _, _ = orc.sg_encode_vectors(-x)
+    ok = m1 > 1e-9
+    assert (d1[ok] == d2[ok]).all()
+    # -x picks -P
+    assert (S[d3[ok]] == -S[d1[ok]]).all()
+
+
+def test_sg_gain_levels_and_reconstruction(orc):
+    D = orc.SG_STEP
+    assert D == 0.375 and orc.SG_LEVELS == 16
+    u = np.zeros((20, 8))
+    u[:, 0] = 1.0
+    g = np.array([0.0, 0.1, 0.374, 0.376, 1.0, 2.9, 5.99, 6.0, 7.5, 100.0] + [0.375 * j + 0.1 for j in range(10)])
+    code, d, k, _ = orc.sg_encode_vectors(u * g[:, None])
+    want = np.minimum(15, np.floor(g / D)).astype(np.int64)
+    assert (k == want).all() and ((code >> 12) == want).all()
+    xh = orc.sg_points(code)
+    assert np.allclose(np.sqrt((xh * xh).sum(1)), (want + 0.5) * D)  # |P| / 4 = 1
+    # the direction of x-hat is the chosen shell point
+    S = orc.sg_shell().astype(np.float64)
+    assert np.allclose(xh, ((want + 0.5) * D)[:, None] * S[code & 0xFFF] / 4)
+
+
+def test_sg_dequant_bases(orc):
+    rng = np.random.default_rng(9)
+    R, C, B = 3, 64, 16
+    w = rng.standard_normal((R, C)) * 0.02
+    d = np.where(rng.random(C) < 0.5, -1, 1).astype(np.int8)
+    out = orc.sg_project_encode(w, d, B)
+    s32 = out["scale"].astype(np.float32).astype(np.float64)
+    rot_bits, rot = orc.sg_dequant(out["xhat"], s32, d, B, "rotated")
+    assert np.array_equal(rot, s32[:, None] * out["xhat"].reshape(R, C))
+    assert all(bf16_neighbours_ok(v, b) for v, b in zip(rot.ravel(), rot_bits.ravel()))
+    orig_bits, orig = orc.sg_dequant(out["xhat"], s32, d, B, "original")
+    H = scipy.linalg.hadamard(B) / math.sqrt(B)
+    ref = (s32[:, None] * out["xhat"].reshape(R, C)).reshape(R, C // B, B) @ H.T
+    assert np.allclose(orig, ref.reshape(R, C) * d[None, :], rtol=0, atol=1e-15)
+    assert all(bf16_neighbours_ok(v, b) for v, b in zip(orig.ravel(), orig_bits.ravel()))
+    # the round trip: rotating the original-basis reconstruction back gives s * x-hat
+    back = orc.rht_vectors(orig, d, B)
+    assert np.allclose(back, s32[:, None] * out["xhat"].reshape(R, C), atol=1e-15)
