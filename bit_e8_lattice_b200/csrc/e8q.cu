@@ -294,11 +294,13 @@ e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_
         (a->ovf_cap > 0 && (!a->ovf || !aligned(a->ovf, 4))))
         return E8Q_ERR_INVALID_ARG;
     if (a->scale_in != 0 && a->scale_in != 1) return E8Q_ERR_INVALID_ARG;
-    if ((a->flags & ~E8Q_ENCODE_CORE_ONLY) != 0 || a->reserved != 0) return E8Q_ERR_INVALID_ARG;
+    if ((a->flags & ~(E8Q_ENCODE_CORE_ONLY | E8Q_ENCODE_SHAPE_GAIN)) != 0 || a->reserved != 0 ||
+        a->flags == (E8Q_ENCODE_CORE_ONLY | E8Q_ENCODE_SHAPE_GAIN))
+        return E8Q_ERR_INVALID_ARG;
 
     static thread_local EncodeParams<kMaxMats> P;  // ~28 KB: keep it off the stack
     std::memset(&P, 0, sizeof(P));
-    bool fast = (a->flags & E8Q_ENCODE_CORE_ONLY) == 0;  // the core-clipped projection runs in the general kernel
+    bool fast = a->flags == 0;  // the core-clipped projection and the shape-gain code run in the general kernel
     for (int i = 0; i < n_mats; ++i) {
         const int logb = resolve_logb(mats[i].cols, mats[i].rht_block);
         if (!valid_cols(mats[i].cols) || mats[i].cols > kMaxCols || logb < 0 ||
@@ -369,6 +371,7 @@ e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_
     P.n_tiles = static_cast<int32_t>(tiles);
     P.total_rows = static_cast<int32_t>(rows_total);
     P.core_only = (a->flags & E8Q_ENCODE_CORE_ONLY) ? 1 : 0;
+    P.shape_gain = (a->flags & E8Q_ENCODE_SHAPE_GAIN) ? 1 : 0;
     {  // |2x| <= 2 kappa sqrt(cols): clamp coordinates only when that could pass 2^14
         int64_t maxc = 0;
         for (int i = 0; i < n_mats; ++i) maxc = mats[i].cols > maxc ? mats[i].cols : maxc;
@@ -626,7 +629,9 @@ extern "C" e8q_status e8q_project_encode_noalloc(const e8q_matrix* mats, int32_t
         (a->ovf_cap > 0 && (!a->ovf || !aligned(a->ovf, 4))))
         return E8Q_ERR_INVALID_ARG;
     if (a->scale_in != 0 && a->scale_in != 1) return E8Q_ERR_INVALID_ARG;
-    if ((a->flags & ~E8Q_ENCODE_CORE_ONLY) != 0 || a->reserved != 0) return E8Q_ERR_INVALID_ARG;
+    if ((a->flags & ~(E8Q_ENCODE_CORE_ONLY | E8Q_ENCODE_SHAPE_GAIN)) != 0 || a->reserved != 0 ||
+        a->flags == (E8Q_ENCODE_CORE_ONLY | E8Q_ENCODE_SHAPE_GAIN))
+        return E8Q_ERR_INVALID_ARG;
 
     static thread_local EncodeParams<kMaxMats> P;
     std::memset(&P, 0, sizeof(P));
@@ -703,6 +708,7 @@ extern "C" e8q_status e8q_project_encode_noalloc(const e8q_matrix* mats, int32_t
     P.n_tiles = static_cast<int32_t>(tiles);
     P.total_rows = static_cast<int32_t>(rows_total);
     P.core_only = (a->flags & E8Q_ENCODE_CORE_ONLY) ? 1 : 0;
+    P.shape_gain = (a->flags & E8Q_ENCODE_SHAPE_GAIN) ? 1 : 0;
     const int grid = static_cast<int>(tiles < g_sms[dev] ? tiles : g_sms[dev]);
     if (n_mats == 1) {
         EncodeParams<1> P1;

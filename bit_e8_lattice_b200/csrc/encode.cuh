@@ -34,9 +34,103 @@ struct EncodeParams {
     int32_t n_tiles;
     int32_t total_rows;
     int32_t clamp;      // fast kernel: inputs may reach |2x| >= 2^14 (given scales or large kappa)
-    int32_t core_only;  // the core-clipped projection (E8Q_ENCODE_CORE_ONLY)
+    int32_t core_only;   // the core-clipped projection (E8Q_ENCODE_CORE_ONLY)
+    int32_t shape_gain;  // the shape-gain code (E8Q_ENCODE_SHAPE_GAIN)
     MatDesc m[MAXM];
 };
+
+// Shape-gain code of X = 2x (SQuAT page, "shape and scale split": a unit
+// direction quantised against a spherical E8 codebook, a scalar gain
+// through a low-bit scalar quantiser).  Directions: the 2160 points of the
+// |p|^2 = 4 shell, core indices kSgShellFirst .. + 2159; the best is the one
+// of largest <X, P>, taken per family of the shell (doubled coordinates):
+//   +-4 e_i                       4 max |X_i|
+//   +-2 on four coordinates       2 (sum of the four largest |X_i|)
+//   odd, one +-3, sum = 0 mod 4   sum |X_i| + 2 |X_j| for the +-3 at j, less
+//                                 the cheapest sign reversal when the number
+//                                 of negative X_i is even (the sum rule):
+//                                 2 |X_i| for a +-1, 6 |X_j| for the +-3.
+// Gain level k = min(15, floor(|x| / (6 / 16))).  On return P holds the
+// direction's doubled point and *xm the factor (k + 1/2) (6 / 16) / 4 that
+// maps P to the reconstruction x-hat = xm P; the result is k << 12 | the
+// direction's index in the shell.
+constexpr int kSgShellFirst = 241;
+constexpr float kSgStep = 6.0f / 16.0f;
+
+__device__ __noinline__ int shape_gain_code(const float (&X)[8], int (&P)[8], float* xm, const uint16_t* __restrict__ st1,
+                                            const uint16_t* __restrict__ st2) {
+    float a[8];
+    float n2 = 0.f, total = 0.f;
+    int neg = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        a[i] = fabsf(X[i]);
+        n2 = fmaf(X[i], X[i], n2);
+        total += a[i];
+        neg += X[i] < 0.f;
+    }
+    // family +-4 e_i; the four largest |X_i| (rank by value, then position);
+    // the two smallest
+    int imax = 0, imin = 0, imin2 = -1;
+    float top4 = 0.f;
+    unsigned in4 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (a[i] > a[imax]) imax = i;
+        int r = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) r += (a[k] > a[i]) || (a[k] == a[i] && k < i);
+        if (r < 4) {
+            top4 += a[i];
+            in4 |= 1u << i;
+        }
+        if (a[i] < a[imin]) imin = i;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        if (i != imin && (imin2 < 0 || a[i] < a[imin2])) imin2 = i;
+    const float sA = 4.f * a[imax], sB = 2.f * top4;
+    // odd family: the +-3 at j
+    float sC = -INFINITY;
+    int jC = 0, fC = -1;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float sc = total + 2.f * a[j];
+        int f = -1;
+        if ((neg & 1) == 0) {
+            const int o = (j == imin) ? imin2 : imin;  // smallest |X_i|, i != j
+            const float c1 = 2.f * a[o], c3 = 6.f * a[j];
+            if (c3 < c1) {
+                sc -= c3;
+                f = j;
+            } else {
+                sc -= c1;
+                f = o;
+            }
+        }
+        if (sc > sC) {
+            sC = sc;
+            jC = j;
+            fC = f;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int sg = X[i] < 0.f ? -1 : 1;
+        if (sA >= sB && sA >= sC) {
+            P[i] = i == imax ? 4 * sg : 0;
+        } else if (sB >= sC) {
+            P[i] = ((in4 >> i) & 1u) ? 2 * sg : 0;
+        } else {
+            const int v = (i == jC ? 3 : 1) * sg;
+            P[i] = i == fC ? -v : v;
+        }
+    }
+    const float g = 0.5f * sqrtf(n2);
+    const int k = min(15, static_cast<int>(floorf(g / kSgStep)));
+    *xm = (static_cast<float>(k) + 0.5f) * kSgStep * 0.25f;
+    return (k << 12) | (core_rank(P, st1, st2) - kSgShellFirst);
+}
 
 // Nearest core point of X = 2x whose nearest E8 point P lies outside the
 // core ("E8-QAT", Figure 2 (a): post-training quantisation starts from the
@@ -356,6 +450,7 @@ __global__ void __launch_bounds__(kEncThreads, 1) k_encode(const __grid_constant
             const int g = base + tid;
             int kind = 0, idxv = 0, rootv = 0;
             int P[8];
+            float xm = 0.5f;  // x-hat = xm P: the lattice point p = P / 2, or the shape-gain reconstruction
             if (g < G) {
                 const int r = g / gpr;
                 const float c = s_rowc[r];
@@ -365,40 +460,45 @@ __global__ void __launch_bounds__(kEncThreads, 1) k_encode(const __grid_constant
                 float X[8];
 #pragma unroll
                 for (int i = 0; i < 8; ++i) X[i] = fminf(fmaxf(fmaf(vv[i], c, 0.f), -1048576.f), 1048576.f);
-                e8_nearest_doubled(X, P);
-                const int rk = core_rank(P, st1, st2);
-                if (rk >= 0) {
-                    idxv = rk;
-                } else if (p.core_only) {
-                    idxv = nearest_core_point(X, P, st1, st2);
+                if (p.shape_gain) {
+                    idxv = shape_gain_code(X, P, &xm, st1, st2);
                 } else {
-                    int R[8], Q[8];
-                    best_escape_root(P, R);
-#pragma unroll
-                    for (int i = 0; i < 8; ++i) Q[i] = P[i] - R[i];
-                    const int rq = core_rank(Q, st1, st2);
-                    if (rq >= 0) {
-                        kind = 1;
-                        idxv = rq;
-                        rootv = core_rank(R, st1, st2) - 1;
+                    e8_nearest_doubled(X, P);
+                    const int rk = core_rank(P, st1, st2);
+                    if (rk >= 0) {
+                        idxv = rk;
+                    } else if (p.core_only) {
+                        idxv = nearest_core_point(X, P, st1, st2);
                     } else {
-                        kind = 2;
+                        int R[8], Q[8];
+                        best_escape_root(P, R);
+#pragma unroll
+                        for (int i = 0; i < 8; ++i) Q[i] = P[i] - R[i];
+                        const int rq = core_rank(Q, st1, st2);
+                        if (rq >= 0) {
+                            kind = 1;
+                            idxv = rq;
+                            rootv = core_rank(R, st1, st2) - 1;
+                        } else {
+                            kind = 2;
+                        }
                     }
                 }
                 M.idx[gbase_local + g] = static_cast<uint16_t>(idxv);
                 if (p.dq_mode == E8Q_DEQUANT_ROTATED) {
                     const float s = s_rows[r];
                     uint4 o;
-                    o.x = pack_bf16x2(bf16_of_product(s, 0.5f * P[0]), bf16_of_product(s, 0.5f * P[1]));
-                    o.y = pack_bf16x2(bf16_of_product(s, 0.5f * P[2]), bf16_of_product(s, 0.5f * P[3]));
-                    o.z = pack_bf16x2(bf16_of_product(s, 0.5f * P[4]), bf16_of_product(s, 0.5f * P[5]));
-                    o.w = pack_bf16x2(bf16_of_product(s, 0.5f * P[6]), bf16_of_product(s, 0.5f * P[7]));
+                    o.x = pack_bf16x2(bf16_of_product(s, xm * P[0]), bf16_of_product(s, xm * P[1]));
+                    o.y = pack_bf16x2(bf16_of_product(s, xm * P[2]), bf16_of_product(s, xm * P[3]));
+                    o.z = pack_bf16x2(bf16_of_product(s, xm * P[4]), bf16_of_product(s, xm * P[5]));
+                    o.w = pack_bf16x2(bf16_of_product(s, xm * P[6]), bf16_of_product(s, xm * P[7]));
                     reinterpret_cast<uint4*>(static_cast<uint16_t*>(M.dq) + static_cast<size_t>(r0) * C)[g] = o;
                 } else if (p.dq_mode == E8Q_DEQUANT_ORIGINAL) {
-                    // p itself; H(p) stays exact in fp32 and is scaled once afterwards
+                    // x-hat itself (p, or the shape-gain reconstruction); H of it stays
+                    // exact in fp32 and is scaled once afterwards
                     float4* dst = reinterpret_cast<float4*>(tile) + 2 * g;
-                    dst[0] = make_float4(0.5f * P[0], 0.5f * P[1], 0.5f * P[2], 0.5f * P[3]);
-                    dst[1] = make_float4(0.5f * P[4], 0.5f * P[5], 0.5f * P[6], 0.5f * P[7]);
+                    dst[0] = make_float4(xm * P[0], xm * P[1], xm * P[2], xm * P[3]);
+                    dst[1] = make_float4(xm * P[4], xm * P[5], xm * P[6], xm * P[7]);
                 }
             }
             const unsigned be = __ballot_sync(0xFFFFFFFFu, kind == 1);

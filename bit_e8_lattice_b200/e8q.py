@@ -44,6 +44,7 @@ class EncodeArgs(ctypes.Structure):
 
 
 ENCODE_CORE_ONLY = 1
+ENCODE_SHAPE_GAIN = 2
 
 
 class EncodedC(ctypes.Structure):
@@ -215,7 +216,8 @@ class Encoder:
 
     def __init__(self, shapes: Sequence[tuple], signs: Sequence[torch.Tensor], in_dtype=torch.bfloat16,
                  rht_block=0, kappa: float = 1.0, dequant: str = "none", scale_in: bool = False,
-                 esc_cap: Optional[int] = None, ovf_cap: Optional[int] = None, device=None, core_only: bool = False):
+                 esc_cap: Optional[int] = None, ovf_cap: Optional[int] = None, device=None, core_only: bool = False,
+                 shape_gain: bool = False):
         self.device = torch.device(device) if device is not None else torch.device("cuda", torch.cuda.current_device())
         self.shapes = [(int(r), int(c)) for r, c in shapes]
         blocks = rht_block if isinstance(rht_block, (list, tuple)) else [rht_block] * len(self.shapes)
@@ -261,10 +263,11 @@ class Encoder:
         ws_bytes = lib().e8q_encode_workspace_bytes(self._mats, len(self.shapes))
         self.workspace = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
         self.core_only = bool(core_only)
+        self.shape_gain = bool(shape_gain)
         self._args = EncodeArgs(self.kappa, self.dq, 1 if self.scale_in else 0, self.esc.data_ptr(), self.esc_cap,
                                 self.ovf.data_ptr(), self.ovf_cap, self.esc_row_ptr.data_ptr(),
                                 self.ovf_row_ptr.data_ptr(), self.counters.data_ptr(),
-                                ENCODE_CORE_ONLY if self.core_only else 0, 0)
+                                (ENCODE_CORE_ONLY if self.core_only else 0) | (ENCODE_SHAPE_GAIN if self.shape_gain else 0), 0)
 
     def __call__(self, weights: Sequence[torch.Tensor], scales: Optional[Sequence[torch.Tensor]] = None,
                  stream=None) -> EncodeResult:

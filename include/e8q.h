@@ -147,7 +147,20 @@ enum {
      * index) instead of the nearest E8 point, so the call writes indices only
      * and no escape or overflow record (rho = 0).  The dequant outputs are
      * those of the chosen core points. */
-    E8Q_ENCODE_CORE_ONLY = 1
+    E8Q_ENCODE_CORE_ONLY = 1,
+    /* Shape-gain code (SQuAT page, "shape and scale split": each weight
+     * vector splits into a unit direction, quantised against a spherical E8
+     * codebook, and a scalar gain through a low-bit scalar quantiser).  After
+     * the same sign flip, RHT and row scale, each group x gets the 16-bit
+     * code k << 12 | d: d (0 .. 2159) the index, in lexicographic order, of
+     * the |p|^2 = 4 shell point c of largest <x, c> (the nearest direction;
+     * core index 241 + d), k = min(15, floor(|x| / (6 / 16))) the gain level.
+     * The reconstruction is x-hat = (k + 1/2) (6 / 16) c / |c|; the dequant
+     * outputs are those of x-hat (rotated: bf16(s x-hat); original:
+     * bf16(d (.) H_B (s x-hat) / sqrt(B))).  No escape or overflow record is
+     * written.  Not combinable with E8Q_ENCODE_CORE_ONLY; decode and GEMV
+     * read the lattice encoding only. */
+    E8Q_ENCODE_SHAPE_GAIN = 2
 };
 
 /* One encoded matrix, as read by decode and GEMV. */
@@ -224,9 +237,10 @@ size_t e8q_encode_workspace_bytes(const e8q_matrix* mats /* host [n_mats] */, in
  * Errors: E8Q_ERR_INVALID_ARG for NULL required pointers, bad shapes,
  *   block, dtype, kappa, flags or misaligned buffers; E8Q_ERR_UNSUPPORTED
  *   for cols > 16384 or too many groups; E8Q_ERR_WORKSPACE; E8Q_ERR_CUDA.
- * flags: E8Q_ENCODE_CORE_ONLY selects the core-clipped projection (then
- *   esc / ovf may be NULL with zero capacity; the counters and row pointers
- *   report no records).
+ * flags: E8Q_ENCODE_CORE_ONLY selects the core-clipped projection,
+ *   E8Q_ENCODE_SHAPE_GAIN the shape-gain code (either way esc / ovf may be
+ *   NULL with zero capacity; the counters and row pointers report no
+ *   records); both together are INVALID_ARG.
  */
 e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_encode_args* args, void* ws,
                               size_t ws_bytes, e8q_stream stream);

@@ -735,3 +735,95 @@ def test_gather_encoded_nccl_one_rank(e8q):
     y_ref = oracle.gemv(st["points"], out[1].cpu().numpy().astype(np.float64), d, 2048,
                         synth.bf16_bits_to_f64(synth.gemv_x(4, 2048)))
     check_gemv(y.cpu().view(torch.int16).numpy(), y_ref, "gathered GEMV")
+
+
+# ----------------------------------------------------------------------
+# shape-gain code (SQuAT page, "shape and scale split")
+# ----------------------------------------------------------------------
+def run_shape_gain(e8q, mats, signs, blocks=0, kappa=1.0, dequant="none", dtype=torch.bfloat16):
+    ws = [dev_bf16(m) if dtype == torch.bfloat16 else dev(m.astype(np.float32)) for m in mats]
+    ss = [dev(s) for s in signs]
+    enc = e8q.Encoder([w.shape for w in ws], ss, dtype, blocks, kappa, dequant, False, 64, 64, shape_gain=True)
+    res = enc(ws)
+    torch.cuda.synchronize()
+    ctr = res.read_counters()
+    assert ctr["err"] == 0 and ctr["n_escape"] == 0 and ctr["n_overflow"] == 0 and ctr["n_dropped"] == 0, ctr
+    assert (res.esc_row_ptr.cpu().numpy() == 0).all() and (res.ovf_row_ptr.cpu().numpy() == 0).all()
+    return res
+
+
+def check_shape_gain(out, code_gpu, label):
+    """Directions equal wherever the best shell point leads the second by
+    more than the tie margin; gain levels equal wherever |x| / (6/16) is not
+    within 1e-4 of a level boundary.  Returns the near-tie count."""
+    code = np.asarray(code_gpu).astype(np.int64).reshape(-1) & 0xFFFF
+    far = out["margin"] > MARGIN
+    bad = far & ((code & 0xFFF) != out["dir"])
+    assert not bad.any(), f"{label}: {bad.sum()} directions differ above the margin, e.g. {np.nonzero(bad)[0][:5]}"
+    assert ((code & 0xFFF) < 2160).all()
+    n = np.sqrt((out["x"].reshape(-1, 8) ** 2).sum(1)) / oracle.SG_STEP
+    clear = np.abs(n - np.rint(n)) > 1e-4
+    bad = clear & ((code >> 12) != out["level"])
+    assert not bad.any(), f"{label}: {bad.sum()} gain levels differ away from a boundary"
+    return int((~far).sum())
+
+
+@pytest.mark.parametrize("kappa", [1.0, 3.0])
+def test_shape_gain_f32_matches_oracle(e8q, kappa):
+    """f32 256x256 (block 256): every direction clear of a tie and every
+    gain level clear of a boundary as the oracle's; kappa 3 puts many gains
+    past the grid (level 15); rotated dequant of the chosen codes exact."""
+    w, d = synth.small_f32()
+    res = run_shape_gain(e8q, [w], [d], 0, kappa, "rotated", torch.float32)
+    out = oracle.sg_project_encode(w.astype(np.float64), d, 256, kappa)
+    ties = check_shape_gain(out, host_idx(res.idx[0]), f"shape-gain kappa {kappa}")
+    assert ties < 50
+    np.testing.assert_allclose(res.scale[0].cpu().numpy(), out["scale"], rtol=1e-5)
+    if kappa > 2:
+        assert ((host_idx(res.idx[0]).astype(np.int64) & 0xFFFF) >> 12 == 15).mean() > 0.2
+    s32 = res.scale[0].cpu().numpy().astype(np.float64)
+    xh = oracle.sg_points(host_idx(res.idx[0]).astype(np.int64).reshape(-1) & 0xFFFF)
+    bits, _ = oracle.sg_dequant(xh, s32, d, 256, "rotated")
+    got = res.dequant[0].cpu().view(torch.int16).numpy().view(np.uint16)
+    assert (got == bits).all()
+
+
+@pytest.mark.parametrize("rows,cols", [(96, 2048), (37, 264), (5, 16384)])
+def test_shape_gain_bf16_original_basis(e8q, rows, cols):
+    """bf16 rows of several widths and RHT blocks (2048, 8, 2048), original-
+    basis dequant of the chosen codes within one bf16 ulp of the fp64
+    inverse transform."""
+    rng = np.random.default_rng(rows + cols)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((rows, cols)) * 0.015)
+    d = synth.signs(rows, cols)
+    B = oracle.default_block(cols)
+    res = run_shape_gain(e8q, [w], [d], 0, 1.0, "original")
+    out = oracle.sg_project_encode(synth.bf16_bits_to_f64(w), d, B)
+    check_shape_gain(out, host_idx(res.idx[0]), f"shape-gain {rows}x{cols}")
+    s = res.scale[0].cpu().numpy().astype(np.float64)
+    xh = oracle.sg_points(host_idx(res.idx[0]).astype(np.int64).reshape(-1) & 0xFFFF)
+    _, f64 = oracle.sg_dequant(xh, s, d, B, "original")
+    got = synth.bf16_bits_to_f64(res.dequant[0].cpu().view(torch.int16).numpy().view(np.uint16)).reshape(f64.shape)
+    ulp = np.where(f64 != 0, 2.0 ** (np.floor(np.log2(np.abs(f64) + 1e-300)) - 7), 0.0)
+    bad = np.abs(got - f64) > ulp + 2.0 ** -20 * s[:, None]
+    assert not bad.any(), f"{bad.sum()} original-basis values off by more than 1 ulp"
+
+
+def test_shape_gain_shell_points_are_fixed(e8q):
+    """Rows made of shell points (doubled / 2, times a per-row factor) map to
+    themselves: direction = the point's own index, for all 2160 points."""
+    S = oracle.sg_shell().astype(np.float64)
+    rows = (S / 2.0).reshape(270, 64)  # 8 points a row, rows of 64
+    w = rows * np.linspace(0.5, 2.0, 270)[:, None]
+    d = np.ones(64, np.int8)
+    res = run_shape_gain(e8q, [w.astype(np.float32)], [d], 1, 1.0, "none", torch.float32)
+    code = host_idx(res.idx[0]).astype(np.int64).reshape(-1) & 0xFFFF
+    assert ((code & 0xFFF) == np.arange(2160)).all()
+
+
+def test_shape_gain_flag_rules(e8q):
+    """The two flags together are rejected."""
+    w, d = synth.small_f32()
+    with pytest.raises(e8q.E8qError):
+        e8q.Encoder([w.shape], [dev(d)], torch.float32, 0, 1.0, "none", False, 64, 64, core_only=True,
+                    shape_gain=True)([dev(w)])
