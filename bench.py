@@ -527,8 +527,6 @@ def main():
     ap.add_argument("--no-workloads", action="store_true",
                     help="skip the attention-projection and expert-bank encode timings")
     ap.add_argument("--eager", action="store_true", help="time eager launches instead of one captured graph")
-    ap.add_argument("--gemv-path", choices=["auto", "mma_sync", "tcgen05"], default="auto",
-                    help="GEMV main kernel (auto: the library's choice)")
     ap.add_argument("--mode", choices=["auto", "replicas", "sharded"], default="auto",
                     help="several GPUs: independent replicas, or row-sharded blocks of one model with their "
                          "exchange (gather_encoded + all-gather of y); auto: sharded when N > 1")
@@ -553,7 +551,6 @@ def main():
     from bit_e8_lattice_b200 import e8q, synth
 
     e8q.init()
-    e8q.set_gemv_path(args.gemv_path)
     mode = args.mode if args.mode != "auto" else ("sharded" if world > 1 else "replicas")
     if mode == "sharded":
         return run_sharded(args, batches, rank, world, dev)
@@ -774,6 +771,18 @@ def main():
             "groups": G, "drift_std_over_weight_std": PAGES_DRIFT, "core_points_clipped": pc["n_escape"] == 0,
             "escape_fraction": qc["n_escape"] / G, "overflow_fraction": qc["n_overflow"] / G}
         del qenc, qres, WP
+
+        # shape-gain code of the dense-MLP pair (SQuAT page, shape and scale
+        # split): the same transform and row scale, 16-bit direction + gain
+        # codes, original-basis dequant; no records
+        senc = e8q.Encoder([(D_MODEL, D_FF), (D_FF, D_MODEL)], S, torch.bfloat16, 0, 1.0, "original",
+                           esc_cap=64, ovf_cap=64, shape_gain=True)
+        senc(W)
+        torch.cuda.synchronize()
+        med, mean = time_flushed(lambda: senc(W), stream, flush)
+        kernels["shape_gain_project_encode"] = kernel_entry(G * (16 + 2 + 16) + rows * (4 + 16), med, mean, peaks,
+                                                            groups=G, note="general kernel")
+        del senc
     del flush
     torch.cuda.empty_cache()
 
@@ -865,7 +874,7 @@ def main():
             "ms_per_step": ms / K, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
             "dtype": "f32", "data": "synthetic",
             "config": {"workload": WORKLOAD, "groups_per_step_per_gpu": G, "kappa": 1.0, "rht_block": 2048,
-                       "gemv_batches": batches, "gemv_main_kernel": args.gemv_path,
+                       "gemv_batches": batches,
                        "l2": "step: inputs larger than L2 (235 MB of latent weights read per step); "
                              "kernels: L2 flushed by a 256 MB write before each timed call",
                        "escape_fraction": n_esc / G, "overflow_fraction": n_ovf / G,

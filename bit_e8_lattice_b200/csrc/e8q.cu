@@ -14,7 +14,6 @@
 #include "encode.cuh"
 #include "encode_fast.cuh"
 #include "gemv.cuh"
-#include "gemv_tc.cuh"
 #include "ste.cuh"
 #include "tables.h"
 
@@ -25,7 +24,6 @@ constexpr int kMaxDevices = 64;
 std::mutex g_mu;
 bool g_ready[kMaxDevices];
 int g_sms[kMaxDevices];
-int g_gemv_path = 0;  // 0: by batch, 1: mma.sync main kernel, 2: tensor-core main kernel
 
 e8q_status cuda_ok(cudaError_t e) { return e == cudaSuccess ? E8Q_OK : E8Q_ERR_CUDA; }
 
@@ -106,21 +104,6 @@ e8q_status ensure_device(int* dev_out) {
         if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_gv_fin<8>, cudaFuncAttributePreferredSharedMemoryCarveout,
                                               cudaSharedmemCarveoutMaxShared));
-        if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_gv_tc<16>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              static_cast<int>(tc_smem_bytes(16))));
-        if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_gv_tc<32>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              static_cast<int>(tc_smem_bytes(32))));
-        if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_gv_tc<64>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              static_cast<int>(tc_smem_bytes(64))));
-        if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_gv_tc<128>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              static_cast<int>(tc_smem_bytes(128))));
-        if (st == E8Q_OK)
-            st = cuda_ok(cudaFuncSetAttribute(k_gv_tc<256>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                              static_cast<int>(tc_smem_bytes(256))));
         if (st == E8Q_OK) st = cuda_ok(cudaDeviceGetAttribute(&g_sms[dev], cudaDevAttrMultiProcessorCount, dev));
         if (st != E8Q_OK) return st;
         g_ready[dev] = true;
@@ -254,28 +237,6 @@ e8q_status e8q_escape_lookup(const int8_t* coord2, int64_t n, uint32_t* out) {
         out[k] = r == kExtNone ? (2u << 24) : t->res[r];
     }
     return E8Q_OK;
-}
-
-e8q_status e8q_set_gemv_path(int32_t mode) {
-    if (mode < 0 || mode > 2) return E8Q_ERR_INVALID_ARG;
-    std::lock_guard<std::mutex> lk(g_mu);
-    g_gemv_path = mode;
-    return E8Q_OK;
-}
-
-e8q_status e8q_device_error_flags(int32_t reset, uint64_t* flags) {
-    if (!flags) return E8Q_ERR_INVALID_ARG;
-    int dev;
-    e8q_status st = ensure_device(&dev);
-    if (st != E8Q_OK) return st;
-    unsigned long long v = 0;
-    st = cuda_ok(cudaMemcpyFromSymbol(&v, g_tc_err, sizeof(v)));
-    if (st == E8Q_OK && reset) {
-        const unsigned long long z = 0;
-        st = cuda_ok(cudaMemcpyToSymbol(g_tc_err, &z, sizeof(z)));
-    }
-    *flags = v;
-    return st;
 }
 
 size_t e8q_encode_workspace_bytes(const e8q_matrix* mats, int32_t n_mats) {
@@ -496,40 +457,10 @@ e8q_status e8q_dequant_gemv(const e8q_encoded* m, const void* x_bf16, int32_t ba
     pp.group_base = m->group_base;
     pp.g = g;
     pp.n_xcta = g.nseg * batch;
-    // main kernel: tcgen05 from kTcMinBatch rows of activations on, mma.sync below
-    // (or as the path hook forces)
-    const bool tc = g_gemv_path == 2 || (g_gemv_path == 0 && batch >= kTcMinBatch);
-    pp.xk = tc ? reinterpret_cast<uint16_t*>(w + L.xk) : nullptr;
     const int n_ecta = has_esc ? (g.rows + 7) / 8 : 0;
     k_gv_prep<<<pp.n_xcta + n_ecta, 256, 0, s>>>(pp);
     st = cuda_ok(cudaGetLastError());
     if (st != E8Q_OK) return st;
-
-    if (tc) {
-        const GvTcGeom t = gv_tc_geometry(g.rows, g.cols);
-        GvTcParams tp;
-        tp.idx = m->idx;
-        tp.map = has_esc ? pp.map : nullptr;
-        tp.xk = pp.xk;
-        tp.part = reinterpret_cast<float*>(w + L.part);
-        tp.rows = g.rows;
-        tp.cols = g.cols;
-        tp.gpr = g.gpr;
-        tp.batch = batch;
-        tp.mstride = g.mstride;
-        tp.nrt = t.nrt;
-        tp.nkt = t.nkt;
-        tp.nsplit = t.nsplit;
-        tp.vec_idx = (g.gpr % 8 == 0 && aligned(m->idx, 16)) ? 1 : 0;
-        const int units = t.nrt * t.nsplit;  // persistent CTAs, one per SM
-        const int grid = units < g_sms[dev] ? units : g_sms[dev];
-        if (batch <= 16) st = launch_pdl(k_gv_tc<16>, grid, kTcThreads, tc_smem_bytes(16), s, tp);
-        else if (batch <= 32) st = launch_pdl(k_gv_tc<32>, grid, kTcThreads, tc_smem_bytes(32), s, tp);
-        else if (batch <= 64) st = launch_pdl(k_gv_tc<64>, grid, kTcThreads, tc_smem_bytes(64), s, tp);
-        else if (batch <= 128) st = launch_pdl(k_gv_tc<128>, grid, kTcThreads, tc_smem_bytes(128), s, tp);
-        else st = launch_pdl(k_gv_tc<256>, grid, kTcThreads, tc_smem_bytes(256), s, tp);
-        if (st != E8Q_OK) return st;
-    }
 
     GvMainParams mp;
     mp.idx = m->idx;
@@ -539,7 +470,7 @@ e8q_status e8q_dequant_gemv(const e8q_encoded* m, const void* x_bf16, int32_t ba
     mp.g = g;
     mp.vec_idx = (g.gpr % 8 == 0 && aligned(m->idx, 16)) ? 1 : 0;
     const int grid = g.nctas;
-    for (int v0 = 0; !tc && v0 < g.nbt; v0 += kGvPassTiles) {
+    for (int v0 = 0; v0 < g.nbt; v0 += kGvPassTiles) {
         const int nt = g.nbt - v0 < kGvPassTiles ? g.nbt - v0 : kGvPassTiles;
         mp.v0 = v0;
         // one 16-row tile per warp, 16 warps (two tiles on 8 warps measured slower at batch 64 and 256)
@@ -561,7 +492,6 @@ e8q_status e8q_dequant_gemv(const e8q_encoded* m, const void* x_bf16, int32_t ba
     fp.ovf_n = m->ovf_row_ptr ? m->ovf_count : 0;
     fp.group_base = m->group_base;
     fp.g = g;
-    fp.nsplit = tc ? gv_tc_geometry(g.rows, g.cols).nsplit : 0;
     fp.bl_log = 0;
     while ((1 << fp.bl_log) < batch && fp.bl_log < 5) ++fp.bl_log;
     const int kb = (batch + 31) / 32;  // batch rows per lane

@@ -93,25 +93,8 @@ inline GvGeom gv_geometry(int64_t rows, int64_t cols, int batch, int logb, int c
     return g;
 }
 
-// Tensor-core path geometry: 128-row tiles, 64-column K tiles, and the
-// K range of each row tile split so that the grid holds about two CTAs per
-// SM of a 148-SM part (fixed, so that the workspace size needs no device).
-constexpr int kTcTargetCtas = 296;
-struct GvTcGeom {
-    int32_t nrt, nkt, nsplit;
-};
-inline GvTcGeom gv_tc_geometry(int64_t rows, int64_t cols) {
-    GvTcGeom t;
-    t.nrt = static_cast<int32_t>((rows + 127) / 128);
-    t.nkt = static_cast<int32_t>((cols + 63) / 64);
-    int32_t s = t.nrt > 0 ? (kTcTargetCtas + t.nrt - 1) / t.nrt : 1;
-    if (s > t.nkt) s = t.nkt;
-    t.nsplit = s < 1 ? 1 : s;
-    return t;
-}
-
 struct GvWs {
-    size_t x32, x16, xe, map, xk, part, total;
+    size_t x32, x16, xe, map, part, total;
 };
 inline size_t gv_round(size_t x) { return (x + 255) / 256 * 256; }
 inline GvWs gv_workspace(const GvGeom& g) {
@@ -120,11 +103,9 @@ inline GvWs gv_workspace(const GvGeom& g) {
     w.x16 = w.x32 + gv_round(static_cast<size_t>(g.batch) * g.cols * 4);
     w.xe = w.x16 + gv_round(static_cast<size_t>(g.nchunks) * g.nbt * 8 * 32 * 16);
     w.map = w.xe + gv_round(static_cast<size_t>(g.nbt) * 8 * 4);
-    w.xk = w.map + gv_round(static_cast<size_t>(g.rows) * g.mstride);
-    w.part = w.xk + gv_round(static_cast<size_t>(g.batch) * g.cols * 2);
+    w.part = w.map + gv_round(static_cast<size_t>(g.rows) * g.mstride);
     const size_t slots = static_cast<size_t>(g.nrb) * g.maxslots * g.batch * kGvBlockRows * 4;
-    const size_t splits = static_cast<size_t>(gv_tc_geometry(g.rows, g.cols).nsplit) * g.rows * g.batch * 4;
-    w.total = w.part + gv_round(slots > splits ? slots : splits);
+    w.total = w.part + gv_round(slots);
     return w;
 }
 
@@ -142,7 +123,6 @@ struct GvPrepParams {
     float* x32;         // [groups][batch][8]: one group's 8 values of every batch row together
     uint4* x16;         // [nchunks][nbt][8 k-steps][32 lanes] x 8 halves
     float* xe;          // [batch]: 2^e, x16 = xr * 2^-e
-    uint16_t* xk;       // null, or fp16 [batch][cols]: the x16 values row-major (tensor-core path)
     const e8q_escape* esc;
     const int64_t* esc_rp;
     uint8_t* map;       // [rows][mstride]: root + 1 of an escaped group, else 0
@@ -228,7 +208,6 @@ __global__ void __launch_bounds__(256) k_gv_prep(const __grid_constant__ GvPrepP
             o.z = pack_half2(v[4], v[5]);
             o.w = pack_half2(v[6], v[7]);
             p.x16[((static_cast<size_t>(c) * G.nbt + (b >> 3)) * 8 + j) * 32 + L] = o;
-            if (p.xk) *reinterpret_cast<uint4*>(p.xk + static_cast<size_t>(b) * C + col) = o;
         }
         if (seg == 0 && threadIdx.x == 0) p.xe[b] = __uint_as_float(static_cast<unsigned>(127 + e) << 23);
         return;
@@ -584,7 +563,6 @@ struct GvFinParams {
     long long group_base;
     GvGeom g;
     int32_t bl_log;  // log2 of the batch lanes: lanes = record lane * BL + batch lane
-    int32_t nsplit;  // > 0: partial sums are [nsplit][rows][batch] (tensor-core path), else slots
 };
 
 // Lanes = record lane rl (slots / overflow records) x batch lane bl; each
@@ -599,21 +577,12 @@ __global__ void __launch_bounds__(256) k_gv_fin(const __grid_constant__ GvFinPar
     const int BL = 1 << p.bl_log, RL = 32 >> p.bl_log;
     const int bl = lane & (BL - 1), rl = lane >> p.bl_log;
     const int rb = r / kGvBlockRows, ri = r % kGvBlockRows;
-    int nsl;
-    const float* pb;
-    size_t sstride;
-    if (p.nsplit > 0) {  // split partials, in split order
-        nsl = p.nsplit;
-        pb = p.part + static_cast<size_t>(r) * G.batch;
-        sstride = static_cast<size_t>(G.rows) * G.batch;
-    } else {
-        const long long ks = static_cast<long long>(G.nchunks) * 8;
-        const long long c0 = gv_cta_of(static_cast<long long>(rb) * ks, G.ksteps, G.nctas);
-        const long long c1 = gv_cta_of(static_cast<long long>(rb) * ks + ks - 1, G.ksteps, G.nctas);
-        nsl = static_cast<int>(c1 - c0 + 1 < G.maxslots ? c1 - c0 + 1 : G.maxslots);
-        pb = p.part + (static_cast<size_t>(rb) * G.maxslots * kGvBlockRows + ri) * G.batch;
-        sstride = static_cast<size_t>(kGvBlockRows) * G.batch;
-    }
+    const long long ks = static_cast<long long>(G.nchunks) * 8;
+    const long long c0 = gv_cta_of(static_cast<long long>(rb) * ks, G.ksteps, G.nctas);
+    const long long c1 = gv_cta_of(static_cast<long long>(rb) * ks + ks - 1, G.ksteps, G.nctas);
+    const int nsl = static_cast<int>(c1 - c0 + 1 < G.maxslots ? c1 - c0 + 1 : G.maxslots);
+    const float* pb = p.part + (static_cast<size_t>(rb) * G.maxslots * kGvBlockRows + ri) * G.batch;
+    const size_t sstride = static_cast<size_t>(kGvBlockRows) * G.batch;
     float acc[KB];
 #pragma unroll
     for (int k = 0; k < KB; ++k) {

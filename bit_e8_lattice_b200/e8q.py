@@ -89,10 +89,6 @@ def lib():
         L.e8q_dequant_gemv.restype = ctypes.c_int
         L.e8q_ste_backward.argtypes = [vp, vp, i64, vp]
         L.e8q_ste_backward.restype = ctypes.c_int
-        L.e8q_set_gemv_path.argtypes = [i32]
-        L.e8q_set_gemv_path.restype = ctypes.c_int
-        L.e8q_device_error_flags.argtypes = [i32, ctypes.POINTER(ctypes.c_uint64)]
-        L.e8q_device_error_flags.restype = ctypes.c_int
         _lib = L
     return _lib
 
@@ -133,21 +129,6 @@ def escape_lookup(P: np.ndarray) -> np.ndarray:
     _check(lib().e8q_escape_lookup(P.ctypes.data_as(ctypes.c_void_p), P.shape[0], out.ctypes.data_as(ctypes.c_void_p)),
            "e8q_escape_lookup")
     return out
-
-
-GEMV_PATHS = {"auto": 0, "mma_sync": 1, "tcgen05": 2}
-
-
-def set_gemv_path(path: str):
-    """Which GEMV main kernel e8q_dequant_gemv uses: "auto", "mma_sync" or "tcgen05"."""
-    _check(lib().e8q_set_gemv_path(GEMV_PATHS[path]), "e8q_set_gemv_path")
-
-
-def device_error_flags(reset: bool = False) -> int:
-    """Device-side error flags of the current GPU (bit 0: a bounded wait gave up)."""
-    v = ctypes.c_uint64(0)
-    _check(lib().e8q_device_error_flags(1 if reset else 0, ctypes.byref(v)), "e8q_device_error_flags")
-    return int(v.value)
 
 
 def init():

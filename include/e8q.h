@@ -204,16 +204,6 @@ e8q_status e8q_core_table(int8_t* out_coord2);
  * compare the table with other encoders. */
 e8q_status e8q_escape_lookup(const int8_t* coord2, int64_t n, uint32_t* out);
 
-/* Test and tuning hook: which main kernel e8q_dequant_gemv uses.  0 (the
- * default): by batch; 1: the mma.sync kernel; 2: the tcgen05 kernel.  Both
- * give the same sums up to fp32 summation order.  Process-wide; not to be
- * changed while GEMV calls are being issued. */
-e8q_status e8q_set_gemv_path(int32_t mode);
-
-/* Device-side error flags of the current GPU (host call, synchronous):
- * bit 0 = a bounded wait in the tcgen05 GEMV kernel gave up (its output is
- * then undefined).  reset != 0 clears them after reading. */
-e8q_status e8q_device_error_flags(int32_t reset, uint64_t* flags);
 
 /* Workspace bytes e8q_project_encode needs for these matrices (>= 16). */
 size_t e8q_encode_workspace_bytes(const e8q_matrix* mats /* host [n_mats] */, int32_t n_mats);
@@ -289,9 +279,8 @@ size_t e8q_gemv_workspace_bytes(const e8q_encoded* m /* host */, int32_t batch);
  * after a per-row power-of-two scaling chosen from the row's largest |x| (no
  * overflow is possible); fp32 accumulation; overflow records use the fp32
  * values; bf16 output (round to nearest even).  Expected relative error
- * about 1e-4 of the output norm.  The product runs on mma.sync fragments
- * (the default) or on tcgen05 with the accumulator in tensor memory
- * (e8q_set_gemv_path); both give these sums up to fp32 summation order.
+ * about 1e-4 of the output norm.  The partial sums are added in a fixed
+ * order, so repeated calls give the same bits.
  * Asynchronous on `stream`; errors: INVALID_ARG, UNSUPPORTED (cols > 16384),
  * WORKSPACE, CUDA.
  */

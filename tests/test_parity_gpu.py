@@ -353,20 +353,8 @@ def test_deterministic_outputs(e8q):
 
 
 
-@pytest.fixture(params=["mma_sync", "tcgen05"])
-def gemv_path(request, e8q):
-    """Each GEMV test runs with both main kernels (mma.sync fragments and
-    tcgen05 with the accumulator in tensor memory); no bounded wait may
-    give up."""
-    e8q.set_gemv_path(request.param)
-    e8q.device_error_flags(reset=True)
-    yield request.param
-    torch.cuda.synchronize()
-    e8q.set_gemv_path("auto")
-    assert e8q.device_error_flags(reset=True) == 0
-
 @pytest.mark.parametrize("batch", [1, 4, 16, 64])
-def test_gemv_small(e8q, gemv_path, batch):
+def test_gemv_small(e8q, batch):
     rng = np.random.default_rng(batch)
     w = synth.f64_to_bf16_bits(rng.standard_normal((512, 2048)) * 0.015)
     d = synth.signs(batch, 2048)
@@ -390,7 +378,7 @@ def test_gemv_small(e8q, gemv_path, batch):
     (128, 128, 16, 1.0),    # one 128-row tile, one 128-column K tile
     (257, 4096, 64, 1.0),   # three row tiles (the last of one row), several K splits
 ])
-def test_gemv_shapes(e8q, gemv_path, rows, cols, batch, kappa):
+def test_gemv_shapes(e8q, rows, cols, batch, kappa):
     rng = np.random.default_rng(rows * 7 + cols)
     w = synth.f64_to_bf16_bits(rng.standard_normal((rows, cols)) * 0.02)
     d = synth.signs(rows, cols)
@@ -408,7 +396,7 @@ def test_gemv_shapes(e8q, gemv_path, rows, cols, batch, kappa):
     check_gemv(y.cpu().view(torch.int16).numpy(), y_ref, f"gemv {rows}x{cols} b={batch}")
 
 
-def test_gemv_large_activations(e8q, gemv_path):
+def test_gemv_large_activations(e8q):
     """Activations near the bf16 range limit: the per-row power-of-two
     scaling keeps the fp16 operand finite."""
     rng = np.random.default_rng(11)
@@ -434,7 +422,7 @@ def test_gemv_large_activations(e8q, gemv_path):
     assert rel < 1e-2, rel
 
 
-def test_gemv_repeatable(e8q, gemv_path):
+def test_gemv_repeatable(e8q):
     """The partial sums are added in a fixed order: two calls on the same
     inputs give the same bits."""
     rng = np.random.default_rng(21)
@@ -449,7 +437,7 @@ def test_gemv_repeatable(e8q, gemv_path):
     assert torch.equal(y1.view(torch.int16), y2.view(torch.int16))
 
 
-def test_gemv_far_overflow_points(e8q, gemv_path):
+def test_gemv_far_overflow_points(e8q):
     """A scale far below the rows' rms (s = rms / kappa, kappa 50) makes
     every group an overflow record, most with doubled coordinates beyond
     +-127; the GEMV applies those records from their 16-bit coordinates."""
@@ -525,7 +513,7 @@ def test_decode_full_size(e8q, mlp_full):
 
 
 @pytest.mark.parametrize("batch", [1, 4, 16, 64])
-def test_gemv_full_size(e8q, gemv_path, mlp_full, batch):
+def test_gemv_full_size(e8q, mlp_full, batch):
     res = mlp_full["res"]
     m = res.encoded[0]
     idx = host_idx(res.idx[0]).reshape(-1)
