@@ -11,6 +11,8 @@ Tolerances (derived in the design notes):
 * GEMV: ||y - y_ref|| / ||y_ref|| <= 1e-2, and each output within its bf16
   rounding (2^-8 |y_ref|) plus 1e-3 rms(y_ref) of its batch row.
 """
+import os
+
 import numpy as np
 
 import oracle
@@ -21,8 +23,11 @@ MARGIN = 1e-4
 
 def gpu_points(idx, esc_rec, ovf_rec, n_groups, group_base=0):
     """Lattice points the GPU encoded (oracle's exact inverse of the encoding)."""
-    e = esc_rec[(esc_rec["group"] >= group_base) & (esc_rec["group"] < group_base + n_groups)]
-    o = ovf_rec[(ovf_rec["group"] >= group_base) & (ovf_rec["group"] < group_base + n_groups)]
+    # records come in group order (checked by check_encode): the matrix's slice by binary search
+    eg, og = esc_rec["group"], ovf_rec["group"]
+    lo, hi = np.uint32(group_base), np.uint32(min(group_base + n_groups, 2 ** 32 - 1))
+    e = esc_rec[np.searchsorted(eg, lo):np.searchsorted(eg, hi)]
+    o = ovf_rec[np.searchsorted(og, lo):np.searchsorted(og, hi)]
     P = oracle.assemble_points(idx.astype(np.int64) & 0xFFFF, e["group"].astype(np.int64), e["root"].astype(np.int64),
                                o["group"].astype(np.int64), o["coord2"].astype(np.int32), n_groups, group_base)
     kind = np.zeros(n_groups, np.int32)
@@ -110,3 +115,48 @@ def check_gemv(y_gpu, y_ref, label=""):
     rel = np.linalg.norm(y - y_ref) / np.linalg.norm(y_ref)
     assert rel <= 1e-2, f"{label}: relative error {rel:.3g}"
     return rel
+
+
+def _oracle_rows(args):
+    """Worker: the oracle on a block of rows (bf16 bits), for a process pool."""
+    bits, signs, block, want_x = args
+    out = oracle.project_encode(synth.bf16_bits_to_f64(bits), signs, block, 1.0, want_x=want_x)
+    return {k: out[k] for k in ("scale", "x", "P", "margin", "idx", "kind", "root")}
+
+
+def oracle_rows_parallel(jobs, procs=None):
+    """The oracle over many (bits, signs, block, want_x) jobs in spawned
+    processes (one pool; spawn, so that no CUDA state is forked)."""
+    return list(oracle_rows_stream(jobs, procs))
+
+
+def oracle_rows_stream(jobs, procs=None):
+    """As oracle_rows_parallel, yielding the results in job order as they
+    complete (bounded memory for many jobs)."""
+    import multiprocessing as mp
+    procs = procs or max(1, min(32, os.cpu_count() or 1))
+    with mp.get_context("spawn").Pool(procs) as pool:
+        yield from pool.imap(_oracle_rows, jobs, chunksize=1)
+
+
+def merge_rows(outs):
+    m = {}
+    for k in ("scale", "P", "margin", "idx", "kind", "root"):
+        m[k] = np.concatenate([o[k] for o in outs])
+    m["x"] = np.concatenate([o["x"] for o in outs]) if outs[0]["x"] is not None else None
+    return m
+
+
+def check_encode_far(out, idx_gpu, scale_gpu, esc_rec, ovf_rec, group_base, label=""):
+    """check_encode without the oracle's x: every group clear of a tie must
+    agree in point, index, record kind and root; returns the near-tie count."""
+    idx_gpu = np.asarray(idx_gpu).astype(np.int64).reshape(-1) & 0xFFFF
+    P, kind, root, e, o = gpu_points(idx_gpu, esc_rec, ovf_rec, idx_gpu.size, group_base)
+    np.testing.assert_allclose(np.asarray(scale_gpu), out["scale"], rtol=1e-5, atol=0, err_msg=f"{label}: scale")
+    far = out["margin"] > MARGIN
+    assert not (far & (P != out["P"]).any(1)).any(), f"{label}: lattice points differ above the margin"
+    assert (idx_gpu[far] == out["idx"][far]).all(), f"{label}: core index differs above the margin"
+    assert (kind[far] == out["kind"][far]).all(), f"{label}: record kind differs above the margin"
+    ef = far & (out["kind"] == 1)
+    assert (root[ef] == out["root"][ef]).all(), f"{label}: escape root differs"
+    return int((~far).sum())

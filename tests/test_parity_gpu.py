@@ -9,7 +9,8 @@ import torch
 
 import oracle
 from bit_e8_lattice_b200 import synth
-from parity import MARGIN, check_encode, check_gemv, check_original_dequant, check_rotated_dequant, gpu_points
+from parity import (MARGIN, check_encode, check_encode_far, check_gemv, check_original_dequant, check_rotated_dequant,
+                    gpu_points, merge_rows, oracle_rows_parallel, oracle_rows_stream)
 import lattice_np
 
 pytestmark = pytest.mark.gpu
@@ -488,6 +489,45 @@ def test_mlp_full_size_sampled_rows(e8q, mlp_full):
                                f"mlp[{i}] original")
     rp = res.esc_row_ptr.cpu().numpy()
     assert rp[0] == 0 and (np.diff(rp) >= 0).all() and rp[-1] == ctr["n_escape"]
+
+
+def test_mlp_full_matrices_match_oracle(e8q, mlp_full):
+    """Every row of both full-size matrices (14.7 M groups) against the
+    oracle, run over the host's cores: points, indices, record kinds and
+    roots of every group clear of a tie, every near tie a valid E8 point as
+    close as the oracle's, scales, and the records' order and fields."""
+    res = mlp_full["res"]
+    esc, ovf = res.escape_records(), res.overflow_records()
+    mats = [(mlp_full["up"], mlp_full["d_up"]), (mlp_full["down"], mlp_full["d_dn"])]
+    ties = 0
+    for i, (w, d) in enumerate(mats):
+        blocks = np.array_split(np.arange(w.shape[0]), 64)
+        out = merge_rows(oracle_rows_parallel([(w[b], d, 2048, True) for b in blocks]))
+        st = check_encode(out, host_idx(res.idx[i]), res.scale[i].cpu().numpy(), esc, ovf, res.group_base[i],
+                          None, w.shape[1] // 8, f"mlp full [{i}]")
+        ties += st["near_ties"]
+        del out, st
+    assert ties < 1000, ties
+
+
+def test_moe_bank_every_matrix_matches_oracle(e8q):
+    """All 384 expert matrices (75.5 M groups, one launch) against the
+    oracle in full: every group clear of a tie identical, scales within
+    1e-5."""
+    mats = synth.moe_bank()
+    W = [m for m, _ in mats]
+    S = [s for _, s in mats]
+    G = sum(m.shape[0] * (m.shape[1] // 8) for m in W)
+    enc, res = run_encode(e8q, W, S, 0, esc_cap=G // 2, ovf_cap=G // 16)
+    esc, ovf = res.escape_records(), res.overflow_records()
+    idx = [host_idx(t) for t in res.idx]
+    scales = [t.cpu().numpy() for t in res.scale]
+    del enc
+    ties = 0
+    jobs = ((W[i], S[i], oracle.default_block(W[i].shape[1]), False) for i in range(len(W)))
+    for i, out in enumerate(oracle_rows_stream(jobs)):
+        ties += check_encode_far(out, idx[i], scales[i], esc, ovf, res.group_base[i], f"expert matrix {i}")
+    assert ties < 0.001 * G, ties
 
 
 def test_decode_full_size(e8q, mlp_full):
