@@ -62,6 +62,12 @@ e8q_status ensure_device(int* dev_out) {
             st = cuda_ok(cudaFuncSetAttribute(k_encode_fast<kMaxMats>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               kFastSmemBytes));
         if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_encode_fast<1, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              kFastSmemBytes));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_encode_fast<kMaxMats, true>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              kFastSmemBytes));
+        if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_decode, cudaFuncAttributeMaxDynamicSharedMemorySize, kTileMaxElems * 4));
         if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_decode_fast<false>, cudaFuncAttributeMaxDynamicSharedMemorySize,
@@ -261,7 +267,7 @@ e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_
 
     static thread_local EncodeParams<kMaxMats> P;  // ~28 KB: keep it off the stack
     std::memset(&P, 0, sizeof(P));
-    bool fast = a->flags == 0;  // the core-clipped projection and the shape-gain code run in the general kernel
+    bool fast = (a->flags & E8Q_ENCODE_CORE_ONLY) == 0;  // the core-clipped projection runs in the general kernel
     for (int i = 0; i < n_mats; ++i) {
         const int logb = resolve_logb(mats[i].cols, mats[i].rht_block);
         if (!valid_cols(mats[i].cols) || mats[i].cols > kMaxCols || logb < 0 ||
@@ -347,7 +353,12 @@ e8q_status e8q_project_encode(const e8q_matrix* mats, int32_t n_mats, const e8q_
             EncodeParams<1> P1;
             std::memcpy(&P1, &P, offsetof(EncodeParams<1>, m));
             P1.m[0] = P.m[0];
-            k_encode_fast<1><<<grid, kFastThreads, kFastSmemBytes, s>>>(P1, scratch);
+            if (P.shape_gain)
+                k_encode_fast<1, true><<<grid, kFastThreads, kFastSmemBytes, s>>>(P1, scratch);
+            else
+                k_encode_fast<1><<<grid, kFastThreads, kFastSmemBytes, s>>>(P1, scratch);
+        } else if (P.shape_gain) {
+            k_encode_fast<kMaxMats, true><<<grid, kFastThreads, kFastSmemBytes, s>>>(P, scratch);
         } else {
             k_encode_fast<kMaxMats><<<grid, kFastThreads, kFastSmemBytes, s>>>(P, scratch);
         }

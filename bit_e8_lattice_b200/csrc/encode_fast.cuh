@@ -418,7 +418,9 @@ __device__ __forceinline__ void tile_scales(const EncodeParams<MAXM>& p, const F
     }
 }
 
-template <int MAXM>
+// kSG: the shape-gain code instead of the lattice projection (a separate
+// instantiation, so that the projection's code is the same with or without it).
+template <int MAXM, bool kSG = false>
 __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_constant__ EncodeParams<MAXM> p,
                                                                   int16_t* __restrict__ ovf_scratch_all) {
     extern __shared__ __align__(16) unsigned char smem[];
@@ -542,107 +544,135 @@ __global__ void __launch_bounds__(kFastThreads, 1) k_encode_fast(const __grid_co
                     // advances at most once (at hcut) when the width is not a multiple of 2048
                     const int e0 = 8 * (256 * w + 32 * a + q);
                     const int r0l = e0 / C, hcut = (C - e0 % C + 31) >> 5;
-                    // the lane's 8 groups are independent: project all of them, then
-                    // rank all of them, then queue, so that the chains overlap
-                    unsigned oddm = 0u;
+                    bool big = false;  // some |P_i| > 255 (|P|^2 > 65025), or a shape-gain reconstruction
+                    if (kSG) {
+                        // shape-gain code (sg_code): the 16-bit code is the map word (no
+                        // record), the reconstruction x-hat = xm P, held doubled in v for the dequant
 #pragma unroll
-                    for (int h = 0; h < 8; ++h) {
-                        const int row = win_rows ? row_w : r0l + (h >= hcut ? 1 : 0);
-                        const float c = rowc_b[lane_ok ? row : 0];
-                        float X[8];
+                        for (int h = 0; h < 8; ++h) {
+                            const int row = win_rows ? row_w : r0l + (h >= hcut ? 1 : 0);
+                            const float c = rowc_b[lane_ok ? row : 0];
+                            float X[8];
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float2 t = __fmul2_rn(make_float2(v[h][2 * j], v[h][2 * j + 1]), make_float2(c, c));
-                            X[2 * j] = t.x;
-                            X[2 * j + 1] = t.y;
-                        }
-                        if (p.clamp) {
-#pragma unroll
-                            for (int e = 0; e < 8; ++e) X[e] = fminf(fmaxf(X[e], -1048576.f), 1048576.f);
-                        }
-                        float Pf[8];
-                        oddm |= (e8_nearest_lean(X, Pf) ? 1u : 0u) << h;
-#pragma unroll
-                        for (int e = 0; e < 8; ++e) v[h][e] = Pf[e];  // keep p for the dequant
-                    }
-                    // Groups that may lie outside the core: the core holds every point with
-                    // |p|^2 <= 10 and none with |p|^2 > 12, so only |P|^2 > 40 can escape.
-                    // Their extended rank comes straight from the coordinates (digits
-                    // (P + 9) >> 1 = P / 2 + 4 or + 4.5, keys base 10, exact in fp32); the two
-                    // table gathers of all 8 groups are issued together with the core ranks,
-                    // so that their latency overlaps them, and the encoding words after them.
-                    // These tables are read through L2 only (__ldcg): their scattered
-                    // lines would otherwise push the rank table T1 out of L1.
-                    uint32_t ia[8], ib[8];
-                    int rks[8];
-                    bool big = false;  // some |P_i| > 255 implies |P|^2 > 65025
-#pragma unroll
-                    for (int h = 0; h < 8; ++h) {
-                        const float (&P)[8] = v[h];
-                        float2 n = __fmul2_rn(make_float2(P[0], P[4]), make_float2(P[0], P[4]));
-                        n = __ffma2_rn(make_float2(P[1], P[5]), make_float2(P[1], P[5]), n);
-                        n = __ffma2_rn(make_float2(P[2], P[6]), make_float2(P[2], P[6]), n);
-                        n = __ffma2_rn(make_float2(P[3], P[7]), make_float2(P[3], P[7]), n);
-                        const float n2 = n.x + n.y;
-                        big |= !(n2 <= 65025.f);
-                        const bool in = lane_ok && n2 > 40.f && n2 <= 88.f;  // then every |P_i| <= 9 as well
-                        float2 k = __fmul2_rn(make_float2(P[0], P[4]), make_float2(1000.f, 1000.f));
-                        k = __ffma2_rn(make_float2(P[1], P[5]), make_float2(100.f, 100.f), k);
-                        k = __ffma2_rn(make_float2(P[2], P[6]), make_float2(10.f, 10.f), k);
-                        k = __fadd2_rn(make_float2(P[3], P[7]), k);
-                        const float base = ((oddm >> h) & 1u) ? 14999.5f : 4444.f;  // type * 10000 + 1111 * (4.5 or 4)
-                        const int hk = __float_as_int(fmaf(k.x, 0.5f, base) + 8388608.f) - 0x4B000000;
-                        const int lk = __float_as_int(fmaf(k.y, 0.5f, base) + 8388608.f) - 0x4B000000;
-                        const int lv = __float_as_int(fmaf(n2, 0.125f, 8388608.f)) - 0x4B000000;
-                        ia[h] = in ? __ldcg(g_t1e + hk * 12 + lv) : 0xFFFFFFFFu;
-                        ib[h] = in ? __ldcg(g_t2e + lk) : 0xFFFFFFFFu;
-                        rks[h] = lane_ok ? core_rank_nb(P, (oddm >> h) & 1u, n2, g_t1, st2) : 0;
-                    }
-                    uint32_t ew[8];
-                    unsigned pendm = 0u;
-#pragma unroll
-                    for (int h = 0; h < 8; ++h) {
-                        const bool pend = lane_ok && rks[h] < 0;
-                        pendm |= (pend ? 1u : 0u) << h;
-                        const uint32_t r = ia[h] + ib[h];
-                        const bool hit = pend && ia[h] != 0xFFFFFFFFu && ib[h] != 0xFFFFFFFFu &&
-                                         r < static_cast<uint32_t>(kExtPoints);
-                        ew[h] = hit ? __ldcg(g_res + r) : (2u << 24);
-                    }
-#pragma unroll
-                    for (int h = 0; h < 8; ++h) {
-                        if (!lane_ok) continue;
-                        const int gt = 256 * w + 32 * a + 4 * h + q;
-                        const bool pend = (pendm >> h) & 1u;
-                        const uint32_t word = pend ? ew[h] : static_cast<uint32_t>(rks[h]);
-                        map[map_slot(gt)] = word;
-                        // an overflow record keeps the coordinates as int16 (saturated when
-                        // the inputs were clamped); formed for every group, without a branch:
-                        // x + 1.5 * 2^23 holds the integer x in its low 16 bits (|x| < 2^22)
-                        const bool ovf = pend && (word >> 24) == 2;
-                        float c[8];
-                        bool clamp = false;
-#pragma unroll
-                        for (int k = 0; k < 8; ++k) c[k] = v[h][k];
-                        if (p.clamp) {
-#pragma unroll
-                            for (int k = 0; k < 8; ++k) {
-                                const float t = fminf(fmaxf(c[k], -32768.f), 32767.f);
-                                clamp |= t != c[k];
-                                c[k] = t;
+                            for (int j = 0; j < 4; ++j) {
+                                const float2 t = __fmul2_rn(make_float2(v[h][2 * j], v[h][2 * j + 1]), make_float2(c, c));
+                                X[2 * j] = t.x;
+                                X[2 * j + 1] = t.y;
                             }
-                        }
-                        unsigned o[4];
+                            if (p.clamp) {
 #pragma unroll
-                        for (int j = 0; j < 4; ++j) {
-                            const float2 t = __fadd2_rn(make_float2(c[2 * j], c[2 * j + 1]), make_float2(12582912.f, 12582912.f));
-                            o[j] = prmt(__float_as_uint(t.x), __float_as_uint(t.y), 0x5410u);
+                                for (int e = 0; e < 8; ++e) X[e] = fminf(fmaxf(X[e], -1048576.f), 1048576.f);
+                            }
+                            int Pi[8];
+                            float xm;
+                            const int code = sg_code(X, Pi, xm, g_t1, st2);
+#pragma unroll
+                            for (int e = 0; e < 8; ++e) v[h][e] = 2.f * xm * static_cast<float>(Pi[e]);
+                            if (lane_ok) map[map_slot(256 * w + 32 * a + 4 * h + q)] = static_cast<uint32_t>(code);
                         }
-                        if (ovf) *reinterpret_cast<uint4*>(oscr + 8 * gt) = make_uint4(o[0], o[1], o[2], o[3]);
-                        if (ovf && clamp) ++clamped;
+                        big = true;  // x-hat has up to 9 significant bits: the three-term bf16 split
+                        __syncwarp();
+                    } else {
+                        // the lane's 8 groups are independent: project all of them, then
+                        // rank all of them, then queue, so that the chains overlap
+                        unsigned oddm = 0u;
+    #pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            const int row = win_rows ? row_w : r0l + (h >= hcut ? 1 : 0);
+                            const float c = rowc_b[lane_ok ? row : 0];
+                            float X[8];
+    #pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const float2 t = __fmul2_rn(make_float2(v[h][2 * j], v[h][2 * j + 1]), make_float2(c, c));
+                                X[2 * j] = t.x;
+                                X[2 * j + 1] = t.y;
+                            }
+                            if (p.clamp) {
+    #pragma unroll
+                                for (int e = 0; e < 8; ++e) X[e] = fminf(fmaxf(X[e], -1048576.f), 1048576.f);
+                            }
+                            float Pf[8];
+                            oddm |= (e8_nearest_lean(X, Pf) ? 1u : 0u) << h;
+    #pragma unroll
+                            for (int e = 0; e < 8; ++e) v[h][e] = Pf[e];  // keep p for the dequant
+                        }
+                        // Groups that may lie outside the core: the core holds every point with
+                        // |p|^2 <= 10 and none with |p|^2 > 12, so only |P|^2 > 40 can escape.
+                        // Their extended rank comes straight from the coordinates (digits
+                        // (P + 9) >> 1 = P / 2 + 4 or + 4.5, keys base 10, exact in fp32); the two
+                        // table gathers of all 8 groups are issued together with the core ranks,
+                        // so that their latency overlaps them, and the encoding words after them.
+                        // These tables are read through L2 only (__ldcg): their scattered
+                        // lines would otherwise push the rank table T1 out of L1.
+                        uint32_t ia[8], ib[8];
+                        int rks[8];
+    #pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            const float (&P)[8] = v[h];
+                            float2 n = __fmul2_rn(make_float2(P[0], P[4]), make_float2(P[0], P[4]));
+                            n = __ffma2_rn(make_float2(P[1], P[5]), make_float2(P[1], P[5]), n);
+                            n = __ffma2_rn(make_float2(P[2], P[6]), make_float2(P[2], P[6]), n);
+                            n = __ffma2_rn(make_float2(P[3], P[7]), make_float2(P[3], P[7]), n);
+                            const float n2 = n.x + n.y;
+                            big |= !(n2 <= 65025.f);
+                            const bool in = lane_ok && n2 > 40.f && n2 <= 88.f;  // then every |P_i| <= 9 as well
+                            float2 k = __fmul2_rn(make_float2(P[0], P[4]), make_float2(1000.f, 1000.f));
+                            k = __ffma2_rn(make_float2(P[1], P[5]), make_float2(100.f, 100.f), k);
+                            k = __ffma2_rn(make_float2(P[2], P[6]), make_float2(10.f, 10.f), k);
+                            k = __fadd2_rn(make_float2(P[3], P[7]), k);
+                            const float base = ((oddm >> h) & 1u) ? 14999.5f : 4444.f;  // type * 10000 + 1111 * (4.5 or 4)
+                            const int hk = __float_as_int(fmaf(k.x, 0.5f, base) + 8388608.f) - 0x4B000000;
+                            const int lk = __float_as_int(fmaf(k.y, 0.5f, base) + 8388608.f) - 0x4B000000;
+                            const int lv = __float_as_int(fmaf(n2, 0.125f, 8388608.f)) - 0x4B000000;
+                            ia[h] = in ? __ldcg(g_t1e + hk * 12 + lv) : 0xFFFFFFFFu;
+                            ib[h] = in ? __ldcg(g_t2e + lk) : 0xFFFFFFFFu;
+                            rks[h] = lane_ok ? core_rank_nb(P, (oddm >> h) & 1u, n2, g_t1, st2) : 0;
+                        }
+                        uint32_t ew[8];
+                        unsigned pendm = 0u;
+    #pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            const bool pend = lane_ok && rks[h] < 0;
+                            pendm |= (pend ? 1u : 0u) << h;
+                            const uint32_t r = ia[h] + ib[h];
+                            const bool hit = pend && ia[h] != 0xFFFFFFFFu && ib[h] != 0xFFFFFFFFu &&
+                                             r < static_cast<uint32_t>(kExtPoints);
+                            ew[h] = hit ? __ldcg(g_res + r) : (2u << 24);
+                        }
+    #pragma unroll
+                        for (int h = 0; h < 8; ++h) {
+                            if (!lane_ok) continue;
+                            const int gt = 256 * w + 32 * a + 4 * h + q;
+                            const bool pend = (pendm >> h) & 1u;
+                            const uint32_t word = pend ? ew[h] : static_cast<uint32_t>(rks[h]);
+                            map[map_slot(gt)] = word;
+                            // an overflow record keeps the coordinates as int16 (saturated when
+                            // the inputs were clamped); formed for every group, without a branch:
+                            // x + 1.5 * 2^23 holds the integer x in its low 16 bits (|x| < 2^22)
+                            const bool ovf = pend && (word >> 24) == 2;
+                            float c[8];
+                            bool clamp = false;
+    #pragma unroll
+                            for (int k = 0; k < 8; ++k) c[k] = v[h][k];
+                            if (p.clamp) {
+    #pragma unroll
+                                for (int k = 0; k < 8; ++k) {
+                                    const float t = fminf(fmaxf(c[k], -32768.f), 32767.f);
+                                    clamp |= t != c[k];
+                                    c[k] = t;
+                                }
+                            }
+                            unsigned o[4];
+    #pragma unroll
+                            for (int j = 0; j < 4; ++j) {
+                                const float2 t = __fadd2_rn(make_float2(c[2 * j], c[2 * j + 1]), make_float2(12582912.f, 12582912.f));
+                                o[j] = prmt(__float_as_uint(t.x), __float_as_uint(t.y), 0x5410u);
+                            }
+                            if (ovf) *reinterpret_cast<uint4*>(oscr + 8 * gt) = make_uint4(o[0], o[1], o[2], o[3]);
+                            if (ovf && clamp) ++clamped;
+                        }
+                        __syncwarp();
                     }
-                    __syncwarp();
-
                     // dequantised weights
                     if (p.dq_mode == E8Q_DEQUANT_ROTATED) {
                         uint16_t* dq = static_cast<uint16_t*>(M.dq) + static_cast<size_t>(cur.r0) * C;

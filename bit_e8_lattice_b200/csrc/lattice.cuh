@@ -296,6 +296,99 @@ __device__ __forceinline__ bool e8_nearest_lean(const float (&X)[8], float (&P)[
     return useB;
 }
 
+// Shape-gain code of X = 2x (SQuAT page, "shape and scale split": a unit
+// direction quantised against a spherical E8 codebook, a scalar gain
+// through a low-bit scalar quantiser).  Directions: the 2160 points of the
+// |p|^2 = 4 shell, core indices kSgShellFirst .. + 2159; the best is the one
+// of largest <X, P>, taken per family of the shell (doubled coordinates):
+//   +-4 e_i                       4 max |X_i|
+//   +-2 on four coordinates       2 (sum of the four largest |X_i|)
+//   odd, one +-3, sum = 0 mod 4   sum |X_i| + 2 |X_j| for the +-3 at j, less
+//                                 the cheapest sign reversal when the number
+//                                 of negative X_i is even (the sum rule):
+//                                 2 |X_i| for a +-1, 6 |X_j| for the +-3.
+// Gain level k = min(15, floor(|x| / (6 / 16))).  On return P holds the
+// direction's doubled point and xm the factor (k + 1/2) (6 / 16) / 4 that
+// maps P to the reconstruction x-hat = xm P; the result is k << 12 | the
+// direction's index in the shell.
+constexpr int kSgShellFirst = 241;
+constexpr float kSgStep = 6.0f / 16.0f;
+
+__device__ __forceinline__ int sg_code(const float (&X)[8], int (&P)[8], float& xm, const uint16_t* __restrict__ st1,
+                                       const uint16_t* __restrict__ st2) {
+    float a[8];
+    float n2 = 0.f, total = 0.f;
+    int neg = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        a[i] = fabsf(X[i]);
+        n2 = fmaf(X[i], X[i], n2);
+        total += a[i];
+        neg += X[i] < 0.f;
+    }
+    // family +-4 e_i; the four largest |X_i| (rank by value, then position);
+    // the two smallest
+    int imax = 0, imin = 0, imin2 = -1;
+    float top4 = 0.f;
+    unsigned in4 = 0;
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        if (a[i] > a[imax]) imax = i;
+        int r = 0;
+#pragma unroll
+        for (int k = 0; k < 8; ++k) r += (a[k] > a[i]) || (a[k] == a[i] && k < i);
+        if (r < 4) {
+            top4 += a[i];
+            in4 |= 1u << i;
+        }
+        if (a[i] < a[imin]) imin = i;
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+        if (i != imin && (imin2 < 0 || a[i] < a[imin2])) imin2 = i;
+    const float sA = 4.f * a[imax], sB = 2.f * top4;
+    // odd family: the +-3 at j
+    float sC = -INFINITY;
+    int jC = 0, fC = -1;
+#pragma unroll
+    for (int j = 0; j < 8; ++j) {
+        float sc = total + 2.f * a[j];
+        int f = -1;
+        if ((neg & 1) == 0) {
+            const int o = (j == imin) ? imin2 : imin;  // smallest |X_i|, i != j
+            const float c1 = 2.f * a[o], c3 = 6.f * a[j];
+            if (c3 < c1) {
+                sc -= c3;
+                f = j;
+            } else {
+                sc -= c1;
+                f = o;
+            }
+        }
+        if (sc > sC) {
+            sC = sc;
+            jC = j;
+            fC = f;
+        }
+    }
+#pragma unroll
+    for (int i = 0; i < 8; ++i) {
+        const int sg = X[i] < 0.f ? -1 : 1;
+        if (sA >= sB && sA >= sC) {
+            P[i] = i == imax ? 4 * sg : 0;
+        } else if (sB >= sC) {
+            P[i] = ((in4 >> i) & 1u) ? 2 * sg : 0;
+        } else {
+            const int v = (i == jC ? 3 : 1) * sg;
+            P[i] = i == fC ? -v : v;
+        }
+    }
+    const float g = 0.5f * sqrtf(n2);
+    const int k = min(15, static_cast<int>(floorf(g / kSgStep)));
+    xm = (static_cast<float>(k) + 0.5f) * kSgStep * 0.25f;
+    return (k << 12) | (core_rank(P, st1, st2) - kSgShellFirst);
+}
+
 // Core index of a point given as exact floats (doubled coordinates) and its
 // type, or -1 outside the core; the two table keys are formed with exact
 // small-integer float arithmetic.
