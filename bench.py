@@ -47,6 +47,7 @@ D_MODEL, D_FF = 4096, 14336
 NOMINAL_HBM_GBS = 8000.0
 CSRC = os.path.join("bit_e8_lattice_b200", "csrc")
 FLUSH_BYTES = 256 << 20
+GV_TABLE_WORDS = 49152  # codeword words the GEMV main kernel holds in shared memory
 PAGES_DRIFT = 0.125  # drift of core-initialised latents, in units of the weights' std
 KERNEL_REPS = 20
 SAMPLE_UP, SAMPLE_DN = 2, 7  # oracle sample rows per step (1 : 3.5, the workload's proportion)
@@ -676,6 +677,12 @@ def main():
         med, mean = time_flushed(lambda b=b: gemvs[b](X[b]), stream, flush)
         e = kernel_entry(gb_bytes, med, mean, peaks)
         e["in_step_us_mean"] = 1e3 * statistics.mean(gem_ms[b])
+        # not algorithmic, reported apart: the dense flops, and the codeword
+        # table each main-kernel CTA stages into shared memory from L2 per pass
+        e["flops"] = 2 * b * D_MODEL * D_FF
+        e["TFLOP_s"] = e["flops"] / (med * 1e-3) / 1e12
+        e["table_staging_bytes_from_l2"] = min(torch.cuda.get_device_properties(dev).multi_processor_count, 160) * \
+            GV_TABLE_WORDS * 4 * ((b + 63) // 64)
         kernels[f"dequant_gemv_b{b}"] = e
 
     # decode of the encoded up matrix: indices, records, scales and row
