@@ -50,15 +50,24 @@ FLUSH_BYTES = 256 << 20
 GV_TABLE_WORDS = 49152  # codeword words the GEMV main kernel holds in shared memory
 PAGES_DRIFT = 0.125  # drift of core-initialised latents, in units of the weights' std
 KERNEL_REPS = 20
+GEMM_BATCHES = (64, 256, 1024, 4096)  # activation rows of the fused dequant-GEMM entries (prefill, QAT forward)
 SAMPLE_UP, SAMPLE_DN = 2, 7  # oracle sample rows per step (1 : 3.5, the workload's proportion)
 
 
-def source_sha() -> str:
-    """Hash of the code of every kernel source file, comments and blank
-    space removed (a profile taken on other code does not describe the
-    current kernels)."""
+# device-code files each profiled kernel is built from (its own header and
+# the headers it includes); a profile describes the kernel while these are unchanged
+KERNEL_SOURCES = {
+    "k_encode_fast": ("encode_fast.cuh", "encode.cuh", "lattice.cuh", "common.cuh", "ptx.cuh"),
+}
+
+
+def source_sha(kernel: str = None) -> str:
+    """Hash of the code of a kernel's source files (every kernel source file
+    when kernel is None), comments and blank space removed: a profile taken
+    on other code does not describe the current kernel."""
     h = hashlib.sha256()
-    for f in sorted(os.listdir(os.path.join(ROOT, CSRC))):
+    names = KERNEL_SOURCES[kernel] if kernel else sorted(os.listdir(os.path.join(ROOT, CSRC)))
+    for f in sorted(names):
         if f.endswith((".cu", ".cuh", ".cpp", ".h")):
             text = open(os.path.join(ROOT, CSRC, f), encoding="utf-8").read()
             text = re.sub(r"/\*.*?\*/", " ", text, flags=re.S)
@@ -72,8 +81,8 @@ def measured_peaks() -> dict:
     p = os.path.join(ROOT, "MEASURED_PEAKS.json")
     if os.path.exists(p):
         d = json.load(open(p))
-        return {"hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
-    return {"hbm_gbs": 6650.0, "source": "fallback"}
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]), "source": "measured"}
+    return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "source": "fallback"}
 
 
 def profile_traffic(kernel: str):
@@ -87,7 +96,7 @@ def profile_traffic(kernel: str):
         if ":" in line and line.strip().startswith("-"):
             k, v = line.strip().lstrip("- ").split(":", 1)
             vals[k.strip()] = v.strip().strip("`")
-    if vals.get("source_sha") != source_sha():
+    if vals.get("source_sha") != source_sha(kernel):
         return None
     try:
         return float(vals["traffic_bytes_per_launch"])
@@ -692,6 +701,33 @@ def main():
     for basis in ("rotated", "original"):
         med, mean = time_flushed(lambda basis=basis: e8q.e8q_decode(res.encoded[0], basis, dq_out), stream, flush)
         kernels[f"decode_{basis}"] = kernel_entry(dec_bytes, med, mean, peaks, groups=up_groups)
+
+    # fused dequant-GEMM of the encoded up matrix for many activation rows,
+    # and the unfused route it replaces: decode to bf16 weights (written to
+    # and read back from HBM), then a cuBLAS bf16 GEMM
+    for b in GEMM_BATCHES:
+        xg = t_bf16(synth.gemv_x(b, D_FF))
+        gm = e8q.Gemm(res.encoded[0], b)
+        gm(xg)
+        torch.cuda.synchronize()
+        if gm.error_word():
+            raise RuntimeError("a bounded wait of the GEMM gave up")
+        med, mean = time_flushed(lambda: gm(xg), stream, flush)
+        g_bytes = 2 * up_groups + 8 * up_esc + 20 * up_ovf + 4 * D_MODEL + 16 * (D_MODEL + 1) + 2 * b * (D_FF + D_MODEL)
+        e = kernel_entry(g_bytes, med, mean, peaks)
+        e["flops"] = 2 * b * D_MODEL * D_FF
+        e["TFLOP_s"] = e["flops"] / (med * 1e-3) / 1e12
+        e["frac_measured_bf16_tensor"] = e["TFLOP_s"] / peaks["bf16_tflops"]
+        yo = torch.empty((b, D_MODEL), dtype=torch.bfloat16, device=dev)
+
+        def unfused(xg=xg, yo=yo):
+            e8q.e8q_decode(res.encoded[0], "original", dq_out)
+            torch.matmul(xg, dq_out.t(), out=yo)
+
+        umed, _ = time_flushed(unfused, stream, flush)
+        e["unfused_decode_then_cublas_us"] = 1e3 * umed
+        kernels[f"dequant_gemm_b{b}"] = e
+        del gm, xg, yo
 
     # identity-STE backward in its copying form (grad_latent a separate buffer)
     gl = [torch.empty_like(g) for g in GRAD]

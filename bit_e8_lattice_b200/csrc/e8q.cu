@@ -13,6 +13,7 @@
 #include "decode_fast.cuh"
 #include "encode.cuh"
 #include "encode_fast.cuh"
+#include "gemm_tc.cuh"
 #include "gemv.cuh"
 #include "ste.cuh"
 #include "tables.h"
@@ -93,6 +94,15 @@ e8q_status ensure_device(int* dev_out) {
             st = cuda_ok(cudaFuncSetAttribute(k_gv_main<1, 4>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
         if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_gv_main<1, 8>, cudaFuncAttributeMaxDynamicSharedMemorySize, kGvSmemBytes));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_gm_main, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                              static_cast<int>(kGmSmemBytes)));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_gm_prep, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                              cudaSharedmemCarveoutMaxShared));
+        if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_gm_fin, cudaFuncAttributePreferredSharedMemoryCarveout,
+                                              cudaSharedmemCarveoutMaxShared));
         // prep and finalize leave the SM configured for the main kernel's shared
         // memory, so that its CTAs can start while they are still running
         if (st == E8Q_OK)
@@ -198,6 +208,14 @@ e8q_status check_encoded(const e8q_encoded* m, int* logb) {
     if (m->esc_count < 0 || m->ovf_count < 0) return E8Q_ERR_INVALID_ARG;
     if (m->group_base < 0) return E8Q_ERR_INVALID_ARG;
     return E8Q_OK;
+}
+
+
+// The GEMM's plan for this matrix and batch, or false for arguments it rejects.
+bool gemm_plan(const e8q_encoded* m, int32_t batch, int logb, GmGeom* g) {
+    if (batch < 1 || batch > kGmMaxBatch) return false;
+    *g = gm_geometry(m->rows, m->cols, batch, logb);
+    return g->nunits >= 0;
 }
 
 }  // namespace
@@ -511,6 +529,92 @@ e8q_status e8q_dequant_gemv(const e8q_encoded* m, const void* x_bf16, int32_t ba
     if (kb == 2) return launch_pdl(k_gv_fin<2>, fgrid, 256, 0, s, fp);
     if (kb <= 4) return launch_pdl(k_gv_fin<4>, fgrid, 256, 0, s, fp);
     return launch_pdl(k_gv_fin<8>, fgrid, 256, 0, s, fp);
+}
+
+size_t e8q_gemm_workspace_bytes(const e8q_encoded* m, int32_t batch) {
+    int logb;
+    GmGeom g;
+    if (check_encoded(m, &logb) != E8Q_OK || !gemm_plan(m, batch, logb, &g)) return 256;
+    return gm_workspace(g).total;
+}
+
+e8q_status e8q_dequant_gemm(const e8q_encoded* m, const void* x_bf16, int32_t batch, void* y_bf16, void* ws,
+                            size_t ws_bytes, e8q_stream stream) {
+    int logb;
+    e8q_status st = check_encoded(m, &logb);
+    if (st != E8Q_OK) return st;
+    if (batch < 1 || batch > kGmMaxBatch) return E8Q_ERR_INVALID_ARG;
+    if (!x_bf16 || !y_bf16 || !m->signs || !aligned(x_bf16, 16) || !aligned(y_bf16, 2)) return E8Q_ERR_INVALID_ARG;
+    if (m->esc_row_ptr && !aligned(m->esc, 8)) return E8Q_ERR_INVALID_ARG;
+    if (m->ovf_row_ptr && !aligned(m->ovf, 4)) return E8Q_ERR_INVALID_ARG;
+    GmGeom g;
+    if (!gemm_plan(m, batch, logb, &g)) return E8Q_ERR_UNSUPPORTED;
+    const GmWs L = gm_workspace(g);
+    if (!ws || ws_bytes < L.total || !aligned(ws, 256)) return E8Q_ERR_WORKSPACE;
+    if (m->rows == 0) return E8Q_OK;
+    int dev;
+    st = ensure_device(&dev);
+    if (st != E8Q_OK) return st;
+    cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+    unsigned char* w = static_cast<unsigned char*>(ws);
+
+    GmPrepParams pp;
+    pp.x = static_cast<const uint16_t*>(x_bf16);
+    pp.signs = m->signs;
+    pp.img = w + L.img;
+    pp.xe = reinterpret_cast<float*>(w + L.xe);
+    pp.esc = m->esc;
+    pp.esc_rp = m->esc_row_ptr;
+    pp.esc_n = m->esc_row_ptr ? m->esc_count : 0;
+    pp.ovf = m->ovf;
+    pp.ovf_rp = m->ovf_row_ptr;
+    pp.ovf_n = m->ovf_row_ptr ? m->ovf_count : 0;
+    pp.map = reinterpret_cast<uint16_t*>(w + L.map);
+    pp.farf = w + L.farf;
+    pp.err = reinterpret_cast<unsigned long long*>(w + L.err);
+    pp.group_base = m->group_base;
+    pp.g = g;
+    pp.n_xcta = (batch + 15) / 16 * 16;
+    const int n_rcta = (g.rows + 7) / 8;
+    k_gm_prep<<<pp.n_xcta + n_rcta, 256, 0, s>>>(pp);
+    st = cuda_ok(cudaGetLastError());
+    if (st != E8Q_OK) return st;
+
+    GmMainParams mp;
+    mp.idx = m->idx;
+    mp.map = pp.map;
+    mp.img = pp.img;
+    mp.xe = pp.xe;
+    mp.scale = m->scale;
+    mp.farf = pp.farf;
+    mp.ovf = m->ovf;
+    mp.ovf_rp = m->ovf_row_ptr;
+    mp.ovf_n = pp.ovf_n;
+    mp.part = reinterpret_cast<float*>(w + L.part);
+    mp.y = static_cast<uint16_t*>(y_bf16);
+    mp.err = pp.err;
+    mp.group_base = m->group_base;
+    mp.g = g;
+    const int grid = g.nunits < g_sms[dev] ? g.nunits : g_sms[dev];
+    st = launch_pdl(k_gm_main, grid, kGmThreads, kGmSmemBytes, s, mp);
+    if (st != E8Q_OK || g.nsplit == 1) return st;
+
+    GmFinParams fp;
+    fp.part = mp.part;
+    fp.xe = pp.xe;
+    fp.scale = m->scale;
+    fp.farf = pp.farf;
+    fp.img = pp.img;
+    fp.ovf = m->ovf;
+    fp.ovf_rp = m->ovf_row_ptr;
+    fp.ovf_n = pp.ovf_n;
+    fp.group_base = m->group_base;
+    fp.y = mp.y;
+    fp.g = g;
+    const size_t n = static_cast<size_t>(batch) * g.rows;
+    const size_t fb = (n + 255) / 256;
+    const int fgrid = static_cast<int>(fb < static_cast<size_t>(16 * g_sms[dev]) ? fb : 16 * g_sms[dev]);
+    return launch_pdl(k_gm_fin, fgrid, 256, 0, s, fp);
 }
 
 e8q_status e8q_ste_backward(const void* grad_dequant, void* grad_latent, int64_t n, e8q_stream stream) {

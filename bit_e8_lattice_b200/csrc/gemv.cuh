@@ -141,6 +141,55 @@ __device__ __forceinline__ unsigned pack_half2(float a, float b) {
     return *reinterpret_cast<const unsigned*>(&h);
 }
 
+// Exponent e of one activation row (a CTA of 256 threads): |xr_i| <=
+// sqrt(B) max|x|, so xr * 2^-e stays below 2^15 and cannot overflow fp16.
+// s_red: 8 words of shared memory.
+__device__ inline int gv_row_exponent(const uint16_t* xb, int C, int logb, unsigned* s_red) {
+    const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+    // largest |x| of the row, as bf16 magnitude bits (integer order = value order)
+    unsigned m = 0;
+    for (int i0 = 0; i0 < C / 8; i0 += 8 * 256) {
+        uint4 v[8];  // all loads of a round before their use
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const int i = i0 + threadIdx.x + 256 * k;
+            v[k] = i < C / 8 ? __ldg(reinterpret_cast<const uint4*>(xb) + i) : make_uint4(0, 0, 0, 0);
+        }
+#pragma unroll
+        for (int k = 0; k < 8; ++k) {
+            const unsigned w4[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e) m = max(m, max(w4[e] & 0x7FFFu, (w4[e] >> 16) & 0x7FFFu));
+        }
+    }
+    m = __reduce_max_sync(0xFFFFFFFFu, m);
+    if (lane == 0) s_red[warp] = m;
+    __syncthreads();
+    m = s_red[0];
+#pragma unroll
+    for (int k = 1; k < 8; ++k) m = max(m, s_red[k]);
+    int e = 0;
+    if (m != 0 && m < 0x7F80u) {
+        const float bound = __uint_as_float(m << 16) * sqrtf(static_cast<float>(1 << logb)) * 1.0001f;
+        int k;
+        frexpf(bound, &k);
+        e = k - 15;
+        e = e < -126 ? -126 : (e > 126 ? 126 : e);
+    }
+    return e;
+}
+
+// buf[0 .. n) = H_B (d (.) x)[c0 .. c0 + n) without the 1/sqrt(B) (a CTA of
+// 256 threads; n a multiple of B).
+__device__ inline void gv_rotate_segment(float* buf, const uint16_t* xb, const int8_t* signs, int c0, int n, int logb) {
+    for (int i = threadIdx.x; i < n; i += 256) {
+        const float v = __uint_as_float(static_cast<unsigned>(xb[c0 + i]) << 16);
+        buf[i] = signs[c0 + i] < 0 ? -v : v;
+    }
+    __syncthreads();
+    if (logb > 0) fwht_smem(buf, n, logb);
+}
+
 __global__ void __launch_bounds__(256) k_gv_prep(const __grid_constant__ GvPrepParams p) {
     __shared__ __align__(16) float buf[kGvSegCols];
     __shared__ unsigned s_red[8];
@@ -151,46 +200,11 @@ __global__ void __launch_bounds__(256) k_gv_prep(const __grid_constant__ GvPrepP
         const int b = blockIdx.x / G.nseg, seg = blockIdx.x % G.nseg;
         const int C = G.cols;
         const uint16_t* xb = p.x + static_cast<size_t>(b) * C;
-        // largest |x| of the row, as bf16 magnitude bits (integer order = value order)
-        unsigned m = 0;
-        for (int i0 = 0; i0 < C / 8; i0 += 8 * 256) {
-            uint4 v[8];  // all loads of a round before their use
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const int i = i0 + threadIdx.x + 256 * k;
-                v[k] = i < C / 8 ? __ldg(reinterpret_cast<const uint4*>(xb) + i) : make_uint4(0, 0, 0, 0);
-            }
-#pragma unroll
-            for (int k = 0; k < 8; ++k) {
-                const unsigned w4[4] = {v[k].x, v[k].y, v[k].z, v[k].w};
-#pragma unroll
-                for (int e = 0; e < 4; ++e) m = max(m, max(w4[e] & 0x7FFFu, (w4[e] >> 16) & 0x7FFFu));
-            }
-        }
-        m = __reduce_max_sync(0xFFFFFFFFu, m);
-        if (lane == 0) s_red[warp] = m;
-        __syncthreads();
-        m = s_red[0];
-#pragma unroll
-        for (int k = 1; k < 8; ++k) m = max(m, s_red[k]);
-        // |xr_i| <= sqrt(B) max|x|: pick e with sqrt(B) max|x| 2^-e < 2^15
-        int e = 0;
-        if (m != 0 && m < 0x7F80u) {
-            const float bound = __uint_as_float(m << 16) * sqrtf(static_cast<float>(1 << G.logb)) * 1.0001f;
-            int k;
-            frexpf(bound, &k);
-            e = k - 15;
-            e = e < -126 ? -126 : (e > 126 ? 126 : e);
-        }
+        const int e = gv_row_exponent(xb, C, G.logb, s_red);
         const float down = __uint_as_float(static_cast<unsigned>(127 - e) << 23);  // 2^-e
         const int c0 = seg * G.seg_cols;
         const int n = min(G.seg_cols, C - c0);
-        for (int i = threadIdx.x; i < n; i += 256) {
-            const float v = __uint_as_float(static_cast<unsigned>(xb[c0 + i]) << 16);
-            buf[i] = p.signs[c0 + i] < 0 ? -v : v;
-        }
-        __syncthreads();
-        if (G.logb > 0) fwht_smem(buf, n, G.logb);
+        gv_rotate_segment(buf, xb, p.signs, c0, n, G.logb);
         const float inv = 1.0f / sqrtf(static_cast<float>(1 << G.logb));
         for (int t = threadIdx.x; t < n / 8; t += 256) {
             const int col = c0 + 8 * t;

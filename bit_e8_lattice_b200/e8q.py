@@ -87,6 +87,10 @@ def lib():
         L.e8q_gemv_workspace_bytes.restype = sz
         L.e8q_dequant_gemv.argtypes = [ctypes.POINTER(EncodedC), vp, i32, vp, vp, sz, vp]
         L.e8q_dequant_gemv.restype = ctypes.c_int
+        L.e8q_gemm_workspace_bytes.argtypes = [ctypes.POINTER(EncodedC), i32]
+        L.e8q_gemm_workspace_bytes.restype = sz
+        L.e8q_dequant_gemm.argtypes = [ctypes.POINTER(EncodedC), vp, i32, vp, vp, sz, vp]
+        L.e8q_dequant_gemm.restype = ctypes.c_int
         L.e8q_ste_backward.argtypes = [vp, vp, i64, vp]
         L.e8q_ste_backward.restype = ctypes.c_int
         _lib = L
@@ -375,3 +379,34 @@ class Gemv:
 
 def e8q_dequant_gemv(m: Encoded, x: torch.Tensor, stream=None) -> torch.Tensor:
     return Gemv(m, x.shape[0])(x, stream=stream).clone()
+
+
+class Gemm:
+    """Pre-allocated workspace and output for Y = X W~^T from the 2-bit form
+    (many activation rows; the fused tensor-core dequant-GEMM)."""
+
+    def __init__(self, m: Encoded, batch: int):
+        self.m, self.batch = m, int(batch)
+        self._mc = m.c()
+        ws = lib().e8q_gemm_workspace_bytes(ctypes.byref(self._mc), self.batch)
+        self.workspace = torch.empty(ws, dtype=torch.uint8, device=m.idx.device)
+        self.y = torch.empty((self.batch, m.rows), dtype=torch.bfloat16, device=m.idx.device)
+
+    def __call__(self, x: torch.Tensor, out: Optional[torch.Tensor] = None, stream=None) -> torch.Tensor:
+        _require_cuda(x, "x")
+        if x.dtype != torch.bfloat16 or tuple(x.shape) != (self.batch, self.m.cols):
+            raise E8qError(f"x must be bf16 [{self.batch}][{self.m.cols}]")
+        y = self.y if out is None else out
+        rc = lib().e8q_dequant_gemm(ctypes.byref(self._mc), _ptr(x), self.batch, _ptr(y),
+                                    ctypes.c_void_p(self.workspace.data_ptr()), self.workspace.numel(),
+                                    _stream_handle(stream))
+        _check(rc, "e8q_dequant_gemm")
+        return y
+
+    def error_word(self) -> int:
+        """The last call's error word (0: every bounded wait completed)."""
+        return int(self.workspace[:8].cpu().numpy().view(np.uint64)[0])
+
+
+def e8q_dequant_gemm(m: Encoded, x: torch.Tensor, stream=None) -> torch.Tensor:
+    return Gemm(m, x.shape[0])(x, stream=stream).clone()

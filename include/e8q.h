@@ -288,6 +288,47 @@ e8q_status e8q_dequant_gemv(const e8q_encoded* m /* host */, const void* x_bf16,
                             void* ws, size_t ws_bytes, e8q_stream stream);
 
 /*
+ * Workspace bytes e8q_dequant_gemm needs for this matrix and batch (exact;
+ * the same on every device; 256 for arguments the GEMM would reject).
+ * Needs no GPU.
+ */
+size_t e8q_gemm_workspace_bytes(const e8q_encoded* m /* host */, int32_t batch);
+
+/*
+ * Fused dequant-GEMM from the 2-bit form, for many activation rows at once
+ * (prefill and the QAT forward; E8-QAT, abstract: decoding throughput of the
+ * 2-bit representation).  The same product as e8q_dequant_gemv,
+ *   y[t][r] = sum_c w~[r][c] x[t][c] = s_r * sum_g < p_rg , (H_B (d (.) x_t) / sqrt(B))_g >,
+ * computed without writing the dequantised weights anywhere: the codewords
+ * are decoded from the indices into the tensor cores' shared-memory operand
+ * (tcgen05 MMA, fp32 accumulators in tensor memory).
+ * x: [batch][cols] bf16, 16-byte aligned; y: [batch][rows] bf16;
+ * 1 <= batch <= 65536 (the kernel is built for batch >= 64; smaller batches
+ * are correct but e8q_dequant_gemv is faster there); m->signs required;
+ * m->esc 8-byte aligned; m->ovf 4-byte aligned, ovf_count < 2^31.
+ * ws: device memory of at least e8q_gemm_workspace_bytes(m, batch) bytes,
+ * 256-byte aligned, owned by the caller, overwritten.  Its first 8 bytes are
+ * the call's error word: 0 after a correct call; nonzero (bit 0) if one of
+ * the kernel's bounded waits gave up, in which case y is not valid.
+ *
+ * Records: as for e8q_dequant_gemv (CSR row pointers, sorted by group within
+ * each row; malformed records give wrong values but no out-of-bounds access).
+ *
+ * Arithmetic: the rotated activations are formed in fp32 and rounded to fp16
+ * after a per-row power-of-two scaling chosen from the row's largest |x|
+ * (no overflow is possible); the integer coordinates are exact in fp16 up
+ * to |P_i| = 2048, and overflow points beyond that are multiplied on CUDA
+ * cores with the same fp16 activations; fp32 accumulation; bf16 output
+ * (round to nearest even).  Expected relative error about 1e-4 of the output
+ * norm.  The K split (and with it the order of the partial sums) depends on
+ * the shapes only, so repeated calls give the same bits on any device.
+ * Asynchronous on `stream`; errors: INVALID_ARG, UNSUPPORTED (cols > 16384,
+ * too many tiles or overflow records), WORKSPACE, CUDA.
+ */
+e8q_status e8q_dequant_gemm(const e8q_encoded* m /* host */, const void* x_bf16, int32_t batch, void* y_bf16,
+                            void* ws, size_t ws_bytes, e8q_stream stream);
+
+/*
  * Identity-STE backward (E8-QAT, Figure 2 (b): the projection is trained
  * with an identity straight-through estimator): the gradient of the loss
  * with respect to the latent weights equals its gradient with respect to the

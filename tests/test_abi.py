@@ -170,6 +170,36 @@ def test_gemv_workspace_holds_its_parts(lib):
     assert lib.e8q_gemv_workspace_bytes(ctypes.byref(m), 257) == 256
 
 
+def test_gemm_argument_checks_and_workspace(lib):
+    """The fused GEMM rejects bad batches, misaligned activations and short
+    workspaces before touching a device, and its workspace holds the fp16
+    activation image (whole 256-token tiles x 32-column K tiles), the row
+    map and the per-split cursor headers; the plan depends on the shapes
+    only, so the size is exact."""
+    from bit_e8_lattice_b200 import e8q
+
+    vp = ctypes.c_void_p
+    m = e8q.EncodedC(0x100000, 0x100000, 0x100000, None, None, None, None, 0, 0, 4096, 14336, 0, 0, 0)
+    for bad in (0, -1, 65537):
+        assert lib.e8q_gemm_workspace_bytes(ctypes.byref(m), bad) == 256
+        assert lib.e8q_dequant_gemm(ctypes.byref(m), vp(0x100000), bad, vp(0x100000), vp(0x100000), 1 << 40,
+                                    None) == 1
+    for batch in (64, 256, 1000, 4096):
+        need = lib.e8q_gemm_workspace_bytes(ctypes.byref(m), batch)
+        tiles = (batch + 255) // 256
+        assert need % 256 == 0
+        assert need >= tiles * 256 * 14336 * 2 + 4096 * 14336 // 8 + 4096 * 32
+        assert need == lib.e8q_gemm_workspace_bytes(ctypes.byref(m), batch)
+        assert lib.e8q_dequant_gemm(ctypes.byref(m), vp(0x100008), batch, vp(0x100000), vp(0x100000), need,
+                                    None) == 1  # x not 16-byte aligned
+        assert lib.e8q_dequant_gemm(ctypes.byref(m), vp(0x100000), batch, vp(0x100000), vp(0x100000), need - 1,
+                                    None) == 4
+        assert lib.e8q_dequant_gemm(ctypes.byref(m), vp(0x100000), batch, vp(0x100000), vp(0x100080), need,
+                                    None) == 4  # workspace not 256-byte aligned
+    m.cols = 12
+    assert lib.e8q_gemm_workspace_bytes(ctypes.byref(m), 64) == 256  # cols % 8
+
+
 def test_escape_table_matches_oracle(lib):
     """Every E8 point with |p|^2 <= 22 (1,113,841 points), plus a shell
     beyond: the kernels' lookup table gives the oracle's encoding (core
@@ -213,3 +243,10 @@ def test_bench_source_hash_ignores_comments_only(tmp_path, monkeypatch):
     assert bench.source_sha() == base
     f.write_text(f.read_text() + "\nnamespace e8q { constexpr int kProbe = 1; }\n")
     assert bench.source_sha() != base
+    # a kernel's own hash follows only the files it is built from
+    enc = bench.source_sha("k_encode_fast")
+    g = dst / "gemm_tc.cuh"
+    g.write_text(g.read_text() + "\nnamespace e8q { constexpr int kProbe2 = 2; }\n")
+    assert bench.source_sha("k_encode_fast") == enc and bench.source_sha() != base
+    f.write_text(f.read_text() + "\nnamespace e8q { constexpr int kProbe3 = 3; }\n")
+    assert bench.source_sha("k_encode_fast") != enc

@@ -459,6 +459,104 @@ def test_gemv_far_overflow_points(e8q):
 
 
 # ----------------------------------------------------------------------
+# fused dequant-GEMM (tensor cores, many activation rows)
+# ----------------------------------------------------------------------
+def run_gemm(e8q, m, xb):
+    g = e8q.Gemm(m, xb.shape[0])
+    y = g(dev_bf16(xb))
+    torch.cuda.synchronize()
+    assert g.error_word() == 0, "a bounded wait of the GEMM gave up"
+    return y.cpu().view(torch.int16).numpy()
+
+
+@pytest.mark.parametrize("rows,cols,batch,kappa", [
+    (256, 2048, 64, 1.0),     # two row tiles, one token tile of 64, K splits
+    (300, 1536, 100, 2.5),    # many escapes and overflow records, ragged rows and tokens
+    (129, 264, 257, 1.0),     # last K tile past the row end (33 groups), block 8, a second token tile of 1
+    (37, 4096, 512, 1.0),     # one partial row tile, two full token tiles, many K splits (finalize)
+    (1000, 256, 300, 1.0),    # eight row tiles, no K split (direct epilogue), ragged second token tile
+    (64, 8, 70, 1.0),         # one group per row: three zero groups in the only K tile
+    (513, 4096, 1024, 1.0),   # five row tiles, four token tiles
+])
+def test_gemm_matches_oracle(e8q, rows, cols, batch, kappa):
+    rng = np.random.default_rng(rows * 11 + cols + batch)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((rows, cols)) * 0.02)
+    d = synth.signs(rows + 5, cols)
+    B = oracle.default_block(cols)
+    enc, res = run_encode(e8q, [w], [d], 0, kappa=kappa)
+    st = compare_all(e8q, res, [w], [d], [B], kappa=kappa, label="gemm_shape")[0]
+    if kappa > 2:
+        ctr = res.read_counters()
+        assert ctr["n_escape"] > rows and ctr["n_overflow"] > rows, ctr
+    xb = synth.gemv_x(batch, cols)
+    y = run_gemm(e8q, res.encoded[0], xb)
+    y_ref = oracle.gemv(st["points"], res.scale[0].cpu().numpy().astype(np.float64), d, B,
+                        synth.bf16_bits_to_f64(xb))
+    check_gemv(y, y_ref, f"gemm {rows}x{cols} b={batch}")
+
+
+@pytest.mark.parametrize("rows,cols", [(160, 1024), (2048, 256)])
+def test_gemm_far_overflow_points(e8q, rows, cols):
+    """kappa 1000 (s = rms / 1000): every group an overflow record, most with
+    doubled coordinates beyond fp16's exact integers (+-2048), which the GEMM
+    adds on CUDA cores -- in the finalize (K splits, 160 x 1024) and in the
+    epilogue (one split, 2048 x 256) -- while the rest go through the tensor
+    cores."""
+    rng = np.random.default_rng(rows + cols)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((rows, cols)) * 0.02)
+    d = synth.signs(rows, cols)
+    B = oracle.default_block(cols)
+    n = rows * cols // 8
+    enc, res = run_encode(e8q, [w], [d], 0, kappa=1000.0, esc_cap=n, ovf_cap=n)
+    assert res.read_counters()["n_clamped"] == 0
+    # the GEMM's reference is the product with the points it was given (at
+    # this scale the fp32 projection's near ties are not the fp64 oracle's)
+    idx = host_idx(res.idx[0]).reshape(-1)
+    P, _, _, _, _ = gpu_points(idx, res.escape_records(), res.overflow_records(), idx.size, 0)
+    far_groups = (np.abs(P) > 2048).any(axis=1).sum()
+    assert far_groups > 100 and (np.abs(P) <= 2048).all(axis=1).sum() > 100, far_groups
+    for batch in (70, 300):
+        xb = synth.gemv_x(batch, cols)
+        y = run_gemm(e8q, res.encoded[0], xb)
+        y_ref = oracle.gemv(P, res.scale[0].cpu().numpy().astype(np.float64), d, B, synth.bf16_bits_to_f64(xb))
+        check_gemv(y, y_ref, f"gemm far points {rows}x{cols} b={batch}")
+
+
+def test_gemm_large_activations_and_repeatable(e8q):
+    """Activation rows near the bf16 range limit stay finite (per-row
+    power-of-two scaling), and two calls give the same bits."""
+    rng = np.random.default_rng(12)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((200, 2048)) * 0.02)
+    d = synth.signs(4, 2048)
+    enc, res = run_encode(e8q, [w], [d], 0)
+    st = compare_all(e8q, res, [w], [d], [2048], label="gemm_big_x")[0]
+    x = rng.standard_normal((96, 2048))
+    x[0] *= 1e30
+    x[1] *= 1e-30
+    xb = synth.f64_to_bf16_bits(x)
+    y = run_gemm(e8q, res.encoded[0], xb)
+    y_ref = oracle.gemv(st["points"], res.scale[0].cpu().numpy().astype(np.float64), d, 2048,
+                        synth.bf16_bits_to_f64(xb))
+    assert np.isfinite(synth.bf16_bits_to_f64(y.view(np.uint16))).all()
+    check_gemv(y, y_ref, "gemm big x")
+    assert (run_gemm(e8q, res.encoded[0], xb) == y).all()
+
+
+def test_gemm_equals_gemv_up_to_rounding(e8q):
+    """At batch 64 both routes compute the same product; their outputs differ
+    by at most the bf16 rounding of each plus the fp16 activation rounding."""
+    rng = np.random.default_rng(13)
+    w = synth.f64_to_bf16_bits(rng.standard_normal((384, 2048)) * 0.02)
+    d = synth.signs(13, 2048)
+    enc, res = run_encode(e8q, [w], [d], 0, kappa=2.0)
+    xb = synth.gemv_x(64, 2048)
+    a = synth.bf16_bits_to_f64(run_gemm(e8q, res.encoded[0], xb).view(np.uint16))
+    b = synth.bf16_bits_to_f64(e8q.Gemv(res.encoded[0], 64)(dev_bf16(xb)).cpu().view(torch.int16).numpy().view(np.uint16))
+    rel = np.linalg.norm(a - b) / np.linalg.norm(b)
+    assert rel < 5e-3, rel
+
+
+# ----------------------------------------------------------------------
 # full-size workloads, in the launch configuration bench.py times
 # ----------------------------------------------------------------------
 @pytest.fixture(scope="module")
@@ -564,6 +662,21 @@ def test_gemv_full_size(e8q, mlp_full, batch):
     y_ref = oracle.gemv(P, res.scale[0].cpu().numpy().astype(np.float64), mlp_full["d_up"], 2048,
                         synth.bf16_bits_to_f64(xb))
     check_gemv(y.cpu().view(torch.int16).numpy(), y_ref, f"gemv full b={batch}")
+
+
+@pytest.mark.parametrize("batch", [256, 1024])
+def test_gemm_full_size(e8q, mlp_full, batch):
+    """The fused GEMM on the encoded up matrix at the benchmark's token
+    counts, every output against the oracle."""
+    res = mlp_full["res"]
+    m = res.encoded[0]
+    idx = host_idx(res.idx[0]).reshape(-1)
+    P, _, _, _, _ = gpu_points(idx, res.escape_records(), res.overflow_records(), idx.size, 0)
+    xb = synth.gemv_x(batch, 14336)
+    y = run_gemm(e8q, m, xb)
+    y_ref = oracle.gemv(P, res.scale[0].cpu().numpy().astype(np.float64), mlp_full["d_up"], 2048,
+                        synth.bf16_bits_to_f64(xb))
+    check_gemv(y, y_ref, f"gemm full b={batch}")
 
 
 def test_moe_bank_full_size_sampled(e8q):
