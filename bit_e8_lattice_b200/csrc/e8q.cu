@@ -98,6 +98,8 @@ e8q_status ensure_device(int* dev_out) {
             st = cuda_ok(cudaFuncSetAttribute(k_gm_main, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                               static_cast<int>(kGmSmemBytes)));
         if (st == E8Q_OK)
+            st = cuda_ok(cudaFuncSetAttribute(k_gm_prep, cudaFuncAttributeMaxDynamicSharedMemorySize, kMaxCols * 4));
+        if (st == E8Q_OK)
             st = cuda_ok(cudaFuncSetAttribute(k_gm_prep, cudaFuncAttributePreferredSharedMemoryCarveout,
                                               cudaSharedmemCarveoutMaxShared));
         if (st == E8Q_OK)
@@ -576,7 +578,7 @@ e8q_status e8q_dequant_gemm(const e8q_encoded* m, const void* x_bf16, int32_t ba
     pp.g = g;
     pp.n_xcta = (batch + 15) / 16 * 16;
     const int n_rcta = (g.rows + 7) / 8;
-    k_gm_prep<<<pp.n_xcta + n_rcta, 256, 0, s>>>(pp);
+    k_gm_prep<<<pp.n_xcta + n_rcta, 256, static_cast<size_t>(g.cols) * 4, s>>>(pp);
     st = cuda_ok(cudaGetLastError());
     if (st != E8Q_OK) return st;
 

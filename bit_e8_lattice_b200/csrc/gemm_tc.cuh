@@ -10,9 +10,10 @@
 // 16-bit indices straight into the tensor cores' shared-memory operand.
 //
 // Launches:
-//  k_gm_prep  (a) per token row (all its 2048-column segments in turn):
-//             xr * 2^-e in fp16, e chosen from the row's largest |x| (no
-//             fp16 overflow), stored as an operand image: per (256-token
+//  k_gm_prep  (a) per token row (the whole row in shared memory, one pass
+//             of the blockwise transform): xr * 2^-e in fp16, e chosen from
+//             the row's largest |x| (no fp16 overflow), stored as an
+//             operand image: per (256-token
 //             tile, 32-column K tile) one contiguous 16 KB block in the
 //             K-major, no-swizzle core-matrix layout, so that one 1-D bulk
 //             copy stages it;
@@ -233,7 +234,7 @@ struct GmPrepParams {
 };
 
 __global__ void __launch_bounds__(256) k_gm_prep(const __grid_constant__ GmPrepParams p) {
-    __shared__ __align__(16) float buf[kGvSegCols];
+    extern __shared__ __align__(16) float xs[];  // one token row (cols floats)
     __shared__ unsigned s_red[8];
     pdl_launch_dependents();
     const GmGeom& G = p.g;
@@ -247,24 +248,46 @@ __global__ void __launch_bounds__(256) k_gm_prep(const __grid_constant__ GmPrepP
                 *reinterpret_cast<uint4*>(p.img + gm_img_off(G, t, i)) = make_uint4(0, 0, 0, 0);
             return;
         }
-        const uint16_t* xb = p.x + static_cast<size_t>(t) * G.cols;
-        const int e = gv_row_exponent(xb, G.cols, G.logb, s_red);
-        const float f = __uint_as_float(static_cast<unsigned>(127 - e) << 23) / sqrtf(static_cast<float>(1 << G.logb));
-        for (int seg = 0; seg < G.nseg; ++seg) {
-            const int c0 = seg * G.seg_cols;
-            const int n = min(G.seg_cols, G.cols - c0);
-            __syncthreads();  // the previous segment's reads of buf are done
-            gv_rotate_segment(buf, xb, p.signs, c0, n, G.logb);
-            const int pad = seg == G.nseg - 1 ? gpad : 0;
-            for (int i = threadIdx.x; i < n / 8 + pad; i += 256) {
-                uint4 o = make_uint4(0, 0, 0, 0);
-                if (i < n / 8) {
-                    const float* v = buf + 8 * i;
-                    o = make_uint4(pack_half2(v[0] * f, v[1] * f), pack_half2(v[2] * f, v[3] * f),
-                                   pack_half2(v[4] * f, v[5] * f), pack_half2(v[6] * f, v[7] * f));
-                }
-                *reinterpret_cast<uint4*>(p.img + gm_img_off(G, t, c0 / 8 + i)) = o;
+        // the row, sign-flipped, into shared memory, and its largest |x| as
+        // bf16 magnitude bits (integer order = value order)
+        const uint4* xb = reinterpret_cast<const uint4*>(p.x + static_cast<size_t>(t) * G.cols);
+        unsigned m = 0;
+        for (int i = threadIdx.x; i < G.gpr; i += 256) {
+            const uint4 v = __ldg(xb + i);
+            const unsigned w4[4] = {v.x, v.y, v.z, v.w};
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+                const unsigned h = (w4[e >> 1] >> (16 * (e & 1))) & 0xFFFFu;
+                m = max(m, h & 0x7FFFu);
+                const float f = __uint_as_float(h << 16);
+                xs[8 * i + e] = __ldg(p.signs + 8 * i + e) < 0 ? -f : f;
             }
+        }
+        m = __reduce_max_sync(0xFFFFFFFFu, m);
+        if (lane == 0) s_red[warp] = m;
+        __syncthreads();
+        m = s_red[0];
+#pragma unroll
+        for (int k = 1; k < 8; ++k) m = max(m, s_red[k]);
+        // |xr_i| <= sqrt(B) max|x|: pick e with sqrt(B) max|x| 2^-e < 2^15
+        int e = 0;
+        if (m != 0 && m < 0x7F80u) {
+            const float bound = __uint_as_float(m << 16) * sqrtf(static_cast<float>(1 << G.logb)) * 1.0001f;
+            int k;
+            frexpf(bound, &k);
+            e = k - 15;
+            e = e < -126 ? -126 : (e > 126 ? 126 : e);
+        }
+        if (G.logb > 0) fwht_smem(xs, G.cols, G.logb);  // every block of the row at once
+        const float f = __uint_as_float(static_cast<unsigned>(127 - e) << 23) / sqrtf(static_cast<float>(1 << G.logb));
+        for (int i = threadIdx.x; i < G.gpr + gpad; i += 256) {
+            uint4 o = make_uint4(0, 0, 0, 0);
+            if (i < G.gpr) {
+                const float* v = xs + 8 * i;
+                o = make_uint4(pack_half2(v[0] * f, v[1] * f), pack_half2(v[2] * f, v[3] * f),
+                               pack_half2(v[4] * f, v[5] * f), pack_half2(v[6] * f, v[7] * f));
+            }
+            *reinterpret_cast<uint4*>(p.img + gm_img_off(G, t, i)) = o;
         }
         if (threadIdx.x == 0) p.xe[t] = __uint_as_float(static_cast<unsigned>(127 + e) << 23);
         return;
@@ -279,11 +302,20 @@ __global__ void __launch_bounds__(256) k_gm_prep(const __grid_constant__ GmPrepP
     if (p.esc_rp) {
         const long long e0 = gv_clamp(p.esc_rp[r], 0, p.esc_n);
         const long long e1 = gv_clamp(p.esc_rp[r + 1], e0, p.esc_n);
-        for (long long k = e0 + lane; k < e1; k += 32) {
-            const uint2 rec = __ldcs(reinterpret_cast<const uint2*>(p.esc + k));
-            const long long gl = static_cast<long long>(rec.x) - g0;
-            const unsigned root = (rec.y >> 16) & 0xFFu;
-            if (gl >= 0 && gl < G.gpr && root < 240) mrow[gl] = static_cast<uint16_t>(root + 1);
+        // records in rounds of 8 per lane: all loads of a round before its stores
+        for (long long k0 = e0; k0 < e1; k0 += 8 * 32) {
+            uint2 rec[8];
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const long long k = k0 + lane + 32 * i;
+                rec[i] = k < e1 ? __ldcs(reinterpret_cast<const uint2*>(p.esc + k)) : make_uint2(0u, 0xFF0000u);
+            }
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+                const long long gl = static_cast<long long>(rec[i].x) - g0;
+                const unsigned root = (rec[i].y >> 16) & 0xFFu;  // 255: no record
+                if (gl >= 0 && gl < G.gpr && root < 240) mrow[gl] = static_cast<uint16_t>(root + 1);
+            }
         }
     }
     bool far = false;
@@ -291,14 +323,25 @@ __global__ void __launch_bounds__(256) k_gm_prep(const __grid_constant__ GmPrepP
         const long long o0 = gv_clamp(p.ovf_rp[r], 0, p.ovf_n);
         const long long o1 = gv_clamp(p.ovf_rp[r + 1], o0, p.ovf_n);
         __syncwarp();  // escape entries first: a group listed twice ends as an overflow
-        for (long long k = o0 + lane; k < o1 && k - o0 < 0x8000; k += 32) {
-            uint32_t grp;
-            uint4 c;
-            gm_load_rec(p.ovf, k, grp, c);
-            const long long gl = static_cast<long long>(grp) - g0;
-            if (gl >= 0 && gl < G.gpr) {
-                mrow[gl] = static_cast<uint16_t>(0x8000u | static_cast<unsigned>(k - o0));
-                far |= gm_far(c);
+        const long long o1c = o1 - o0 < 0x8000 ? o1 : o0 + 0x8000;  // offsets fit 15 bits
+        for (long long k0 = o0; k0 < o1c; k0 += 4 * 32) {
+            uint32_t grp[4];
+            uint4 c[4];
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const long long k = k0 + lane + 32 * i;
+                grp[i] = 0xFFFFFFFFu;
+                c[i] = make_uint4(0, 0, 0, 0);
+                if (k < o1c) gm_load_rec(p.ovf, k, grp[i], c[i]);
+            }
+#pragma unroll
+            for (int i = 0; i < 4; ++i) {
+                const long long k = k0 + lane + 32 * i;
+                const long long gl = static_cast<long long>(grp[i]) - g0;
+                if (k < o1c && gl >= 0 && gl < G.gpr) {
+                    mrow[gl] = static_cast<uint16_t>(0x8000u | static_cast<unsigned>(k - o0));
+                    far |= gm_far(c[i]);
+                }
             }
         }
     }
