@@ -50,7 +50,8 @@
  * without waiting.  The return code covers argument checks and launch
  * errors only; conditions found in the data (escape counts, capacity
  * shortfall, non-finite inputs, a wait that gave up) are written to the
- * device-side e8q_counters, which the caller reads after synchronising.
+ * device-side e8q_counters (for e8q_dequant_gemm: the first word of its
+ * workspace), which the caller reads after synchronising.
  */
 #ifndef E8Q_H
 #define E8Q_H
@@ -303,8 +304,8 @@ size_t e8q_gemm_workspace_bytes(const e8q_encoded* m /* host */, int32_t batch);
  * are decoded from the indices into the tensor cores' shared-memory operand
  * (tcgen05 MMA, fp32 accumulators in tensor memory).
  * x: [batch][cols] bf16, 16-byte aligned; y: [batch][rows] bf16;
- * 1 <= batch <= 65536 (the kernel is built for batch >= 64; smaller batches
- * are correct but e8q_dequant_gemv is faster there); m->signs required;
+ * 1 <= batch <= 65536 (any batch is correct; on a 4096 x 14336 matrix
+ * e8q_dequant_gemv is faster at 64 rows and this call at 256); m->signs required;
  * m->esc 8-byte aligned; m->ovf 4-byte aligned, ovf_count < 2^31.
  * ws: device memory of at least e8q_gemm_workspace_bytes(m, batch) bytes,
  * 256-byte aligned, owned by the caller, overwritten.  Its first 8 bytes are
