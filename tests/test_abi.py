@@ -200,6 +200,34 @@ def test_gemm_argument_checks_and_workspace(lib):
     assert lib.e8q_gemm_workspace_bytes(ctypes.byref(m), 64) == 256  # cols % 8
 
 
+def test_gemm_plan_splits_k_where_tiles_are_few(lib):
+    """The GEMM's K split (read off its exact workspace: fp32 partial sums
+    exist only with several splits): a 4096-row matrix at 64 activation rows
+    has 32 row tiles for 148 SMs and is split; a 14336-row matrix at 4096
+    rows has 1,792 units and is not."""
+    from bit_e8_lattice_b200 import e8q
+
+    def rnd(x):
+        return (x + 255) // 256 * 256
+
+    def unsplit(rows, cols, batch):
+        nkt = (cols + 31) // 32
+        ntt = (batch + 255) // 256
+        mstride = (4 * nkt + 7) // 8 * 8
+        return 256 + rnd(ntt * nkt * 16384) + rnd(ntt * 256 * 4) + rnd(rows * mstride * 2) + rnd(rows)
+
+    for rows, cols, batch, split in ((4096, 14336, 64, True), (4096, 14336, 256, True),
+                                     (14336, 4096, 4096, False), (14336, 4096, 64, False)):
+        m = e8q.EncodedC(0x100000, 0x100000, 0x100000, None, None, None, None, 0, 0, rows, cols, 0, 0, 0)
+        need = lib.e8q_gemm_workspace_bytes(ctypes.byref(m), batch)
+        base = unsplit(rows, cols, batch)
+        if split:
+            parts = (need - base) // (batch * rows * 4)
+            assert need > base and 2 <= parts <= 32, (rows, cols, batch, need, base)
+        else:
+            assert need == base, (rows, cols, batch, need, base)
+
+
 def test_escape_table_matches_oracle(lib):
     """Every E8 point with |p|^2 <= 22 (1,113,841 points), plus a shell
     beyond: the kernels' lookup table gives the oracle's encoding (core
