@@ -16,7 +16,10 @@ value = groups encoded per second over whole steps (Ggroups/s, all ranks).
 The step's inputs are larger than L2 (235 MB read per step), so the step
 needs no flush.  The per-kernel GEMV, decode and small-workload figures in
 "kernels" are medians of 20 calls, each after a 256 MB write that flushes
-L2.
+L2.  So are the fused dequant-GEMM entries (e8q_dequant_gemm of the up
+matrix at 64..4096 activation rows, with the unfused route -- decode to
+bf16, then a cuBLAS GEMM -- timed beside each); the GEMM is not part of the
+step.
 
 --impl reference runs the fp64 CPU oracle on a bounded sample of the same
 step on the host cores (rank 0 only).
