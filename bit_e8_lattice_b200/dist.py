@@ -143,8 +143,9 @@ def gather_encoded(idx, scale, esc, n_esc: int, ovf, n_ovf: int, esc_row_ptr, ov
 
 
 def gemv_rows_allgather(y_local, group=None):
-    """Row-split dequant-GEMV, exchange step: every rank computed
-    y_local = W_r x for its own row shard W_r (bf16 [batch][rows_r]); one
+    """Row-split dequant-GEMV or -GEMM, exchange step: every rank computed
+    y_local = W_r x for its own row shard W_r (bf16 [batch][rows_r], from
+    e8q_dequant_gemv or e8q_dequant_gemm: both write that layout); one
     all_gather (padded to the largest shard) gives every rank the whole
     y = W x, [batch][sum of rows_r] in rank order."""
     import torch
